@@ -173,13 +173,14 @@ def rotate_quant(X, xdtype, g, d=None, return_u=False):
 
 
 def w4_pack(W, wdtype, gw):
-    """(Wq, sw, zw): per-channel symmetric (gw = 0) or group asymmetric int4."""
+    """(Wq, sw, zw): per-channel symmetric (gw = 0; sw [N]) or group asymmetric
+    int4 (sw, zw group-major [K/gw, N])."""
     W = _raw(W, wdtype)
     N, K = W.shape
     Wq = _np.empty((N, K // 2), _np.uint8)
     G = K // gw if gw else 1
-    sw = _np.empty((N, G) if gw else (N,), _np.uint16)
-    zw = _np.empty((N, G), _np.uint16) if gw else None
+    sw = _np.empty((G, N) if gw else (N,), _np.uint16)   # group-major [K/gw][N]
+    zw = _np.empty((G, N), _np.uint16) if gw else None
     _lib.hqo_w4_pack(_ptr(W), _DT[wdtype], N, K, gw, _ptr(Wq), _ptr(sw), _ptr(zw))
     return Wq, sw.view(_np.float16), (zw.view(_np.float16) if gw else None)
 

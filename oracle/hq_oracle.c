@@ -267,7 +267,7 @@ void hqo_rotate_quant(const void* X, int dtype, int64_t M, int64_t K, int32_t g,
  *   spanning [min(mn,0), max(mx,0)]: s16 = fl16(fl32(fl32(hi - lo) / 15)), 1
  *   if that is zero; z = clamp(rint(fl32(-lo / s16)), 0, 15);
  *   q = clamp(rint(fl32(w / s16)) + z, 0, 15), unsigned nibbles;
- *   sw[n][b] = s16, zw[n][b] = fl16(z) (exact).
+ *   sw[b][n] = s16, zw[b][n] = fl16(z) (exact): group-major [K/gw][N].
  * The stored (rounded) scale is the one used to form the codes. */
 void hqo_w4_pack(const void* W, int dtype, int64_t N, int64_t K, int32_t gw,
                  uint8_t* Wq, uint16_t* sw, uint16_t* zw)
@@ -300,8 +300,8 @@ void hqo_w4_pack(const void* W, int dtype, int64_t N, int64_t K, int32_t gw,
                 if (hqo_f16_to_f32(s16) == 0.0f) s16 = 0x3C00u; /* 1.0 */
                 float s = hqo_f16_to_f32(s16);
                 float z = clampf(rintf(-lo / s), 0.0f, 15.0f);
-                sw[n * G + b] = s16;
-                zw[n * G + b] = hqo_f32_to_f16(z);
+                sw[b * N + n] = s16;
+                zw[b * N + n] = hqo_f32_to_f16(z);
                 for (int64_t k = b * gw; k < (b + 1) * gw; ++k) {
                     float w = load_elem(W, dtype, n * K + k);
                     int q = (int)clampf(rintf(w / s) + z, 0.0f, 15.0f);
@@ -314,20 +314,20 @@ void hqo_w4_pack(const void* W, int dtype, int64_t N, int64_t K, int32_t gw,
 
 /* Dequantised weight value of element (n, k), exact in fp32. */
 static float w_dequant(const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw,
-                       int64_t K, int32_t gw, int64_t n, int64_t k)
+                       int64_t N, int64_t K, int32_t gw, int64_t n, int64_t k)
 {
     const uint8_t* row = Wq + n * (K / 2);
     if (gw == 0) return (float)get_nibble_s(row, k) * hqo_f16_to_f32(sw[n]);
-    int64_t G = K / gw, b = k / gw;
-    float z = hqo_f16_to_f32(zw[n * G + b]);
-    return ((float)get_nibble_u(row, k) - z) * hqo_f16_to_f32(sw[n * G + b]);
+    int64_t b = k / gw;
+    float z = hqo_f16_to_f32(zw[b * N + n]);
+    return ((float)get_nibble_u(row, k) - z) * hqo_f16_to_f32(sw[b * N + n]);
 }
 
 void hqo_w4_dequant(const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw,
                     int64_t N, int64_t K, int32_t gw, float* What)
 {
     for (int64_t n = 0; n < N; ++n)
-        for (int64_t k = 0; k < K; ++k) What[n * K + k] = w_dequant(Wq, sw, zw, K, gw, n, k);
+        for (int64_t k = 0; k < K; ++k) What[n * K + k] = w_dequant(Wq, sw, zw, N, K, gw, n, k);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -350,7 +350,7 @@ void hqo_serq_prepare(const float* Wrot, int64_t N, int64_t K, const uint8_t* Wq
         float amax = 0.0f;
         for (int32_t j = 0; j < r; ++j) {
             int64_t k = sal[j];
-            e[j] = Wrot[n * K + k] - w_dequant(Wq, sw, zw, K, gw, n, k);
+            e[j] = Wrot[n * K + k] - w_dequant(Wq, sw, zw, N, K, gw, n, k);
             amax = fmaxf(amax, fabsf(e[j]));
             if (e_out) e_out[n * r + j] = e[j];
         }
@@ -369,7 +369,7 @@ void hqo_serq_prepare(const float* Wrot, int64_t N, int64_t K, const uint8_t* Wq
 /* Integer GEMM and epilogue [SERQ s2.2, s3; WaterSIC s1: Y = W X].          */
 /* ------------------------------------------------------------------------ */
 
-/* acc[m][n][b] = sum_{k in group b} qx[m][k] * (qw[n][k] - z[n][b]) in int64
+/* acc[m][n][b] = sum_{k in group b} qx[m][k] * (qw[n][k] - z[b][n]) in int64
  * (one group when gw == 0, with symmetric weight codes), and
  * acc_c[m][n] = sum_{j<r} qx[m][S_j] * qr[n][j].  Plain triple loop.
  * Returns 0, or 1 if any value does not fit in int32. */
@@ -388,7 +388,7 @@ int hqo_accum(const uint8_t* Xq, int64_t M, int64_t K, const uint8_t* Wq, const 
             const uint8_t* wrow = Wq + n * (K / 2);
             for (int64_t b = 0; b < G; ++b) {
                 int64_t s = 0;
-                int z = gw ? (int)hqo_f16_to_f32(zw[n * G + b]) : 0;
+                int z = gw ? (int)hqo_f16_to_f32(zw[b * N + n]) : 0;
                 for (int64_t k = b * glen; k < (b + 1) * glen; ++k) {
                     int wv = gw ? get_nibble_u(wrow, k) - z : get_nibble_s(wrow, k);
                     s += (int64_t)get_nibble_s(xrow, k) * wv;
@@ -405,7 +405,7 @@ int hqo_accum(const uint8_t* Xq, int64_t M, int64_t K, const uint8_t* Wq, const 
     return overflow;
 }
 
-/* y64[m][n] = sx[m] * (sum_b sw[n][b] * acc[m][n][b] + sr[n] * acc_c[m][n]),
+/* y64[m][n] = sx[m] * (sum_b sw[b][n] * acc[m][n][b] + sr[n] * acc_c[m][n]),
  * evaluated in fp64 from the exact integers: the ground truth of the
  * dequantising epilogue.  sr / acc_c may be NULL (no correction). */
 void hqo_epilogue_f64(const int64_t* acc, const int64_t* acc_c, int64_t M, int64_t N, int64_t G,
@@ -416,7 +416,7 @@ void hqo_epilogue_f64(const int64_t* acc, const int64_t* acc_c, int64_t M, int64
         for (int64_t n = 0; n < N; ++n) {
             double t = 0.0;
             for (int64_t b = 0; b < G; ++b)
-                t += (double)hqo_f16_to_f32(sw[n * G + b]) * (double)acc[(m * N + n) * G + b];
+                t += (double)hqo_f16_to_f32(sw[b * N + n]) * (double)acc[(m * N + n) * G + b];
             if (acc_c && sr) t += (double)hqo_f16_to_f32(sr[n]) * (double)acc_c[m * N + n];
             y[m * N + n] = (double)sx[m] * t;
         }
@@ -440,12 +440,12 @@ void hqo_linear_rows_f64(const uint8_t* Xq, const float* sx, int64_t K, const ui
             double t = 0.0;
             for (int64_t b = 0; b < G; ++b) {
                 int64_t s = 0;
-                int z = gw ? (int)hqo_f16_to_f32(zw[n * G + b]) : 0;
+                int z = gw ? (int)hqo_f16_to_f32(zw[b * N + n]) : 0;
                 for (int64_t k = b * glen; k < (b + 1) * glen; ++k) {
                     int wv = gw ? get_nibble_u(wrow, k) - z : get_nibble_s(wrow, k);
                     s += (int64_t)get_nibble_s(xrow, k) * wv;
                 }
-                t += (double)hqo_f16_to_f32(sw[n * G + b]) * (double)s;
+                t += (double)hqo_f16_to_f32(sw[b * N + n]) * (double)s;
             }
             if (r > 0) {
                 int64_t c = 0;

@@ -247,12 +247,12 @@ def test_w4_pack_group_asymmetric_round_trip():
     W[4, gw:2 * gw] = 0.0                             # an all-zero group
     Wq, sw, zw = O.w4_pack(W, "f32", gw)
     G = K // gw
-    assert sw.shape == (32, G) and zw.shape == (32, G)
+    assert sw.shape == (G, 32) and zw.shape == (G, 32)
     z = zw.astype(np.float64)
     assert np.all(z == np.round(z)) and np.all((z >= 0) & (z <= 15))
     q = O.unpack_u4(Wq, K).astype(np.float64)
-    s = np.repeat(sw.astype(np.float64), gw, axis=1)
-    zz = np.repeat(z, gw, axis=1)
+    s = np.repeat(sw.astype(np.float64).T, gw, axis=1)
+    zz = np.repeat(z.T, gw, axis=1)
     err = np.abs(W - (q - zz) * s)
     # half a step, plus the fp16 rounding of the step over a 15-step span
     assert np.all(err <= s * (0.5 + 15 * 2 ** -11 / (1 - 2 ** -11)) * (1 + 2 ** -20))
@@ -261,7 +261,7 @@ def test_w4_pack_group_asymmetric_round_trip():
     hi = np.maximum(Wg.max(axis=2), 0)
     span = (hi - lo).astype(np.float32) / np.float32(15)
     expect = np.where(span.astype(np.float16) == 0, np.float16(1), span.astype(np.float16))
-    assert np.array_equal(sw, expect)
+    assert np.array_equal(sw, expect.T)
     assert np.all(err[4, gw:2 * gw] == 0)
 
 
@@ -330,8 +330,8 @@ def test_accum_brute_force_matches_numpy_matmul(gw):
         qw = rng.integers(0, 16, (N, K)).astype(np.int8)
         Wq = O.pack_s4(qw)  # the nibble bits are what matter; read back unsigned
         qw_u = O.unpack_u4(Wq, K).astype(np.int64)
-        z = rng.integers(0, 16, (N, K // gw)).astype(np.float16)
-        wv = qw_u - np.repeat(z.astype(np.int64), gw, axis=1)
+        z = rng.integers(0, 16, (K // gw, N)).astype(np.float16)
+        wv = qw_u - np.repeat(z.astype(np.int64).T, gw, axis=1)
     else:
         qw = rng.integers(-8, 8, (N, K)).astype(np.int8)
         Wq = O.pack_s4(qw)
