@@ -1,0 +1,234 @@
+/*
+ * hq.h -- C ABI of libhq, a B200 (sm_100a) implementation of the W4A4 rotated
+ * linear layer: an online grouped Walsh-Hadamard rotation of the activations
+ * with per-token symmetric int4 quantisation, packed int4 x int4 GEMM on the
+ * tcgen05 tensor cores with int32 accumulation, a per-token x per-channel (or
+ * per-group) dequantising epilogue, and SERQ's single rank-r error term on the
+ * salient input channels fused into the same launch.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Y[M,N] = X[M,K] * W[N,K]^T (PyTorch Linear layout; the pages write Y = W X,
+ *    "WaterSIC", technical summary section 1).
+ *  - Pointers named "device" are CUDA device pointers owned by the caller; the
+ *    library never frees or keeps them.  Pointers named "host" are host memory.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every device
+ *    call only enqueues work on that stream and returns; results are valid
+ *    after the stream has been synchronised.  Argument errors are detected on
+ *    the host before anything is launched and leave all outputs untouched.
+ *  - No call prints, aborts or traps.  Errors are reported by the return code;
+ *    a device-side wait that exceeds its time limit records HQ_ERR_TIMEOUT,
+ *    read back with hq_last_device_status().
+ *  - Packed int4: element 2j is the low nibble of byte j, 2j+1 the high nibble.
+ *    Activation codes and symmetric weight codes are two's complement nibbles;
+ *    group-asymmetric weight codes are unsigned 0..15 with an integer zero
+ *    point.  Every packed row holds ceil(cols/2) bytes.
+ *  - fp16 values (scales, zero points) are passed as uint16_t bit patterns.
+ *  - Device pointers to packed rows and to X must be 16-byte aligned, and
+ *    row strides in bytes must be multiples of 16 (HQ_ERR_ALIGN otherwise).
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HQ_OK = 0,
+    HQ_ERR_ARG = 1,          /* a size, a pointer or an index is invalid      */
+    HQ_ERR_ALIGN = 2,        /* a pointer or a stride is not 16-byte aligned  */
+    HQ_ERR_UNSUPPORTED = 3,  /* valid, but outside what the kernels implement */
+    HQ_ERR_CUDA = 4,         /* a CUDA runtime call failed                    */
+    HQ_ERR_TIMEOUT = 5       /* a device-side wait gave up (device status)    */
+} hq_status;
+
+typedef enum { HQ_F16 = 0, HQ_BF16 = 1, HQ_F32 = 2 } hq_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hq_status_str(hq_status s);
+
+/* Number of streaming multiprocessors of the current device, or -1. */
+int hq_device_sm_count(void);
+
+/*
+ * hq_rotate_quant -- online activation transform, kernel K1.
+ * Source: "OffQ: Taming Structured Outliers in LLM Quantization by Offsetting",
+ * Methodology 2 (Hadamard rotation whose first row is all ones turns an
+ * outlier concentrated in one channel into a constant offset over the group)
+ * and 3 (group-wise rotation); "SERQ: Saliency-Aware Low-Rank Error
+ * Reconstruction for LLM Quantization", technical summary section 1 (4-bit
+ * activations, outliers set the step size).
+ *
+ * For every row m and every group b of `group` consecutive channels:
+ *   u = (x_b .* d) * H_sylv            fp32 butterfly, stages h = 1,2,4,...
+ *                                      ascending, (a,b) -> (a+b, a-b)
+ *   amax = max over the whole row of |u|
+ *   q = clamp(rint(fl32(u * fl32(7/amax))), -7, 7)   (all 0 if amax == 0)
+ *   sx[m] = fl32(fl32(amax/7) * fl32(1/sqrt(group)))  (0 if amax == 0)
+ * so that x*blockdiag(H)/sqrt(group) ~= q * sx[m].  H = diag(d)*Sylvester is a
+ * Hadamard matrix with H[0,:] = 1 when d[0] = +1.
+ *
+ *  X       device, [M][ld_x] elements of type xt (HQ_F16 or HQ_BF16), row-major
+ *  ld_x    row stride of X in elements, >= K, ld_x*2 a multiple of 16
+ *  group   power of two, 8 <= group <= 4096, K % group == 0, K % 32 == 0
+ *  H_signs device, [group] int8 in {+1,-1} with H_signs[0] == +1, or NULL (d = 1).
+ *          The sign of d[0] is not checked on the device; values other than
+ *          -1 are treated as +1.
+ *  Xq      device, [M][K/2] packed int4 codes (output)
+ *  sx      device, [M] fp32 scales (output)
+ * Errors: HQ_ERR_ARG (M < 0, K <= 0, bad group, K % group, K % 32, NULL
+ * pointer with M > 0), HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED (xt not 16-bit),
+ * HQ_ERR_CUDA (launch failure).  M == 0 is a no-op.
+ */
+hq_status hq_rotate_quant(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                          int32_t group, const int8_t* H_signs, uint8_t* Xq, float* sx,
+                          void* stream);
+
+/*
+ * hq_rotate -- the same rotation without quantisation, normalised:
+ *   out[m][k] = fl32(u[m][k] * fl32(1/sqrt(group))).
+ * Used offline to fold the rotation into the weights (W_rot = W * H~ keeps
+ * X*W^T = (X*H~)*(W*H~)^T for the orthonormal H~ = blockdiag(H)/sqrt(group);
+ * implied by OffQ, Methodology 2).
+ *  X       device, [M][K] (xt = HQ_F16, HQ_BF16 or HQ_F32), contiguous rows
+ *  out     device, [M][K] fp32 (output)
+ * Errors as hq_rotate_quant.
+ */
+hq_status hq_rotate(const void* X, hq_dtype xt, int64_t M, int64_t K, int32_t group,
+                    const int8_t* H_signs, float* out, void* stream);
+
+/*
+ * hq_channel_sqnorm -- calibration statistic for choosing the salient input
+ * channels: norm2[k] += sum_m u[m][k]^2 over the rotated (unnormalised) rows.
+ * Source: the per-channel activation L2 norm of "Adaptacion a cualquier
+ * ancho de bits: Cuantizacion de precision mixta por canal para LLMs (CMPQ)",
+ * Methodology A; SERQ section 2.2 (salient rows are those with the largest
+ * accumulated error from activation outliers).
+ *  norm2   device, [K] fp32, ACCUMULATED into (zero it before the first call);
+ *          the summation order across rows is not fixed (atomics).
+ * Errors as hq_rotate_quant.
+ */
+hq_status hq_channel_sqnorm(const void* X, hq_dtype xt, int64_t M, int64_t K, int32_t group,
+                            const int8_t* H_signs, float* norm2, void* stream);
+
+/*
+ * hq_select_salient -- host helper: the r largest entries of norm2 (ties to the
+ * lower index), written in ascending index order to sal (host, [r] int32).
+ *  norm2   host, [K] fp32
+ * Errors: HQ_ERR_ARG (NULL, r < 0, r > K).
+ */
+hq_status hq_select_salient(const float* norm2, int64_t K, int32_t r, int32_t* sal);
+
+/*
+ * w4_pack -- offline weight quantiser, kernel K0.  Source: 4-bit weights of
+ * SERQ sections 1-3; group-wise scale and zero point of OffQ Methodology 3;
+ * uniform grid (OffQ contribution 2).
+ *  group == 0: per output channel symmetric:
+ *      s16 = fp16(fl32(amax_n/7)); q = clamp(rint(fl32(w/s16)), -8, 7), or 0
+ *      when s16 == 0; sw[n] = s16; zw unused (may be NULL).
+ *  group  > 0: per (channel, group) asymmetric over [min(lo,0), max(hi,0)]:
+ *      s16 = fp16(fl32(fl32(hi-lo)/15)), 1.0 if that is 0;
+ *      z = clamp(rint(fl32(-lo/s16)), 0, 15); q = clamp(rint(fl32(w/s16))+z, 0, 15);
+ *      sw[b][n] = s16; zw[b][n] = fp16(z) (an integer): group-major layout.
+ *  W       device, [N][K] of type wt (HQ_F16, HQ_BF16 or HQ_F32), contiguous
+ *  Wq      device, [N][K/2] packed codes (output)
+ *  sw      device, fp16 bits, [N] (group == 0) or [K/group][N] (output)
+ *  zw      device, fp16 bits, [K/group][N] (output, group > 0)
+ * Errors: HQ_ERR_ARG (sizes, K odd, K % group, group < 0 or odd, NULLs),
+ * HQ_ERR_ALIGN, HQ_ERR_CUDA.
+ */
+hq_status w4_pack(const void* W, hq_dtype wt, int64_t N, int64_t K, int32_t group,
+                  uint8_t* Wq, uint16_t* sw, uint16_t* zw, void* stream);
+
+/*
+ * serq_prepare -- SERQ's single low-rank error matrix, offline.
+ * Source: "SERQ ...", technical summary section 2.2 (extract the salient rows
+ * of the weight error and reconstruct them with one matrix R, so that the
+ * residual path is a single 4-bit matmul on those rows) and section 3.
+ *   E[n][j] = fl32(W_rot[n][S_j] - What[n][S_j]), What the dequantised w4_pack
+ *   output; R = E quantised per output row like a symmetric weight row:
+ *   sr[n] = fp16(fl32(amax_j|E[n][j]|/7)), Rq codes in [-8,7].
+ *  W_rot   device, [N][K] fp32 (the rotated weights that were packed)
+ *  Wq, sw, zw, group   the w4_pack outputs and its group argument
+ *  sal_idx device, [r] int32 input channels, strictly ascending, in [0, K)
+ *  r       0 <= r <= 256
+ *  Rq      device, [N][ceil(r/2)] packed codes (output), the "A" operand
+ *  sr      device, [N] fp16 bits (output), the "B" operand
+ * Errors: HQ_ERR_ARG, HQ_ERR_CUDA.  sal_idx is not range-checked on the device.
+ */
+hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* Wq,
+                       const uint16_t* sw, const uint16_t* zw, int32_t group,
+                       const int32_t* sal_idx, int32_t r, uint8_t* Rq, uint16_t* sr,
+                       void* stream);
+
+/*
+ * w4a4_linear -- the W4A4 GEMM with the fused SERQ term, kernel K2.
+ * Source: "SERQ ...", technical summary section 2.2 (Y = X*W^T on 4-bit
+ * operands plus one residual path X[:,S]*R^T, all in 4 bit) and section 3
+ * (a single 4-bit matmul, no sequential low-rank factors, no intermediate
+ * quantisation); OffQ Methodology 3 (group-wise scale and zero point).
+ *   acc_b[m][n] = sum_{k in group b} qx[m][k] * (qw[n][k] - z[b][n])  (int32)
+ *   acc_c[m][n] = sum_{j<r} qx[m][S_j] * qr[n][j]                      (int32)
+ *   Y[m][n]     = sx[m] * (sum_b sw[b][n] * acc_b[m][n] + sr[n] * acc_c[m][n])
+ * computed in fp32 and rounded once to yt.  One launch.
+ *  Xq, sx   device, hq_rotate_quant outputs, [M][K/2] and [M]
+ *  Wq, sw, zw, group   device, w4_pack outputs; group is 0 or a multiple of 128
+ *  A, B     device, serq_prepare outputs Rq [N][ceil(r/2)] and sr [N] (NULL if r == 0)
+ *  sal_idx  device, [r] int32 (NULL if r == 0)
+ *  r        0 <= r <= 128
+ *  Y        device, [M][N] of type yt (HQ_F16, HQ_BF16 or HQ_F32) (output)
+ *  workspace, ws_bytes   device scratch of at least
+ *           hq_linear_workspace_size(M, N, K, group) bytes (may be NULL when
+ *           that size is 0).  Zero it once before its first use; every call
+ *           leaves it zeroed again.  Calls that share a workspace must not
+ *           overlap in time.
+ * Requirements: K % 128 == 0, 0 < K <= 65536, N % 8 == 0.
+ * Errors: HQ_ERR_ARG, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA.
+ */
+size_t hq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group);
+
+hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,
+                      const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
+                      int32_t group, const uint8_t* A, const uint16_t* B,
+                      const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hq_debug_accum -- test hook: runs the GEMM kernel of w4a4_linear with the
+ * epilogue replaced by a raw store of the exact integer accumulators.
+ *  acc     device, int32 [M][N][G] with G = K/group (1 when group == 0)
+ *  acc_c   device, int32 [M][N] (may be NULL when r == 0)
+ *  decode  0 = the large-M kernel, 1 = the small-M (swap-operand) kernel
+ * Same requirements and errors as w4a4_linear.
+ */
+hq_status hq_debug_accum(const uint8_t* Xq, int64_t M, int64_t K, const uint8_t* Wq,
+                         const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
+                         const int32_t* sal_idx, int32_t r, int32_t* acc, int32_t* acc_c,
+                         int32_t decode, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hq_last_device_status -- synchronises `stream`, then reads and clears the
+ * device status word that kernels set when a bounded wait gives up
+ * (HQ_ERR_TIMEOUT) or an internal check fails (HQ_ERR_ARG).  HQ_OK if clean.
+ */
+hq_status hq_last_device_status(void* stream);
+
+/*
+ * hq_debug_wait_probe -- test hook for the failure path: launches one block
+ * that waits, with the same bounded wait the GEMM kernels use, on an
+ * mbarrier that nothing ever arrives on, with a time limit of `limit_ns`
+ * nanoseconds (1 <= limit_ns <= 1e9).  The wait gives up, records
+ * HQ_ERR_TIMEOUT in the device status word and the block exits normally, so
+ * the context stays usable.  Read the status with hq_last_device_status().
+ */
+hq_status hq_debug_wait_probe(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

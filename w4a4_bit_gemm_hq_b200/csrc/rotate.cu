@@ -1,0 +1,339 @@
+// rotate.cu -- kernel K1 and its relatives: the grouped Walsh-Hadamard
+// rotation of activation rows with an all-ones first row of H, fused with the
+// per-token absmax, round-to-nearest-even int4 quantisation and nibble packing
+// ("OffQ: Taming Structured Outliers in LLM Quantization by Offsetting",
+// Methodology 2-3; "SERQ: Saliency-Aware Low-Rank Error Reconstruction for LLM
+// Quantization", technical summary section 1).  The same butterfly also serves
+// the offline weight fold (normalised rotation to fp32) and the calibration
+// statistic (per-channel sum of squares).
+//
+// Work mapping: one CTA owns one row at a time and walks rows persistently;
+// thread t holds the 32 consecutive channels [32t, 32t+32) of the row in
+// registers, loaded with 16-byte vector loads.  Butterfly stages with h < 32
+// run in registers (packed f32x2 adds where both operands are pairs), stages
+// 32 <= h < 1024 use warp shuffles, and stages h >= 1024 (groups of 2048 and
+// 4096) exchange through shared memory.  Every stage is an IEEE fp32 add/sub
+// of the pair (u[i], u[i+h]) in ascending h, so the codes are exactly those of
+// the plain definition regardless of which thread computes a pair.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "hq_device.cuh"
+
+namespace hq {
+
+constexpr int EPT = 32;  // channels per thread
+
+enum { MODE_QUANT = 0, MODE_ROTATE = 1, MODE_SQNORM = 2 };
+enum { XT_F16 = 0, XT_BF16 = 1, XT_F32 = 2 };
+
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+template <int G, int XT, int MODE>
+__global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int64_t M, int64_t K, int64_t ldx,
+                                                 const int8_t* __restrict__ dsign, uint8_t* __restrict__ Xq,
+                                                 float* __restrict__ sx, float* __restrict__ out, float cg) {
+    constexpr int TPG = (G > EPT) ? G / EPT : 1;     // threads per group
+    constexpr int HREG = (G < EPT) ? G : EPT;        // in-register stages: h < HREG
+    constexpr int TSHFL = (TPG < 32) ? TPG : 32;     // shuffle stages: s < TSHFL
+    extern __shared__ float xch[];                   // [EPT][blockDim] exchange (G >= 2048)
+    __shared__ float red[32];
+
+    const int t = threadIdx.x;
+    const int nthr = blockDim.x;
+    const int64_t tpr = K / EPT;
+    const bool active = t < tpr;
+    const int64_t col0 = static_cast<int64_t>(t) * EPT;
+
+    // Sign words of d for this thread's channels, in the bit positions of the
+    // element sign: XT 16-bit -> bits 15 / 31 of a packed pair; f32 -> bit 31.
+    uint32_t sgn[EPT / 2];
+#pragma unroll
+    for (int i = 0; i < EPT / 2; ++i) sgn[i] = 0;
+    float accsq[MODE == MODE_SQNORM ? EPT : 1];
+#pragma unroll
+    for (int i = 0; i < (MODE == MODE_SQNORM ? EPT : 1); ++i) accsq[i] = 0.f;
+    if (active && dsign != nullptr) {
+        const int p0 = static_cast<int>(col0 % G);
+#pragma unroll
+        for (int i = 0; i < EPT; i += 2) {
+            const int8_t d0 = dsign[(p0 + i) % G];
+            const int8_t d1 = dsign[(p0 + i + 1) % G];
+            sgn[i / 2] = (d0 == -1 ? 0x8000u : 0u) | (d1 == -1 ? 0x80000000u : 0u);
+        }
+    }
+
+    for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+        float2 v[EPT / 2];
+        if (active) {
+            if constexpr (XT == XT_F32) {
+                const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(X) + m * ldx + col0);
+#pragma unroll
+                for (int j = 0; j < EPT / 4; ++j) {
+                    float4 f = __ldg(src + j);
+                    uint32_t s0 = sgn[2 * j], s1 = sgn[2 * j + 1];
+                    v[2 * j].x = __uint_as_float(__float_as_uint(f.x) ^ (s0 << 16));
+                    v[2 * j].y = __uint_as_float(__float_as_uint(f.y) ^ (s0 & 0x80000000u));
+                    v[2 * j + 1].x = __uint_as_float(__float_as_uint(f.z) ^ (s1 << 16));
+                    v[2 * j + 1].y = __uint_as_float(__float_as_uint(f.w) ^ (s1 & 0x80000000u));
+                }
+            } else {
+                const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + m * ldx + col0);
+#pragma unroll
+                for (int j = 0; j < EPT / 8; ++j) {
+                    uint4 q = __ldg(src + j);
+                    uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t x = w[e] ^ sgn[4 * j + e];
+                        if constexpr (XT == XT_BF16) {
+                            v[4 * j + e].x = __uint_as_float(x << 16);
+                            v[4 * j + e].y = __uint_as_float(x & 0xFFFF0000u);
+                        } else {
+                            __half2 h2 = *reinterpret_cast<const __half2*>(&x);
+                            v[4 * j + e] = __half22float2(h2);
+                        }
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < EPT / 2; ++i) v[i] = make_float2(0.f, 0.f);
+        }
+
+        // ---- in-register stages, ascending h
+        if constexpr (HREG > 1) {
+#pragma unroll
+            for (int i = 0; i < EPT / 2; ++i) {  // h = 1: inside each pair
+                const float a = v[i].x, b = v[i].y;
+                v[i].x = __fadd_rn(a, b);
+                v[i].y = __fsub_rn(a, b);
+            }
+        }
+#pragma unroll
+        for (int h = 2; h < HREG; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < EPT; i += 2) {
+                if ((i & h) == 0) {
+                    const float2 a = v[i / 2], b = v[(i + h) / 2];
+                    v[i / 2] = __fadd2_rn(a, b);
+                    v[(i + h) / 2] = f2sub(a, b);
+                }
+            }
+        }
+        // ---- shuffle stages: partner thread t ^ s holds channels +-32s
+#pragma unroll
+        for (int s = 1; s < TSHFL; s <<= 1) {
+            const bool upper = (t & s) != 0;
+#pragma unroll
+            for (int i = 0; i < EPT / 2; ++i) {
+                float2 p;
+                p.x = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, s);
+                p.y = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, s);
+                v[i] = upper ? f2sub(p, v[i]) : __fadd2_rn(v[i], p);
+            }
+        }
+        // ---- cross-warp stages through shared memory (G >= 2048)
+        if constexpr (TPG > 32) {
+#pragma unroll
+            for (int s = 32; s < TPG; s <<= 1) {
+                const bool upper = (t & s) != 0;
+#pragma unroll
+                for (int i = 0; i < EPT / 2; ++i) {
+                    xch[(2 * i) * nthr + t] = v[i].x;
+                    xch[(2 * i + 1) * nthr + t] = v[i].y;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int i = 0; i < EPT / 2; ++i) {
+                    float2 p = make_float2(xch[(2 * i) * nthr + (t ^ s)], xch[(2 * i + 1) * nthr + (t ^ s)]);
+                    v[i] = upper ? f2sub(p, v[i]) : __fadd2_rn(v[i], p);
+                }
+                __syncthreads();
+            }
+        }
+
+        if constexpr (MODE == MODE_ROTATE) {
+            if (active) {
+                float4* dst = reinterpret_cast<float4*>(out + m * K + col0);
+                const float2 c2 = make_float2(cg, cg);
+#pragma unroll
+                for (int j = 0; j < EPT / 4; ++j) {
+                    const float2 a = __fmul2_rn(v[2 * j], c2), b = __fmul2_rn(v[2 * j + 1], c2);
+                    dst[j] = make_float4(a.x, a.y, b.x, b.y);
+                }
+            }
+        } else if constexpr (MODE == MODE_SQNORM) {
+#pragma unroll
+            for (int i = 0; i < EPT / 2; ++i) {
+                accsq[2 * i] = __fmaf_rn(v[i].x, v[i].x, accsq[2 * i]);
+                accsq[2 * i + 1] = __fmaf_rn(v[i].y, v[i].y, accsq[2 * i + 1]);
+            }
+        } else {
+            // ---- per-token absmax over the whole row
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < EPT / 2; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            const int nw = nthr >> 5;
+            if (nw > 1) {
+                if ((t & 31) == 0) red[t >> 5] = amax;
+                __syncthreads();
+                amax = 0.f;
+                for (int w = 0; w < nw; ++w) amax = fmaxf(amax, red[w]);
+                __syncthreads();  // red is rewritten by the next row
+            }
+            // ---- scale, round half to even, pack
+            uint32_t words[EPT / 8];
+            if (amax == 0.f) {
+#pragma unroll
+                for (int j = 0; j < EPT / 8; ++j) words[j] = 0u;
+            } else {
+                const float inv = __fdiv_rn(7.0f, amax);
+                const float2 inv2 = make_float2(inv, inv);
+                const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+#pragma unroll
+                for (int j = 0; j < EPT / 8; ++j) {
+                    uint32_t w = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // |u * inv| <= 7 (1 + 2^-23): adding 1.5*2^23 rounds it to an
+                        // integer with ties to even; the low nibble of the sum's bits is
+                        // that integer in two's complement.
+                        const float2 r = __fadd2_rn(__fmul2_rn(v[4 * j + e], inv2), magic);
+                        const uint32_t b0 = __float_as_uint(r.x) & 0xFu;
+                        const uint32_t b1 = __float_as_uint(r.y) & 0xFu;
+                        w |= (b0 | (b1 << 4)) << (8 * e);
+                    }
+                    words[j] = w;
+                }
+            }
+            if (active) {
+                uint4* dst = reinterpret_cast<uint4*>(Xq + m * (K / 2) + col0 / 2);
+                *dst = make_uint4(words[0], words[1], words[2], words[3]);
+            }
+            if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+        }
+    }
+
+    if constexpr (MODE == MODE_SQNORM) {
+        if (active) {
+#pragma unroll
+            for (int i = 0; i < EPT; ++i) atomicAdd(out + col0 + i, accsq[i]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ dispatch
+template <int XT, int MODE>
+static hq_status launch_g(int group, const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* d, uint8_t* Xq,
+                          float* sx, float* out, cudaStream_t st) {
+    const int threads = static_cast<int>(((K / EPT) + 31) / 32 * 32);
+    const float cg = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(group)));
+    const size_t shm = (group >= 2048) ? static_cast<size_t>(EPT) * threads * sizeof(float) : 0;
+    int nsm = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    auto run = [&](auto kern) -> hq_status {
+        if (shm > 48 * 1024) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shm)) !=
+                cudaSuccess)
+                return HQ_ERR_CUDA;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, shm) != cudaSuccess || per_sm < 1)
+            return HQ_ERR_CUDA;
+        int64_t grid = static_cast<int64_t>(per_sm) * nsm;
+        if (grid > M) grid = M;
+        kern<<<static_cast<unsigned>(grid), threads, shm, st>>>(X, M, K, ldx, d, Xq, sx, out, cg);
+        return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    };
+    switch (group) {
+        case 8: return run(k_rotate<8, XT, MODE>);
+        case 16: return run(k_rotate<16, XT, MODE>);
+        case 32: return run(k_rotate<32, XT, MODE>);
+        case 64: return run(k_rotate<64, XT, MODE>);
+        case 128: return run(k_rotate<128, XT, MODE>);
+        case 256: return run(k_rotate<256, XT, MODE>);
+        case 512: return run(k_rotate<512, XT, MODE>);
+        case 1024: return run(k_rotate<1024, XT, MODE>);
+        case 2048: return run(k_rotate<2048, XT, MODE>);
+        case 4096: return run(k_rotate<4096, XT, MODE>);
+        default: return HQ_ERR_UNSUPPORTED;
+    }
+}
+
+template <int MODE>
+static hq_status launch_rotate(int xt, int group, const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* d,
+                               uint8_t* Xq, float* sx, float* out, cudaStream_t st) {
+    if (xt == HQ_F16) return launch_g<XT_F16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
+    if (xt == HQ_BF16) return launch_g<XT_BF16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
+    if constexpr (MODE != MODE_QUANT) {
+        if (xt == HQ_F32) return launch_g<XT_F32, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
+    }
+    return HQ_ERR_UNSUPPORTED;
+}
+
+static bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static hq_status check_rotate_args(int xt, int64_t M, int64_t K, int group) {
+    if (M < 0 || K <= 0) return HQ_ERR_ARG;
+    if (!is_pow2(group) || group < 8 || group > 4096) return HQ_ERR_ARG;
+    if (K % group != 0 || K % EPT != 0) return HQ_ERR_ARG;
+    if (xt != HQ_F16 && xt != HQ_BF16 && xt != HQ_F32) return HQ_ERR_UNSUPPORTED;
+    if (K / EPT > 512) return HQ_ERR_UNSUPPORTED;
+    return HQ_OK;
+}
+
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" hq_status hq_rotate_quant(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x, int32_t group,
+                                     const int8_t* H_signs, uint8_t* Xq, float* sx, void* stream) {
+    hq_status s = check_rotate_args(xt, M, K, group);
+    if (s != HQ_OK) return s;
+    if (xt == HQ_F32) return HQ_ERR_UNSUPPORTED;
+    if (ld_x < K) return HQ_ERR_ARG;
+    if (M == 0) return HQ_OK;
+    if (!X || !Xq || !sx) return HQ_ERR_ARG;
+    if (!al16(X) || !al16(Xq) || (ld_x * 2) % 16 != 0) return HQ_ERR_ALIGN;
+    return launch_rotate<MODE_QUANT>(xt, group, X, M, K, ld_x, H_signs, Xq, sx, nullptr,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hq_status hq_rotate(const void* X, hq_dtype xt, int64_t M, int64_t K, int32_t group,
+                               const int8_t* H_signs, float* out, void* stream) {
+    hq_status s = check_rotate_args(xt, M, K, group);
+    if (s != HQ_OK) return s;
+    if (M == 0) return HQ_OK;
+    if (!X || !out) return HQ_ERR_ARG;
+    if (!al16(X) || !al16(out)) return HQ_ERR_ALIGN;
+    return launch_rotate<MODE_ROTATE>(xt, group, X, M, K, K, H_signs, nullptr, nullptr, out,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hq_status hq_channel_sqnorm(const void* X, hq_dtype xt, int64_t M, int64_t K, int32_t group,
+                                       const int8_t* H_signs, float* norm2, void* stream) {
+    hq_status s = check_rotate_args(xt, M, K, group);
+    if (s != HQ_OK) return s;
+    if (M == 0) return HQ_OK;
+    if (!X || !norm2) return HQ_ERR_ARG;
+    if (!al16(X)) return HQ_ERR_ALIGN;
+    return launch_rotate<MODE_SQNORM>(xt, group, X, M, K, K, H_signs, nullptr, nullptr, norm2,
+                                      static_cast<cudaStream_t>(stream));
+}

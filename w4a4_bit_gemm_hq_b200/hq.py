@@ -1,0 +1,198 @@
+"""User-facing calls of the W4A4 rotated linear layer, one per C-ABI entry point
+(same names), plus :class:`W4A4Linear`, which holds a prepared layer.
+
+Every function takes and returns PyTorch CUDA tensors, checks nothing beyond
+shapes and dtypes needed to size its outputs (the C ABI validates the rest and
+its status is raised as :class:`HQError`), and enqueues on the current stream.
+
+Sources (page title, section): the rotation and quantiser follow "OffQ:
+Taming Structured Outliers in LLM Quantization by Offsetting", Methodology 2-3,
+and "SERQ: Saliency-Aware Low-Rank Error Reconstruction for LLM Quantization",
+technical summary sections 1-3; the salient channels are those with the
+largest activation L2 norm ("CMPQ", Methodology A).
+"""
+import torch
+
+from . import _lib
+from ._lib import HQError, check, dtype_code, lib, ptr, stream_handle
+
+__all__ = [
+    "HQError", "hq_rotate_quant", "hq_rotate", "hq_channel_sqnorm", "hq_select_salient", "w4_pack",
+    "serq_prepare", "w4a4_linear", "hq_linear_workspace_size", "hq_debug_accum", "hq_last_device_status",
+    "hq_debug_wait_probe", "W4A4Linear",
+]
+
+
+def _signs_arg(H_signs):
+    if H_signs is None:
+        return None
+    assert H_signs.dtype == torch.int8 and H_signs.is_cuda
+    return ptr(H_signs)
+
+
+def hq_rotate_quant(X, group, H_signs=None, Xq=None, sx=None):
+    """(Xq uint8 [M, K/2], sx float32 [M]): grouped Hadamard rotation with H[0,:] = 1,
+    per-token symmetric int4 codes packed two per byte."""
+    M, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    if sx is None:
+        sx = torch.empty((M,), dtype=torch.float32, device=X.device)
+    check(lib.hq_rotate_quant(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), group, _signs_arg(H_signs),
+                              ptr(Xq), ptr(sx), stream_handle()), "hq_rotate_quant")
+    return Xq, sx
+
+
+def hq_rotate(X, group, H_signs=None, out=None):
+    """fp32 X * blockdiag(H) / sqrt(group) (the rotation folded into weights)."""
+    M, K = X.shape
+    X = X.contiguous()
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.float32, device=X.device)
+    check(lib.hq_rotate(ptr(X), dtype_code(X.dtype), M, K, group, _signs_arg(H_signs), ptr(out), stream_handle()),
+          "hq_rotate")
+    return out
+
+
+def hq_channel_sqnorm(X, group, H_signs=None, norm2=None):
+    """Accumulates the per-channel sum of squares of the rotated rows into norm2 [K]."""
+    M, K = X.shape
+    X = X.contiguous()
+    if norm2 is None:
+        norm2 = torch.zeros((K,), dtype=torch.float32, device=X.device)
+    check(lib.hq_channel_sqnorm(ptr(X), dtype_code(X.dtype), M, K, group, _signs_arg(H_signs), ptr(norm2),
+                                stream_handle()), "hq_channel_sqnorm")
+    return norm2
+
+
+def hq_select_salient(norm2, r):
+    """Indices of the r largest entries (ascending), as an int32 CPU tensor."""
+    n = norm2.detach().to("cpu", torch.float32).contiguous()
+    out = torch.empty((r,), dtype=torch.int32)
+    check(lib.hq_select_salient(ptr(n), n.numel(), r, ptr(out)), "hq_select_salient")
+    return out
+
+
+def w4_pack(W, group):
+    """(Wq uint8 [N, K/2], sw fp16 [N] or [K/group, N], zw fp16 [K/group, N] or None)."""
+    N, K = W.shape
+    W = W.contiguous()
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    if group:
+        sw = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
+        zw = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
+    else:
+        sw = torch.empty((N,), dtype=torch.float16, device=W.device)
+        zw = None
+    check(lib.w4_pack(ptr(W), dtype_code(W.dtype), N, K, group, ptr(Wq), ptr(sw), ptr(zw), stream_handle()),
+          "w4_pack")
+    return Wq, sw, zw
+
+
+def serq_prepare(W_rot, Wq, sw, zw, group, sal_idx):
+    """(Rq uint8 [N, ceil(r/2)], sr fp16 [N]): SERQ's single error matrix on the salient inputs."""
+    N, K = W_rot.shape
+    r = int(sal_idx.numel())
+    Rq = torch.empty((N, (r + 1) // 2), dtype=torch.uint8, device=W_rot.device)
+    sr = torch.empty((N,), dtype=torch.float16, device=W_rot.device)
+    check(lib.serq_prepare(ptr(W_rot), N, K, ptr(Wq), ptr(sw), ptr(zw), group, ptr(sal_idx), r, ptr(Rq), ptr(sr),
+                           stream_handle()), "serq_prepare")
+    return Rq, sr
+
+
+def hq_linear_workspace_size(M, N, K, group):
+    return int(lib.hq_linear_workspace_size(M, N, K, group))
+
+
+def w4a4_linear(Xq, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat16, Y=None, workspace=None):
+    """Y [M, N] = sx * (sum_b sw * acc_b + sr * acc_c), one fused launch."""
+    M = Xq.shape[0]
+    K = Xq.shape[1] * 2
+    N = Wq.shape[0]
+    r = 0 if sal_idx is None else int(sal_idx.numel())
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=Xq.device)
+    need = hq_linear_workspace_size(M, N, K, group)
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=Xq.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.w4a4_linear(ptr(Xq), ptr(sx), M, K, ptr(Wq), ptr(sw), ptr(zw), N, group,
+                          ptr(A) if r else None, ptr(B) if r else None, ptr(sal_idx) if r else None, r,
+                          ptr(Y), dtype_code(Y.dtype), ptr(workspace), ws_bytes, stream_handle()), "w4a4_linear")
+    return Y
+
+
+def hq_debug_accum(Xq, Wq, zw, group, A, sal_idx, decode=False, workspace=None):
+    """Exact int32 accumulators of the GEMM kernel: (acc [M, N, G], acc_c [M, N])."""
+    M = Xq.shape[0]
+    K = Xq.shape[1] * 2
+    N = Wq.shape[0]
+    r = 0 if sal_idx is None else int(sal_idx.numel())
+    G = K // group if group else 1
+    acc = torch.zeros((M, N, G), dtype=torch.int32, device=Xq.device)
+    acc_c = torch.zeros((M, N), dtype=torch.int32, device=Xq.device)
+    need = hq_linear_workspace_size(M, N, K, group) if decode else 0
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=Xq.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.hq_debug_accum(ptr(Xq), M, K, ptr(Wq), ptr(zw), N, group, ptr(A) if r else None,
+                             ptr(sal_idx) if r else None, r, ptr(acc), ptr(acc_c), 1 if decode else 0,
+                             ptr(workspace), ws_bytes, stream_handle()), "hq_debug_accum")
+    return acc, acc_c
+
+
+def hq_last_device_status():
+    return int(lib.hq_last_device_status(stream_handle()))
+
+
+def hq_debug_wait_probe(limit_ns):
+    check(lib.hq_debug_wait_probe(int(limit_ns), stream_handle()), "hq_debug_wait_probe")
+
+
+class W4A4Linear:
+    """A prepared W4A4 layer: rotation signs, packed weights, SERQ term, workspace.
+
+    ``prepare`` runs the offline steps on the GPU: fold the rotation into W,
+    pack to int4, pick the r salient input channels from calibration
+    activations (largest rotated L2 norm), build SERQ's error matrix.
+    ``forward`` is the online path: one rotate/quant launch and one GEMM launch.
+    """
+
+    def __init__(self, group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype):
+        self.group, self.gw, self.H_signs = group, gw, H_signs
+        self.Wq, self.sw, self.zw, self.Rq, self.sr, self.sal_idx = Wq, sw, zw, Rq, sr, sal_idx
+        self.K, self.N, self.out_dtype = K, N, out_dtype
+        self._ws = {}
+
+    @classmethod
+    def prepare(cls, W, group, gw, r, H_signs=None, X_calib=None, sal_idx=None, out_dtype=torch.bfloat16):
+        N, K = W.shape
+        W_rot = hq_rotate(W, group, H_signs)
+        Wq, sw, zw = w4_pack(W_rot, gw)
+        if sal_idx is None and r > 0:
+            norm2 = hq_channel_sqnorm(X_calib, group, H_signs)
+            sal_idx = hq_select_salient(norm2, r).to(W.device)
+        if r > 0:
+            sal_idx = sal_idx.to(device=W.device, dtype=torch.int32).contiguous()
+            Rq, sr = serq_prepare(W_rot, Wq, sw, zw, gw, sal_idx)
+        else:
+            sal_idx, Rq, sr = None, None, None
+        del W_rot
+        return cls(group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype)
+
+    def workspace(self, M, device):
+        need = hq_linear_workspace_size(M, self.N, self.K, self.gw)
+        if need == 0:
+            return None
+        ws = self._ws.get(need)
+        if ws is None:
+            ws = torch.zeros((need,), dtype=torch.uint8, device=device)
+            self._ws[need] = ws
+        return ws
+
+    def forward(self, X, Y=None, Xq=None, sx=None):
+        Xq, sx = hq_rotate_quant(X, self.group, self.H_signs, Xq, sx)
+        return w4a4_linear(Xq, sx, self.Wq, self.sw, self.zw, self.gw, self.Rq, self.sr, self.sal_idx,
+                           self.out_dtype, Y, self.workspace(X.shape[0], X.device))
+
+    __call__ = forward
