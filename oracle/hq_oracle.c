@@ -299,7 +299,8 @@ void hqo_w4_pack(const void* W, int dtype, int64_t N, int64_t K, int32_t gw,
                 uint16_t s16 = hqo_f32_to_f16((hi - lo) / 15.0f);
                 if (hqo_f16_to_f32(s16) == 0.0f) s16 = 0x3C00u; /* 1.0 */
                 float s = hqo_f16_to_f32(s16);
-                float z = clampf(rintf(-lo / s), 0.0f, 15.0f);
+                /* an integer in 0..15; the int round trip makes a zero +0 (never -0) */
+                float z = (float)(int)clampf(rintf(-lo / s), 0.0f, 15.0f);
                 sw[b * N + n] = s16;
                 zw[b * N + n] = hqo_f32_to_f16(z);
                 for (int64_t k = b * gw; k < (b + 1) * gw; ++k) {
