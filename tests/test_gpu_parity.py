@@ -39,6 +39,16 @@ def f16bits(a):
     return np.ascontiguousarray(a).view(np.uint16)
 
 
+def assert_same(a, b, what="values"):
+    a = np.ascontiguousarray(a)
+    b = np.ascontiguousarray(b)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    if a.dtype.itemsize == 4 and a.dtype.kind == "f":
+        a, b = a.view(np.uint32), b.view(np.uint32)
+    bad = a != b
+    assert not bad.any(), "%s: %d of %d differ, first at %s" % (what, bad.sum(), bad.size, np.argwhere(bad)[:4])
+
+
 def assert_y_close(y, y64, tol):
     y = y.astype(np.float64)
     ref = np.abs(y64)
@@ -78,8 +88,8 @@ def test_rotate_quant_bit_exact_workloads(name, M, _):
     d = synth.hadamard_signs(wl.g)
     Xq_o, sx_o = O.rotate_quant(X, wl.xdtype, wl.g, d)
     Xq, sx = hq.hq_rotate_quant(dev(X, wl.xdtype), wl.g, torch.from_numpy(d).cuda())
-    assert np.array_equal(host(Xq), Xq_o)
-    assert np.array_equal(host(sx).view(np.uint32), sx_o.view(np.uint32))
+    assert_same(host(Xq), Xq_o, "codes")
+    assert_same(host(sx), sx_o, "scales")
     no_device_error()
 
 
@@ -94,12 +104,25 @@ def test_rotate_quant_bit_exact_group_sweep(g, dtype):
     d = synth.hadamard_signs(g, seed=g)
     Xq_o, sx_o = O.rotate_quant(X, dtype, g, d)
     Xq, sx = hq.hq_rotate_quant(dev(X, dtype), g, torch.from_numpy(d).cuda())
-    assert np.array_equal(host(Xq), Xq_o)
-    assert np.array_equal(host(sx).view(np.uint32), sx_o.view(np.uint32))
+    assert_same(host(Xq), Xq_o, "codes")
+    assert_same(host(sx), sx_o, "scales")
     # H = None means d = 1
     Xq_o, sx_o = O.rotate_quant(X, dtype, g, None)
     Xq, sx = hq.hq_rotate_quant(dev(X, dtype), g, None)
     assert np.array_equal(host(Xq), Xq_o) and np.array_equal(host(sx), sx_o)
+
+
+def test_rotate_quant_rounding_ties_follow_the_definition():
+    # fl32(u * inv) lands exactly on x.5 while the exact product does not: a
+    # fused multiply-add would round the other way
+    X = np.zeros((3, 32), np.float16)
+    X[0, 0], X[0, 8] = 1.5, 3.0
+    X[1, 0], X[1, 8] = 2.75, 5.5
+    X[2, 0], X[2, 8] = 5.5, 11.0
+    Xq_o, sx_o = O.rotate_quant(X, "f16", 8, None)
+    Xq, sx = hq.hq_rotate_quant(dev(X, "f16"), 8, None)
+    assert_same(host(Xq), Xq_o, "codes")
+    assert np.all(O.unpack_s4(host(Xq), 32)[:, :8] == 4)
 
 
 def test_rotate_quant_edge_rows_and_strides():
@@ -130,7 +153,7 @@ def test_rotate_normalised_bit_exact(dtype, g):
     d = synth.hadamard_signs(g, seed=5)
     ref = O.rotate_normalised(W, dtype, g, d)
     out = hq.hq_rotate(dev(W, dtype), g, torch.from_numpy(d).cuda())
-    assert np.array_equal(host(out).view(np.uint32), ref.view(np.uint32))
+    assert_same(host(out), ref, "rotated")
 
 
 def test_channel_sqnorm_and_salient_selection():
@@ -231,9 +254,9 @@ def test_gemm_accumulators_bit_exact(M, N, K, gw, r):
     acc_o, accc_o = O.accum(t["Xq"], K, t["Wq"], t["zw"], gw, t["Rq"], t["sal"])
     g = _dev_inputs(t)
     acc, acc_c = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, g["Rq"], g["sal"])
-    assert np.array_equal(host(acc).astype(np.int64), acc_o)
+    assert_same(host(acc).astype(np.int64), acc_o, "acc")
     if r:
-        assert np.array_equal(host(acc_c).astype(np.int64), accc_o)
+        assert_same(host(acc_c).astype(np.int64), accc_o, "acc_c")
     no_device_error()
 
 

@@ -200,6 +200,21 @@ def test_activation_quant_round_trip(name):
     assert np.allclose(sx, s * cg, rtol=2 ** -22)
 
 
+def test_activation_codes_round_the_fp32_product_ties_to_even():
+    # reading of the quantiser: q = rint(fl32(u * fl32(7/amax))), two roundings.
+    # u = 1.5 on group 0, amax = 3: fl32(1.5 * fl32(7/3)) is exactly 3.5 (the exact
+    # product is 3.49999988), so q = 4 (tie to even), not 3.
+    X = np.zeros((2, 32), np.float16)
+    X[0, 0], X[0, 8] = 1.5, 3.0
+    X[1, 0], X[1, 8] = 2.75, 5.5
+    Xq, _ = O.rotate_quant(X, "f16", 8, None)
+    q = O.unpack_s4(Xq, 32)
+    inv = np.float32(7) / np.float32(3)
+    assert np.float32(np.float32(1.5) * inv) == np.float32(3.5)
+    assert np.all(q[0, :8] == 4) and np.all(q[0, 8:16] == 7) and np.all(q[0, 16:] == 0)
+    assert np.all(q[1, :8] == 4) and np.all(q[1, 8:16] == 7)
+
+
 def test_activation_zero_row():
     X = np.zeros((2, 256), np.float16)
     X[1, 3] = 1.0

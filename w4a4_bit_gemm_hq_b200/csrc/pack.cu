@@ -88,7 +88,8 @@ __global__ void k_pack_asym(const void* __restrict__ W, int64_t N, int64_t K, in
     uint16_t s16 = half_bits(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
     if (bits_half(s16) == 0.f) s16 = 0x3C00u;  // 1.0
     const float s = bits_half(s16);
-    const float z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), 15.f);
+    // an integer in 0..15; the int round trip makes a zero +0 (never -0)
+    const float z = static_cast<float>(static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), 15.f)));
     if (lane == 0) {
         sw[b * N + n] = s16;
         zw[b * N + n] = half_bits(z);

@@ -41,6 +41,31 @@ __device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
     return r;
 }
 
+// Packed IEEE round-to-nearest multiply / add (sm_100 f32x2).
+__device__ __forceinline__ float2 f2mul_rn(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 f2add_rn(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
 template <int G, int XT, int MODE>
 __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int64_t M, int64_t K, int64_t ldx,
                                                  const int8_t* __restrict__ dsign, uint8_t* __restrict__ Xq,
@@ -128,7 +153,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
             for (int i = 0; i < EPT; i += 2) {
                 if ((i & h) == 0) {
                     const float2 a = v[i / 2], b = v[(i + h) / 2];
-                    v[i / 2] = __fadd2_rn(a, b);
+                    v[i / 2] = f2add_rn(a, b);
                     v[(i + h) / 2] = f2sub(a, b);
                 }
             }
@@ -142,7 +167,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 float2 p;
                 p.x = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, s);
                 p.y = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, s);
-                v[i] = upper ? f2sub(p, v[i]) : __fadd2_rn(v[i], p);
+                v[i] = upper ? f2sub(p, v[i]) : f2add_rn(v[i], p);
             }
         }
         // ---- cross-warp stages through shared memory (G >= 2048)
@@ -159,7 +184,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
 #pragma unroll
                 for (int i = 0; i < EPT / 2; ++i) {
                     float2 p = make_float2(xch[(2 * i) * nthr + (t ^ s)], xch[(2 * i + 1) * nthr + (t ^ s)]);
-                    v[i] = upper ? f2sub(p, v[i]) : __fadd2_rn(v[i], p);
+                    v[i] = upper ? f2sub(p, v[i]) : f2add_rn(v[i], p);
                 }
                 __syncthreads();
             }
@@ -171,7 +196,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 const float2 c2 = make_float2(cg, cg);
 #pragma unroll
                 for (int j = 0; j < EPT / 4; ++j) {
-                    const float2 a = __fmul2_rn(v[2 * j], c2), b = __fmul2_rn(v[2 * j + 1], c2);
+                    const float2 a = f2mul_rn(v[2 * j], c2), b = f2mul_rn(v[2 * j + 1], c2);
                     dst[j] = make_float4(a.x, a.y, b.x, b.y);
                 }
             }
@@ -203,7 +228,6 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 for (int j = 0; j < EPT / 8; ++j) words[j] = 0u;
             } else {
                 const float inv = __fdiv_rn(7.0f, amax);
-                const float2 inv2 = make_float2(inv, inv);
                 const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
 #pragma unroll
                 for (int j = 0; j < EPT / 8; ++j) {
@@ -213,7 +237,10 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                         // |u * inv| <= 7 (1 + 2^-23): adding 1.5*2^23 rounds it to an
                         // integer with ties to even; the low nibble of the sum's bits is
                         // that integer in two's complement.
-                        const float2 r = __fadd2_rn(__fmul2_rn(v[4 * j + e], inv2), magic);
+                        // __fmul_rn is never merged into an fma, so fl32(u * inv) is
+                        // rounded before the rounding add, as the codes are defined.
+                        const float2 t = make_float2(__fmul_rn(v[4 * j + e].x, inv), __fmul_rn(v[4 * j + e].y, inv));
+                        const float2 r = f2add_rn(t, magic);
                         const uint32_t b0 = __float_as_uint(r.x) & 0xFu;
                         const uint32_t b1 = __float_as_uint(r.y) & 0xFu;
                         w |= (b0 | (b1 << 4)) << (8 * e);
