@@ -22,7 +22,16 @@
  *  - Packed int4: element 2j is the low nibble of byte j, 2j+1 the high nibble.
  *    Activation codes and symmetric weight codes are two's complement nibbles;
  *    group-asymmetric weight codes are unsigned 0..15 with an integer zero
- *    point.  Every packed row holds ceil(cols/2) bytes.
+ *    point.  Packed activation rows (Xq) and SERQ rows (Rq) are row-major,
+ *    ceil(cols/2) bytes per row.
+ *  - Packed weights (Wq) are TILE-MAJOR: the row-major [N][K/2] byte matrix is
+ *    cut into tiles of 128 rows x 64 bytes (128 rows x 128 input channels);
+ *    tile (t, kb) is 8192 contiguous bytes at offset (t*(K/128) + kb) * 8192,
+ *    row r of the tile at +r*64.  Byte j of row n is therefore at
+ *    ((n/128 * (K/128) + j/64) * 128 + n%128) * 64 + j%64.  N is padded to a
+ *    multiple of 128 with zero codes: the buffer holds
+ *    hq_packed_weight_bytes(N, K) = ceil(N/128)*128 * K/2 bytes.  Every weight
+ *    tile a GEMM stage needs is thus one contiguous 8 KB block in HBM.
  *  - fp16 values (scales, zero points) are passed as uint16_t bit patterns.
  *  - Device pointers to packed rows and to X must be 16-byte aligned, and
  *    row strides in bytes must be multiples of 16 (HQ_ERR_ALIGN otherwise).
@@ -53,6 +62,9 @@ const char* hq_status_str(hq_status s);
 
 /* Number of streaming multiprocessors of the current device, or -1. */
 int hq_device_sm_count(void);
+
+/* Bytes of a tile-major packed weight buffer for N x K weights (K % 128 == 0). */
+size_t hq_packed_weight_bytes(int64_t N, int64_t K);
 
 /*
  * hq_rotate_quant -- online activation transform, kernel K1.
@@ -135,10 +147,11 @@ hq_status hq_select_salient(const float* norm2, int64_t K, int32_t r, int32_t* s
  *      z = clamp(rint(fl32(-lo/s16)), 0, 15); q = clamp(rint(fl32(w/s16))+z, 0, 15);
  *      sw[b][n] = s16; zw[b][n] = fp16(z) (an integer): group-major layout.
  *  W       device, [N][K] of type wt (HQ_F16, HQ_BF16 or HQ_F32), contiguous
- *  Wq      device, [N][K/2] packed codes (output)
+ *  Wq      device, hq_packed_weight_bytes(N, K) bytes, tile-major codes
+ *          (output; padding rows are zero)
  *  sw      device, fp16 bits, [N] (group == 0) or [K/group][N] (output)
  *  zw      device, fp16 bits, [K/group][N] (output, group > 0)
- * Errors: HQ_ERR_ARG (sizes, K odd, K % group, group < 0 or odd, NULLs),
+ * Errors: HQ_ERR_ARG (sizes, K % 128, K % group, group < 0 or odd, NULLs),
  * HQ_ERR_ALIGN, HQ_ERR_CUDA.
  */
 hq_status w4_pack(const void* W, hq_dtype wt, int64_t N, int64_t K, int32_t group,
@@ -153,7 +166,7 @@ hq_status w4_pack(const void* W, hq_dtype wt, int64_t N, int64_t K, int32_t grou
  *   output; R = E quantised per output row like a symmetric weight row:
  *   sr[n] = fp16(fl32(amax_j|E[n][j]|/7)), Rq codes in [-8,7].
  *  W_rot   device, [N][K] fp32 (the rotated weights that were packed)
- *  Wq, sw, zw, group   the w4_pack outputs and its group argument
+ *  Wq, sw, zw, group   the w4_pack outputs (Wq tile-major) and its group argument
  *  sal_idx device, [r] int32 input channels, strictly ascending, in [0, K)
  *  r       0 <= r <= 256
  *  Rq      device, [N][ceil(r/2)] packed codes (output), the "A" operand
@@ -176,7 +189,8 @@ hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* 
  *   Y[m][n]     = sx[m] * (sum_b sw[b][n] * acc_b[m][n] + sr[n] * acc_c[m][n])
  * computed in fp32 and rounded once to yt.  One launch.
  *  Xq, sx   device, hq_rotate_quant outputs, [M][K/2] and [M]
- *  Wq, sw, zw, group   device, w4_pack outputs; group is 0 or a multiple of 128
+ *  Wq, sw, zw, group   device, w4_pack outputs (Wq tile-major); group is 0 or a
+ *           multiple of 128
  *  A, B     device, serq_prepare outputs Rq [N][ceil(r/2)] and sr [N] (NULL if r == 0)
  *  sal_idx  device, [r] int32 (NULL if r == 0)
  *  r        0 <= r <= 128

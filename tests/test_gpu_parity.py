@@ -65,6 +65,21 @@ def y_host(Y):
     return y.astype(np.float32)
 
 
+def tile_wq(Wq_rows):
+    """Row-major packed weights -> the C ABI's tile-major layout (marshalling)."""
+    N, Kh = Wq_rows.shape
+    T = (N + 127) // 128
+    pad = np.zeros((T * 128, Kh), np.uint8)
+    pad[:N] = Wq_rows
+    return np.ascontiguousarray(pad.reshape(T, 128, Kh // 64, 64).transpose(0, 2, 1, 3))
+
+
+def untile_wq(Wq, N):
+    Wq = np.asarray(Wq)
+    T, KB = Wq.shape[0], Wq.shape[1]
+    return np.ascontiguousarray(Wq.transpose(0, 2, 1, 3).reshape(T * 128, KB * 64)[:N])
+
+
 def no_device_error():
     assert hq.hq_last_device_status() == 0
 
@@ -183,7 +198,9 @@ def test_w4_pack_bit_exact(gw, N):
         W[2, :gw] = np.abs(W[2, :gw]) + 1e-3
     Wq_o, sw_o, zw_o = O.w4_pack(W, "f32", gw)
     Wq, sw, zw = hq.w4_pack(dev(W, "f32"), gw)
-    assert np.array_equal(host(Wq), Wq_o)
+    assert_same(untile_wq(host(Wq), N), Wq_o, "codes")
+    if N % 128:   # padding rows of the last row tile are zero codes
+        assert np.all(host(Wq)[-1, :, N % 128:, :] == 0)
     assert np.array_equal(f16bits(host(sw)), f16bits(sw_o))
     if gw:
         assert np.array_equal(f16bits(host(zw)), f16bits(zw_o))
@@ -197,7 +214,7 @@ def test_w4_pack_from_16bit_inputs(wdtype):
     for gw in (0, 128):
         Wq_o, sw_o, zw_o = O.w4_pack(W, wdtype, gw)
         Wq, sw, zw = hq.w4_pack(dev(W, wdtype), gw)
-        assert np.array_equal(host(Wq), Wq_o) and np.array_equal(f16bits(host(sw)), f16bits(sw_o))
+        assert np.array_equal(untile_wq(host(Wq), 40), Wq_o) and np.array_equal(f16bits(host(sw)), f16bits(sw_o))
 
 
 @pytest.mark.parametrize("gw,r", [(0, 8), (128, 16), (0, 64), (256, 40), (128, 0)])
@@ -208,7 +225,7 @@ def test_serq_prepare_bit_exact(gw, r):
     Wq, sw, zw = O.w4_pack(Wrot, "f32", gw)
     sal = np.sort(rng.choice(K, r, replace=False)).astype(np.int32)
     Rq_o, sr_o = O.serq_prepare(Wrot, Wq, sw, zw, gw, sal)
-    Rq, sr = hq.serq_prepare(dev(Wrot, "f32"), torch.from_numpy(Wq).cuda(), dev(sw, "f16"),
+    Rq, sr = hq.serq_prepare(dev(Wrot, "f32"), torch.from_numpy(tile_wq(Wq)).cuda(), dev(sw, "f16"),
                              None if zw is None else dev(zw, "f16"), gw, torch.from_numpy(sal).cuda())
     assert np.array_equal(host(Rq), Rq_o)
     assert np.array_equal(f16bits(host(sr)), f16bits(sr_o))
@@ -230,7 +247,7 @@ def _gemm_inputs(M, N, K, gw, r, seed=0):
 
 def _dev_inputs(t):
     return dict(Xq=torch.from_numpy(t["Xq"]).cuda(), sx=torch.from_numpy(t["sx"]).cuda(),
-                Wq=torch.from_numpy(t["Wq"]).cuda(), sw=dev(t["sw"], "f16"),
+                Wq=torch.from_numpy(tile_wq(t["Wq"])).cuda(), sw=dev(t["sw"], "f16"),
                 zw=None if t["zw"] is None else dev(t["zw"], "f16"),
                 sal=torch.from_numpy(t["sal"]).cuda() if len(t["sal"]) else None,
                 Rq=torch.from_numpy(t["Rq"]).cuda(), sr=dev(t["sr"], "f16"))
@@ -253,10 +270,54 @@ def test_gemm_accumulators_bit_exact(M, N, K, gw, r):
     t = _gemm_inputs(M, N, K, gw, r)
     acc_o, accc_o = O.accum(t["Xq"], K, t["Wq"], t["zw"], gw, t["Rq"], t["sal"])
     g = _dev_inputs(t)
-    acc, acc_c = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, g["Rq"], g["sal"])
+    acc, acc_c = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, g["Rq"], g["sal"], N)
     assert_same(host(acc).astype(np.int64), acc_o, "acc")
     if r:
         assert_same(host(acc_c).astype(np.int64), accc_o, "acc_c")
+    no_device_error()
+
+
+SMALL_CASES = [
+    # small-M (swap-operand, stream-K) kernel; several cases split a weight tile
+    # across CTAs, which exercises the last-arriver fixup and its counter reset
+    (1, 256, 256, 0, 8),
+    (4, 1024, 2048, 0, 16),
+    (16, 1024, 2048, 128, 16),
+    (17, 520, 1024, 128, 8),
+    (33, 264, 512, 0, 24),
+    (64, 1032, 1024, 256, 64),
+    (16, 11008, 4096, 128, 16),
+]
+
+
+@pytest.mark.parametrize("M,N,K,gw,r", SMALL_CASES)
+def test_small_m_accumulators_bit_exact(M, N, K, gw, r):
+    t = _gemm_inputs(M, N, K, gw, r, seed=2)
+    acc_o, accc_o = O.accum(t["Xq"], K, t["Wq"], t["zw"], gw, t["Rq"], t["sal"])
+    g = _dev_inputs(t)
+    for _ in range(2):
+        acc, acc_c = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, g["Rq"], g["sal"], N, decode=True)
+        assert_same(host(acc).astype(np.int64), acc_o, "acc")
+        if r:
+            assert_same(host(acc_c).astype(np.int64), accc_o, "acc_c")
+    no_device_error()
+
+
+@pytest.mark.parametrize("M,N,K,gw,r", SMALL_CASES)
+@pytest.mark.parametrize("out", [torch.float16, torch.float32])
+def test_small_m_linear_within_tolerance(M, N, K, gw, r, out):
+    t = _gemm_inputs(M, N, K, gw, r, seed=3)
+    acc_o, accc_o = O.accum(t["Xq"], K, t["Wq"], t["zw"], gw, t["Rq"], t["sal"])
+    y64 = O.epilogue_f64(acc_o, accc_o, t["sx"], t["sw"], t["sr"] if r else None)
+    g = _dev_inputs(t)
+    ws = torch.zeros((hq.hq_linear_workspace_size(M, N, K, gw),), dtype=torch.uint8, device="cuda")
+    Y = hq.w4a4_linear(g["Xq"], g["sx"], g["Wq"], g["sw"], g["zw"], gw, g["Rq"], g["sr"], g["sal"], out,
+                       workspace=ws)
+    assert_y_close(y_host(Y), y64, 1e-3 if out == torch.float32 else 1e-2)
+    Y2 = hq.w4a4_linear(g["Xq"], g["sx"], g["Wq"], g["sw"], g["zw"], gw, g["Rq"], g["sr"], g["sal"], out,
+                        workspace=ws)
+    assert torch.equal(Y, Y2)          # same workspace, counters were reset: identical bytes
+    assert int(ws.view(torch.int32)[: (N + 127) // 128].abs().sum()) == 0
     no_device_error()
 
 
@@ -267,7 +328,7 @@ def test_gemm_accumulators_many_tiles_per_cta(M, N, K, gw):
     t = _gemm_inputs(M, N, K, gw, 8, seed=4)
     acc_o, accc_o = O.accum(t["Xq"], K, t["Wq"], t["zw"], gw, t["Rq"], t["sal"])
     g = _dev_inputs(t)
-    acc, acc_c = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, g["Rq"], g["sal"])
+    acc, acc_c = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, g["Rq"], g["sal"], N)
     assert np.array_equal(host(acc).astype(np.int64), acc_o)
     assert np.array_equal(host(acc_c).astype(np.int64), accc_o)
 
@@ -298,7 +359,7 @@ def test_layer_end_to_end_from_raw_inputs(name, M, N):
     Xd = dev(X, wl.xdtype)
     layer = hq.W4A4Linear.prepare(dev(W, wl.wdtype), wl.g, wl.gw, wl.r, torch.from_numpy(d).cuda(),
                                   sal_idx=torch.from_numpy(ref["sal"]), out_dtype=out_dt)
-    assert np.array_equal(host(layer.Wq), ref["Wq"])
+    assert np.array_equal(untile_wq(host(layer.Wq), N), ref["Wq"])
     assert np.array_equal(f16bits(host(layer.sw)), f16bits(ref["sw"]))
     assert np.array_equal(host(layer.Rq), ref["Rq"])
     assert np.array_equal(f16bits(host(layer.sr)), f16bits(ref["sr"]))
@@ -327,7 +388,7 @@ def test_full_size_sampled_rows(name, M):
     out_dt = torch.float16 if wl.xdtype == "f16" else torch.bfloat16
     layer = hq.W4A4Linear.prepare(dev(W, wl.wdtype), wl.g, wl.gw, wl.r, torch.from_numpy(d).cuda(),
                                   sal_idx=torch.from_numpy(sal), out_dtype=out_dt)
-    assert np.array_equal(host(layer.Wq), Wq_o)
+    assert_same(untile_wq(host(layer.Wq), wl.N), Wq_o, "weight codes")
     assert np.array_equal(host(layer.Rq), Rq_o)
     Xd = dev(X, wl.xdtype)
     Xq, sx = hq.hq_rotate_quant(Xd, wl.g, layer.H_signs)
@@ -347,6 +408,6 @@ def test_bounded_wait_records_timeout_and_context_survives():
     assert hq.hq_last_device_status() == 0
     t = _gemm_inputs(16, 128, 256, 0, 8)
     g = _dev_inputs(t)
-    acc, _ = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], 0, g["Rq"], g["sal"])
+    acc, _ = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], 0, g["Rq"], g["sal"], 128)
     acc_o, _ = O.accum(t["Xq"], 256, t["Wq"], None, 0, t["Rq"], t["sal"])
     assert np.array_equal(host(acc).astype(np.int64), acc_o)

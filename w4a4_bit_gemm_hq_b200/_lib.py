@@ -33,6 +33,7 @@ _ST = ct.c_int  # hq_status
 SIGNATURES = {
     "hq_status_str": ([_ST], ct.c_char_p),
     "hq_device_sm_count": ([], ct.c_int),
+    "hq_packed_weight_bytes": ([_I64, _I64], ct.c_size_t),
     "hq_rotate_quant": ([_P, ct.c_int, _I64, _I64, _I64, _I32, _P, _P, _P, _P], _ST),
     "hq_rotate": ([_P, ct.c_int, _I64, _I64, _I32, _P, _P, _P], _ST),
     "hq_channel_sqnorm": ([_P, ct.c_int, _I64, _I64, _I32, _P, _P, _P], _ST),

@@ -86,7 +86,7 @@ extern "C" hq_status hq_debug_wait_probe(uint64_t limit_ns, void* stream) {
 }
 
 extern "C" size_t hq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group) {
-    if (M <= 0 || N <= 0 || K <= 0 || !small_supported(M)) return 0;
+    if (M <= 0 || N <= 0 || K <= 0 || !small_supported(M, group)) return 0;
     return small_workspace_bytes(M, N, K, group, sm_count());
 }
 
@@ -118,7 +118,7 @@ extern "C" hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, 
     a.Xq = Xq; a.sx = sx; a.Wq = Wq; a.sw = sw; a.zw = zw; a.Rq = A; a.sr = B; a.sal = sal_idx;
     a.Y = Y;
     a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
-    return run_gemm(a, yt, small_supported(M), workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+    return run_gemm(a, yt, small_supported(M, group), workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" hq_status hq_debug_accum(const uint8_t* Xq, int64_t M, int64_t K, const uint8_t* Wq, const uint16_t* zw,
@@ -129,8 +129,8 @@ extern "C" hq_status hq_debug_accum(const uint8_t* Xq, int64_t M, int64_t K, con
     if (s != HQ_OK) return s;
     if (M == 0 || N == 0) return HQ_OK;
     if (!acc || (r > 0 && !acc_c)) return HQ_ERR_ARG;
-    if (decode && !small_supported(M)) return HQ_ERR_UNSUPPORTED;
-    // the debug epilogue still reads the scales: give it harmless ones
+    if (decode && !small_supported(M, group)) return HQ_ERR_UNSUPPORTED;
+    // the debug epilogue stores raw accumulators and reads no scales
     GemmArgs a{};
     a.Xq = Xq; a.Wq = Wq; a.zw = zw; a.Rq = A; a.sal = sal_idx;
     a.dbg_acc = acc; a.dbg_acc_c = acc_c;

@@ -89,7 +89,7 @@ __device__ __forceinline__ void prod_load(const GemmArgs& p, int m0, int n0, int
             const int row = cj >> 2, c = cj & 3;
             const int n = n0 + row;
             if (n < p.N) {
-                R.d[j] = __ldg(reinterpret_cast<const uint4*>(p.Wq + n * kbytes + kb * 64 + c * 16));
+                R.d[j] = __ldg(reinterpret_cast<const uint4*>(p.Wq + wq_offset(n, kb * 64 + c * 16, p.K / 128)));
                 if constexpr (ASYM) {
                     const int b = (kb * pf::BK) / p.gw;
                     const float zf = __half2float(__ushort_as_half(p.zw[static_cast<int64_t>(b) * p.N + n]));

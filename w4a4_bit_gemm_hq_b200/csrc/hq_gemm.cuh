@@ -30,6 +30,6 @@ struct GemmArgs {
 hq_status launch_gemm_prefill(const GemmArgs& a, int out, cudaStream_t st, int nsm);
 hq_status launch_gemm_small(const GemmArgs& a, int out, cudaStream_t st, int nsm);
 size_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int gw, int nsm);
-bool small_supported(int64_t M);
+bool small_supported(int64_t M, int gw);
 
 }  // namespace hq

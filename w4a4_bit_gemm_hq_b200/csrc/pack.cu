@@ -40,13 +40,19 @@ __device__ __forceinline__ float warp_min(float v) {
 __device__ __forceinline__ uint16_t half_bits(float f) { return __half_as_ushort(__float2half_rn(f)); }
 __device__ __forceinline__ float bits_half(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
-// Per output channel symmetric: one warp per row.
+// Per output channel symmetric: one warp per row (rows N..Npad-1 of the last
+// tile are written as zero codes).
 template <int WT>
-__global__ void k_pack_sym(const void* __restrict__ W, int64_t N, int64_t K, uint8_t* __restrict__ Wq,
+__global__ void k_pack_sym(const void* __restrict__ W, int64_t N, int64_t Npad, int64_t K, uint8_t* __restrict__ Wq,
                            uint16_t* __restrict__ sw) {
     const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
-    if (n >= N) return;
+    const int64_t KB = K / 128;
+    if (n >= Npad) return;
+    if (n >= N) {
+        for (int64_t j = lane; j < K / 2; j += 32) Wq[wq_offset(n, j, KB)] = 0;
+        return;
+    }
     float amax = 0.f;
     for (int64_t k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(load_w<WT>(W, n * K + k)));
     amax = warp_max(amax);
@@ -62,21 +68,26 @@ __global__ void k_pack_sym(const void* __restrict__ W, int64_t N, int64_t K, uin
                 q[e] = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(w, s)), -8.f), 7.f));
             }
         }
-        Wq[n * (K / 2) + j] = static_cast<uint8_t>((q[0] & 0xF) | ((q[1] & 0xF) << 4));
+        Wq[wq_offset(n, j, KB)] = static_cast<uint8_t>((q[0] & 0xF) | ((q[1] & 0xF) << 4));
     }
 }
 
 // Per (channel, group) asymmetric over [min(lo,0), max(hi,0)]: one warp per
 // (row, group); scales and zero points are stored group-major [K/gw][N].
 template <int WT>
-__global__ void k_pack_asym(const void* __restrict__ W, int64_t N, int64_t K, int gw, uint8_t* __restrict__ Wq,
-                            uint16_t* __restrict__ sw, uint16_t* __restrict__ zw) {
+__global__ void k_pack_asym(const void* __restrict__ W, int64_t N, int64_t Npad, int64_t K, int gw,
+                            uint8_t* __restrict__ Wq, uint16_t* __restrict__ sw, uint16_t* __restrict__ zw) {
     const int64_t G = K / gw;
+    const int64_t KB = K / 128;
     const int64_t item = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
-    if (item >= N * G) return;
+    if (item >= Npad * G) return;
     const int64_t n = item / G, b = item % G;
     const int64_t k0 = b * gw;
+    if (n >= N) {
+        for (int j = lane; j < gw / 2; j += 32) Wq[wq_offset(n, k0 / 2 + j, KB)] = 0;
+        return;
+    }
     float lo = 0.f, hi = 0.f;
     for (int k = lane; k < gw; k += 32) {
         const float w = load_w<WT>(W, n * K + k0 + k);
@@ -101,7 +112,7 @@ __global__ void k_pack_asym(const void* __restrict__ W, int64_t N, int64_t K, in
             const float w = load_w<WT>(W, n * K + k0 + 2 * j + e);
             q[e] = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(w, s)) + z, 0.f), 15.f));
         }
-        Wq[n * (K / 2) + k0 / 2 + j] = static_cast<uint8_t>(q[0] | (q[1] << 4));
+        Wq[wq_offset(n, k0 / 2 + j, KB)] = static_cast<uint8_t>(q[0] | (q[1] << 4));
     }
 }
 
@@ -125,7 +136,7 @@ __global__ void k_serq_prepare(const float* __restrict__ Wrot, int64_t N, int64_
             float ev = 0.f;
             if (j < r) {
                 const int64_t k = sal[j];
-                const uint8_t byte = Wq[n * (K / 2) + k / 2];
+                const uint8_t byte = Wq[wq_offset(n, k / 2, K / 128)];
                 const int nib = (byte >> (4 * (k & 1))) & 0xF;
                 float what;
                 if (gw == 0) {
@@ -159,40 +170,44 @@ __global__ void k_serq_prepare(const float* __restrict__ Wrot, int64_t N, int64_
     }
 }
 
-static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace hq
 
 using namespace hq;
 
 extern "C" hq_status w4_pack(const void* W, hq_dtype wt, int64_t N, int64_t K, int32_t group, uint8_t* Wq,
                              uint16_t* sw, uint16_t* zw, void* stream) {
-    if (N < 0 || K <= 0 || (K & 1) || group < 0 || (group & 1)) return HQ_ERR_ARG;
+    if (N < 0 || K <= 0 || K % 128 != 0 || group < 0 || (group & 1)) return HQ_ERR_ARG;
     if (group > 0 && K % group != 0) return HQ_ERR_ARG;
     if (wt != HQ_F16 && wt != HQ_BF16 && wt != HQ_F32) return HQ_ERR_UNSUPPORTED;
     if (N == 0) return HQ_OK;
     if (!W || !Wq || !sw || (group > 0 && !zw)) return HQ_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int threads = 256, wpb = threads / 32;
+    const int64_t Npad = (N + 127) / 128 * 128;
     if (group == 0) {
-        const unsigned blocks = static_cast<unsigned>((N + wpb - 1) / wpb);
-        if (wt == HQ_F16) k_pack_sym<HQ_F16><<<blocks, threads, 0, st>>>(W, N, K, Wq, sw);
-        else if (wt == HQ_BF16) k_pack_sym<HQ_BF16><<<blocks, threads, 0, st>>>(W, N, K, Wq, sw);
-        else k_pack_sym<HQ_F32><<<blocks, threads, 0, st>>>(W, N, K, Wq, sw);
+        const unsigned blocks = static_cast<unsigned>((Npad + wpb - 1) / wpb);
+        if (wt == HQ_F16) k_pack_sym<HQ_F16><<<blocks, threads, 0, st>>>(W, N, Npad, K, Wq, sw);
+        else if (wt == HQ_BF16) k_pack_sym<HQ_BF16><<<blocks, threads, 0, st>>>(W, N, Npad, K, Wq, sw);
+        else k_pack_sym<HQ_F32><<<blocks, threads, 0, st>>>(W, N, Npad, K, Wq, sw);
     } else {
-        const int64_t items = N * (K / group);
+        const int64_t items = Npad * (K / group);
         const unsigned blocks = static_cast<unsigned>((items + wpb - 1) / wpb);
-        if (wt == HQ_F16) k_pack_asym<HQ_F16><<<blocks, threads, 0, st>>>(W, N, K, group, Wq, sw, zw);
-        else if (wt == HQ_BF16) k_pack_asym<HQ_BF16><<<blocks, threads, 0, st>>>(W, N, K, group, Wq, sw, zw);
-        else k_pack_asym<HQ_F32><<<blocks, threads, 0, st>>>(W, N, K, group, Wq, sw, zw);
+        if (wt == HQ_F16) k_pack_asym<HQ_F16><<<blocks, threads, 0, st>>>(W, N, Npad, K, group, Wq, sw, zw);
+        else if (wt == HQ_BF16) k_pack_asym<HQ_BF16><<<blocks, threads, 0, st>>>(W, N, Npad, K, group, Wq, sw, zw);
+        else k_pack_asym<HQ_F32><<<blocks, threads, 0, st>>>(W, N, Npad, K, group, Wq, sw, zw);
     }
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+extern "C" size_t hq_packed_weight_bytes(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0 || K % 128 != 0) return 0;
+    return static_cast<size_t>((N + 127) / 128 * 128) * static_cast<size_t>(K / 2);
 }
 
 extern "C" hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* Wq, const uint16_t* sw,
                                   const uint16_t* zw, int32_t group, const int32_t* sal_idx, int32_t r, uint8_t* Rq,
                                   uint16_t* sr, void* stream) {
-    if (N < 0 || K <= 0 || (K & 1) || r < 0 || r > 256 || r > K || group < 0) return HQ_ERR_ARG;
+    if (N < 0 || K <= 0 || K % 128 != 0 || r < 0 || r > 256 || r > K || group < 0) return HQ_ERR_ARG;
     if (group > 0 && K % group != 0) return HQ_ERR_ARG;
     if (N == 0) return HQ_OK;
     if (!W_rot || !Wq || !sw || !sr || (group > 0 && !zw) || (r > 0 && (!sal_idx || !Rq))) return HQ_ERR_ARG;

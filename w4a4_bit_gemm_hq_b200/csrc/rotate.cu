@@ -76,6 +76,10 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
     extern __shared__ float xch[];                   // [EPT][blockDim] exchange (G >= 2048)
     __shared__ float red[32];
 
+    // a kernel launched after this one with programmatic stream serialization
+    // (the small-M GEMM) may start now: it waits for this grid's completion
+    // before it reads the activation codes
+    asm volatile("griddepcontrol.launch_dependents;");
     const int t = threadIdx.x;
     const int nthr = blockDim.x;
     const int64_t tpr = K / EPT;

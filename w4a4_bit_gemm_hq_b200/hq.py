@@ -19,7 +19,7 @@ from ._lib import HQError, check, dtype_code, lib, ptr, stream_handle
 __all__ = [
     "HQError", "hq_rotate_quant", "hq_rotate", "hq_channel_sqnorm", "hq_select_salient", "w4_pack",
     "serq_prepare", "w4a4_linear", "hq_linear_workspace_size", "hq_debug_accum", "hq_last_device_status",
-    "hq_debug_wait_probe", "W4A4Linear",
+    "hq_debug_wait_probe", "hq_packed_weight_bytes", "wq_tile", "wq_untile", "W4A4Linear",
 ]
 
 
@@ -73,11 +73,32 @@ def hq_select_salient(norm2, r):
     return out
 
 
+def hq_packed_weight_bytes(N, K):
+    return int(lib.hq_packed_weight_bytes(N, K))
+
+
+def wq_tile(Wq_rows):
+    """Row-major packed weights [N, K/2] -> the tile-major layout of the C ABI,
+    shaped [ceil(N/128), K/128, 128, 64] (padding rows are zero)."""
+    N, Kh = Wq_rows.shape
+    T = (N + 127) // 128
+    pad = torch.zeros((T * 128, Kh), dtype=torch.uint8, device=Wq_rows.device)
+    pad[:N] = Wq_rows
+    return pad.view(T, 128, Kh // 64, 64).permute(0, 2, 1, 3).contiguous()
+
+
+def wq_untile(Wq, N):
+    """Tile-major packed weights -> row-major [N, K/2]."""
+    T, KB = Wq.shape[0], Wq.shape[1]
+    return Wq.permute(0, 2, 1, 3).reshape(T * 128, KB * 64)[:N]
+
+
 def w4_pack(W, group):
-    """(Wq uint8 [N, K/2], sw fp16 [N] or [K/group, N], zw fp16 [K/group, N] or None)."""
+    """(Wq uint8 tile-major [ceil(N/128), K/128, 128, 64], sw fp16 [N] or [K/group, N],
+    zw fp16 [K/group, N] or None)."""
     N, K = W.shape
     W = W.contiguous()
-    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    Wq = torch.empty(((N + 127) // 128, K // 128, 128, 64), dtype=torch.uint8, device=W.device)
     if group:
         sw = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
         zw = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
@@ -105,10 +126,11 @@ def hq_linear_workspace_size(M, N, K, group):
 
 
 def w4a4_linear(Xq, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat16, Y=None, workspace=None):
-    """Y [M, N] = sx * (sum_b sw * acc_b + sr * acc_c), one fused launch."""
+    """Y [M, N] = sx * (sum_b sw * acc_b + sr * acc_c), one fused launch.
+    N is taken from the scales (sw [N] or [K/group, N])."""
     M = Xq.shape[0]
     K = Xq.shape[1] * 2
-    N = Wq.shape[0]
+    N = sw.shape[-1]
     r = 0 if sal_idx is None else int(sal_idx.numel())
     if Y is None:
         Y = torch.empty((M, N), dtype=out_dtype, device=Xq.device)
@@ -122,11 +144,10 @@ def w4a4_linear(Xq, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat
     return Y
 
 
-def hq_debug_accum(Xq, Wq, zw, group, A, sal_idx, decode=False, workspace=None):
+def hq_debug_accum(Xq, Wq, zw, group, A, sal_idx, N, decode=False, workspace=None):
     """Exact int32 accumulators of the GEMM kernel: (acc [M, N, G], acc_c [M, N])."""
     M = Xq.shape[0]
     K = Xq.shape[1] * 2
-    N = Wq.shape[0]
     r = 0 if sal_idx is None else int(sal_idx.numel())
     G = K // group if group else 1
     acc = torch.zeros((M, N, G), dtype=torch.int32, device=Xq.device)
