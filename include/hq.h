@@ -212,6 +212,38 @@ hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,
                       void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * w4a4_linear_noalloc -- w4a4_linear for callers that cannot allocate device
+ * memory when they call it.  The pages have no counterpart: this is a service
+ * of the library, not a step of the method.
+ *
+ * w4a4_linear asks its caller for a workspace whenever it uses the small-M
+ * (decode, M <= 64) kernel, which needs scratch for the per-tile arrival
+ * counters and partial sums of weight tiles split across SMs.  Runtimes that
+ * plan all their device buffers once at start-up and forbid allocating later,
+ * or whose memory pool is exhausted, cannot provide it.  This entry point takes
+ * the same arguments minus the workspace and uses a fixed scratch array of
+ * 8 MiB that lives in the library itself (every GPU that loads the library
+ * holds it until the process exits); the call allocates nothing.
+ *
+ *  - The first call on a device looks up the array's device address (a set-up
+ *    step done once per device, with that device current); make that first
+ *    call before any stream capture.
+ *  - All calls share the one array and it keeps the previous call's contents:
+ *    each call first clears the arrival counters (an asynchronous memset on
+ *    `stream`).  Calls that overlap on the GPU (different streams, or several
+ *    host threads) race on the array and must not be issued.
+ *  - Shapes whose scratch would exceed 8 MiB (hq_linear_workspace_size(M, N,
+ *    K, group) > 8 MiB) are rejected with HQ_ERR_UNSUPPORTED before anything
+ *    is enqueued.  Large M (> 64) uses the large-M kernel, which needs no
+ *    scratch.
+ * Arguments, results and the other errors are those of w4a4_linear.
+ */
+hq_status w4a4_linear_noalloc(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,
+                              const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
+                              int32_t group, const uint8_t* A, const uint16_t* B,
+                              const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt, void* stream);
+
+/*
  * hq_debug_accum -- test hook: runs the GEMM kernel of w4a4_linear with the
  * epilogue replaced by a raw store of the exact integer accumulators.
  *  acc     device, int32 [M][N][G] with G = K/group (1 when group == 0)

@@ -43,6 +43,7 @@ SIGNATURES = {
     "hq_linear_workspace_size": ([_I64, _I64, _I64, _I32], ct.c_size_t),
     "w4a4_linear": ([_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _P, ct.c_int, _P,
                      ct.c_size_t, _P], _ST),
+    "w4a4_linear_noalloc": ([_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _P, ct.c_int, _P], _ST),
     "hq_debug_accum": ([_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32, _P, ct.c_size_t, _P],
                        _ST),
     "hq_last_device_status": ([_P], _ST),
