@@ -44,78 +44,102 @@ constexpr int THREADS = 512;
 constexpr int MMA_WARP = 4;
 constexpr int EPI_WARP0 = 8;
 constexpr int NPROD = 7 * 32;         // producer threads: warps 0-3 and 5-7
-constexpr int STAGES = 4;
 constexpr int RQ_LD = 64;             // bytes per unpacked Rq row (r <= 64) in the per-warp scratch
 }  // namespace pf
 
-template <int BN>
+// Shared memory: an int8 operand ring read by the tensor core (STAGES deep) and
+// a packed-code ring (PD deep) that each producer thread fills with cp.async
+// for its own 16-byte chunks (and, for group weights, the zero-point pair of
+// its weight row), PD stages ahead of their use.
+template <int BN, bool ASYM>
 struct PfSmem {
+    static constexpr int STAGES = (BN == 256) ? 2 : 3;
+    static constexpr int PD = (BN == 256) ? 4 : 5;
     static constexpr int A_BYTES = pf::BM * pf::BK;
     static constexpr int B_BYTES = BN * pf::BK;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int OFF_RQ = pf::STAGES * STAGE;                 // 8 warps x 32 rows x RQ_LD
-    static constexpr int OFF_SAL = OFF_RQ + 8 * 32 * pf::RQ_LD;       // int32[128]
+    static constexpr int NCHUNK = (pf::BM + BN) * 4;                   // 16-byte packed chunks per stage
+    static constexpr int NCH = (NCHUNK + pf::NPROD - 1) / pf::NPROD;  // per producer thread
+    static constexpr int PK_DATA = NCHUNK * 16;
+    static constexpr int PK_Z = ASYM ? BN * 4 * 4 : 0;                 // zero-point pair per weight chunk
+    static constexpr int PK_STAGE = ((PK_DATA + PK_Z) + 127) / 128 * 128;
+    static constexpr int OFF_PK = STAGES * STAGE;
+    static constexpr int OFF_RQ = OFF_PK + PD * PK_STAGE;              // 8 warps x 32 rows x RQ_LD
+    static constexpr int OFF_SAL = OFF_RQ + 8 * 32 * pf::RQ_LD;        // int32[128]
     static constexpr int OFF_BAR = OFF_SAL + 128 * 4;
-    static constexpr int NBAR = 2 * pf::STAGES + 4 + 1;
+    static constexpr int NBAR = 2 * STAGES + 4 + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16;
-    static constexpr int ALLOC = BYTES + 1024;                        // 1024-byte alignment slack
+    static constexpr int ALLOC = BYTES + 1024;                         // 1024-byte alignment slack
 };
 
 __device__ __forceinline__ uint32_t swz_chunk(int row, int chunk) { return static_cast<uint32_t>(chunk ^ (row & 7)); }
 
-// Producer: the 16-byte packed chunks of one stage, prefetched to registers.
-template <int BN, int NCH>
-struct ProdRegs {
-    uint4 d[NCH];
-    uint32_t z[NCH];
-};
+// 16-byte (4-byte) async copies that zero-fill when `valid` is false.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(valid ? 4 : 0)
+                 : "memory");
+}
 
+// Producer thread `pi`: issue the async copies of its chunks of one stage
+// (tile m0/n0, K-block kb) into packed slot `pk` (smem address).
 template <int BN, bool ASYM>
-__device__ __forceinline__ void prod_load(const GemmArgs& p, int m0, int n0, int kb, int pi, ProdRegs<BN, (((pf::BM + BN) * 4) + pf::NPROD - 1) / pf::NPROD>& R) {
-    constexpr int NCH = (((pf::BM + BN) * 4) + pf::NPROD - 1) / pf::NPROD;
+__device__ __forceinline__ void prod_issue(const GemmArgs& p, int m0, int n0, int kb, int pi, uint32_t pk) {
+    using L = PfSmem<BN, ASYM>;
     const int64_t kbytes = static_cast<int64_t>(p.K) / 2;
 #pragma unroll
-    for (int j = 0; j < NCH; ++j) {
+    for (int j = 0; j < L::NCH; ++j) {
         const int ci = pi + j * pf::NPROD;
-        R.d[j] = make_uint4(0, 0, 0, 0);
-        R.z[j] = 0;
+        if (ci >= L::NCHUNK) continue;
         if (ci < pf::BM * 4) {
             const int row = ci >> 2, c = ci & 3;
             const int m = m0 + row;
-            if (m < p.M) R.d[j] = __ldg(reinterpret_cast<const uint4*>(p.Xq + m * kbytes + kb * 64 + c * 16));
-        } else if (ci < (pf::BM + BN) * 4) {
+            const bool ok = m < p.M;
+            cp_async16_zfill(pk + ci * 16, ok ? p.Xq + m * kbytes + kb * 64 + c * 16 : p.Xq, ok);
+        } else {
             const int cj = ci - pf::BM * 4;
             const int row = cj >> 2, c = cj & 3;
             const int n = n0 + row;
-            if (n < p.N) {
-                R.d[j] = __ldg(reinterpret_cast<const uint4*>(p.Wq + wq_offset(n, kb * 64 + c * 16, p.K / 128)));
-                if constexpr (ASYM) {
-                    const int b = (kb * pf::BK) / p.gw;
-                    const float zf = __half2float(__ushort_as_half(p.zw[static_cast<int64_t>(b) * p.N + n]));
-                    R.z[j] = static_cast<uint32_t>(zf) * 0x01010101u;
-                }
+            const bool ok = n < p.N;
+            cp_async16_zfill(pk + ci * 16, ok ? p.Wq + wq_offset(n, kb * 64 + c * 16, p.K / 128) : p.Wq, ok);
+            if constexpr (ASYM) {
+                const int b = (kb * pf::BK) / p.gw;
+                cp_async4_zfill(pk + L::PK_DATA + cj * 4, ok ? p.zw + static_cast<int64_t>(b) * p.N + (n & ~1) : p.zw,
+                                ok);
             }
         }
     }
 }
 
+// Producer thread `pi`: its packed chunks of one stage (slot `pk`, generic
+// pointer) -> int8 operand tiles of the stage.
 template <int BN, bool ASYM>
-__device__ __forceinline__ void prod_store(uint8_t* stage, int pi, const ProdRegs<BN, (((pf::BM + BN) * 4) + pf::NPROD - 1) / pf::NPROD>& R) {
-    constexpr int NCH = (((pf::BM + BN) * 4) + pf::NPROD - 1) / pf::NPROD;
+__device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, int pi) {
+    using L = PfSmem<BN, ASYM>;
 #pragma unroll
-    for (int j = 0; j < NCH; ++j) {
+    for (int j = 0; j < L::NCH; ++j) {
         const int ci = pi + j * pf::NPROD;
-        if (ci >= (pf::BM + BN) * 4) continue;
+        if (ci >= L::NCHUNK) continue;
         const bool isA = ci < pf::BM * 4;
         const int cl = isA ? ci : ci - pf::BM * 4;
         const int row = cl >> 2, c = cl & 3;
-        uint8_t* base = stage + (isA ? 0 : PfSmem<BN>::A_BYTES) + row * 128;
+        const uint4 d = *reinterpret_cast<const uint4*>(pk + ci * 16);
+        uint8_t* base = stage + (isA ? 0 : L::A_BYTES) + row * 128;
         uint32_t o[8];
-        const uint32_t w[4] = {R.d[j].x, R.d[j].y, R.d[j].z, R.d[j].w};
+        const uint32_t w[4] = {d.x, d.y, d.z, d.w};
         if (!isA && ASYM) {
+            // zero point of weight row n = (n0 + row): half (row & 1) of the copied pair
+            const uint32_t zp = *reinterpret_cast<const uint32_t*>(pk + L::PK_DATA + cl * 4);
+            const uint16_t zh = static_cast<uint16_t>((row & 1) ? (zp >> 16) : (zp & 0xFFFFu));
+            const uint32_t z4 = static_cast<uint32_t>(__half2float(__ushort_as_half(zh))) * 0x01010101u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) unpack_u4x8_minus_z(w[e], R.z[j], o[2 * e], o[2 * e + 1]);
+            for (int e = 0; e < 4; ++e) unpack_u4x8_minus_z(w[e], z4, o[2 * e], o[2 * e + 1]);
         } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e) unpack_s4x8_times16(w[e], o[2 * e], o[2 * e + 1]);
@@ -260,7 +284,8 @@ __device__ __forceinline__ void load_h32(const uint16_t* src, float (&o)[32]) {
 // OUT: HQ_F16 / HQ_BF16 / HQ_F32, or OUT_DEBUG for raw accumulators.
 template <int BN, bool ASYM, int OUT>
 __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
-    using L = PfSmem<BN>;
+    using L = PfSmem<BN, ASYM>;
+    constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -268,10 +293,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (pf::STAGES + s); };
-    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * pf::STAGES + b); };
-    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * pf::STAGES + 2 + b); };
-    const uint32_t done_bar = bar0 + 8u * (2 * pf::STAGES + 4);
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
     int32_t* sal_s = reinterpret_cast<int32_t*>(smem + L::OFF_SAL);
 
@@ -284,7 +309,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
     constexpr uint32_t TMEM_COLS = 2 * BN;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < pf::STAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), pf::NPROD);
             mbar_init(empty_bar(s), 1);
         }
@@ -308,28 +333,30 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
     if (warp < pf::EPI_WARP0 && warp != pf::MMA_WARP) {
         // ======================= producers
         const int pi = (warp < pf::MMA_WARP ? warp : warp - 1) * 32 + lane;
-        constexpr int NCH = (((pf::BM + BN) * 4) + pf::NPROD - 1) / pf::NPROD;
-        ProdRegs<BN, NCH> cur, nxt;
+        const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        const int items = my_tiles * KB;
+        const uint32_t pk0 = smem_u32(smem + L::OFF_PK);
+        auto issue = [&](int item) {
+            if (item < items) {
+                const int tile = blockIdx.x + (item / KB) * gridDim.x;
+                prod_issue<BN, ASYM>(p, (tile % MT) * pf::BM, (tile / MT) * BN, item % KB, pi,
+                                     pk0 + (item % L::PD) * L::PK_STAGE);
+            }
+            cp_async_commit();   // one group per stage (possibly empty)
+        };
+        for (int d = 0; d < L::PD; ++d) issue(d);
         int stage = 0;
         uint32_t phase = 0;
-        bool ok = true;
-        int tile = blockIdx.x, kb = 0;
-        if (tile < num_tiles)
-            prod_load<BN, ASYM>(p, (tile % MT) * pf::BM, (tile / MT) * BN, 0, pi, cur);
-        while (ok && tile < num_tiles) {
-            int ntile = tile, nkb = kb + 1;
-            if (nkb == KB) { nkb = 0; ntile += gridDim.x; }
-            if (ntile < num_tiles)
-                prod_load<BN, ASYM>(p, (ntile % MT) * pf::BM, (ntile / MT) * BN, nkb, pi, nxt);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, p.limit_ns))) { ok = false; break; }
-            prod_store<BN, ASYM>(smem + stage * L::STAGE, pi, cur);
+        for (int item = 0; item < items; ++item) {
+            cp_async_wait_group<L::PD - 1>();      // this thread's chunks of `item` have landed
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, p.limit_ns))) break;
+            prod_unpack<BN, ASYM>(smem + L::OFF_PK + (item % L::PD) * L::PK_STAGE, smem + stage * L::STAGE, pi);
+            issue(item + L::PD);                   // refill the packed slot just read
             fence_proxy_async_smem();
             mbar_arrive(full_bar(stage));
-            if (++stage == pf::STAGES) { stage = 0; phase ^= 1u; }
-            cur = nxt;
-            tile = ntile;
-            kb = nkb;
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        cp_async_wait_all();   // nothing in flight when the CTA exits
     } else if (warp == pf::MMA_WARP) {
         // ======================= MMA issuer
         if (lane == 0) {
@@ -356,7 +383,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
                     for (int kk = 0; kk < pf::BK / 32; ++kk)
                         mma_i8_ss(dcol, adesc + 2u * kk, bdesc + 2u * kk, IDESC, (first && kk == 0) ? 0u : 1u);
                     tc_commit(empty_bar(stage));
-                    if (++stage == pf::STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     if ((kb % GPK) == GPK - 1) {
                         tc_commit(accf_bar(abuf));
                         aphase ^= 1u << abuf;
@@ -519,7 +546,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
 template <int BN, bool ASYM, int OUT>
 static hq_status launch_pf_t(const GemmArgs& a, cudaStream_t st, int nsm) {
     auto kern = k_gemm_pf<BN, ASYM, OUT>;
-    const int smem = PfSmem<BN>::ALLOC;
+    const int smem = PfSmem<BN, ASYM>::ALLOC;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
     const int tiles = ((a.M + pf::BM - 1) / pf::BM) * ((a.N + BN - 1) / BN);

@@ -86,47 +86,53 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
     const bool active = t < tpr;
     const int64_t col0 = static_cast<int64_t>(t) * EPT;
 
-    // Sign words of d for this thread's channels, in the bit positions of the
-    // element sign: XT 16-bit -> bits 15 / 31 of a packed pair; f32 -> bit 31.
-    uint32_t sgn[EPT / 2];
-#pragma unroll
-    for (int i = 0; i < EPT / 2; ++i) sgn[i] = 0;
+    // Signs of d for this thread's channels: bit i set = flip channel col0 + i.
+    uint32_t smask = 0;
     float accsq[MODE == MODE_SQNORM ? EPT : 1];
 #pragma unroll
     for (int i = 0; i < (MODE == MODE_SQNORM ? EPT : 1); ++i) accsq[i] = 0.f;
     if (active && dsign != nullptr) {
         const int p0 = static_cast<int>(col0 % G);
 #pragma unroll
-        for (int i = 0; i < EPT; i += 2) {
-            const int8_t d0 = dsign[(p0 + i) % G];
-            const int8_t d1 = dsign[(p0 + i + 1) % G];
-            sgn[i / 2] = (d0 == -1 ? 0x8000u : 0u) | (d1 == -1 ? 0x80000000u : 0u);
-        }
+        for (int i = 0; i < EPT; ++i) smask |= (dsign[(p0 + i) % G] == -1 ? 1u : 0u) << i;
     }
 
+    // raw 16-byte words of this thread's channels, loaded one row ahead so that
+    // the next row's HBM latency hides under this row's butterfly
+    constexpr int NRAW = (XT == XT_F32) ? EPT / 4 : EPT / 8;
+    uint4 raw[NRAW], raw_next[NRAW];
+    auto load_row = [&](int64_t m, uint4 (&r)[NRAW]) {
+        if (active && m < M) {
+            const uint4* src = (XT == XT_F32)
+                                   ? reinterpret_cast<const uint4*>(static_cast<const float*>(X) + m * ldx + col0)
+                                   : reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + m * ldx + col0);
+#pragma unroll
+            for (int j = 0; j < NRAW; ++j) r[j] = __ldg(src + j);
+        }
+    };
+    load_row(blockIdx.x, raw);
     for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+        load_row(m + gridDim.x, raw_next);
         float2 v[EPT / 2];
         if (active) {
             if constexpr (XT == XT_F32) {
-                const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(X) + m * ldx + col0);
 #pragma unroll
                 for (int j = 0; j < EPT / 4; ++j) {
-                    float4 f = __ldg(src + j);
-                    uint32_t s0 = sgn[2 * j], s1 = sgn[2 * j + 1];
-                    v[2 * j].x = __uint_as_float(__float_as_uint(f.x) ^ (s0 << 16));
-                    v[2 * j].y = __uint_as_float(__float_as_uint(f.y) ^ (s0 & 0x80000000u));
-                    v[2 * j + 1].x = __uint_as_float(__float_as_uint(f.z) ^ (s1 << 16));
-                    v[2 * j + 1].y = __uint_as_float(__float_as_uint(f.w) ^ (s1 & 0x80000000u));
+                    const uint4 f = raw[j];
+                    v[2 * j].x = __uint_as_float(f.x ^ (((smask >> (4 * j)) & 1u) << 31));
+                    v[2 * j].y = __uint_as_float(f.y ^ (((smask >> (4 * j + 1)) & 1u) << 31));
+                    v[2 * j + 1].x = __uint_as_float(f.z ^ (((smask >> (4 * j + 2)) & 1u) << 31));
+                    v[2 * j + 1].y = __uint_as_float(f.w ^ (((smask >> (4 * j + 3)) & 1u) << 31));
                 }
             } else {
-                const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + m * ldx + col0);
 #pragma unroll
                 for (int j = 0; j < EPT / 8; ++j) {
-                    uint4 q = __ldg(src + j);
+                    const uint4 q = raw[j];
                     uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const uint32_t x = w[e] ^ sgn[4 * j + e];
+                        const int i0 = 8 * j + 2 * e;   // channel of the pair's low half
+                        const uint32_t x = w[e] ^ (((smask >> i0) & 1u) << 15) ^ (((smask >> (i0 + 1)) & 1u) << 31);
                         if constexpr (XT == XT_BF16) {
                             v[4 * j + e].x = __uint_as_float(x << 16);
                             v[4 * j + e].y = __uint_as_float(x & 0xFFFF0000u);
@@ -258,6 +264,8 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
             }
             if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
         }
+#pragma unroll
+        for (int j = 0; j < NRAW; ++j) raw[j] = raw_next[j];
     }
 
     if constexpr (MODE == MODE_SQNORM) {
