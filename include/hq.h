@@ -200,7 +200,8 @@ hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* 
  *           that size is 0).  Zero it once before its first use; every call
  *           leaves it zeroed again.  Calls that share a workspace must not
  *           overlap in time.
- * Requirements: K % 128 == 0, 0 < K <= 65536, N % 8 == 0.
+ * Requirements: K % 128 == 0, 0 < K <= 65536, N % 8 == 0; Xq, Wq, sw, zw,
+ * B, Y and workspace 16-byte aligned, A 4-byte aligned (HQ_ERR_ALIGN).
  * Errors: HQ_ERR_ARG, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA.
  */
 size_t hq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group);

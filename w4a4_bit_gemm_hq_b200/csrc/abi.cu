@@ -48,7 +48,7 @@ static hq_status check_gemm(const uint8_t* Xq, int64_t M, int64_t K, const uint8
     if (M == 0 || N == 0) return HQ_OK;
     if (!Xq || !Wq || (group > 0 && !zw)) return HQ_ERR_ARG;
     if (r > 0 && (!A || !sal)) return HQ_ERR_ARG;
-    if (!al16(Xq) || !al16(Wq)) return HQ_ERR_ALIGN;
+    if (!al16(Xq) || !al16(Wq) || (group > 0 && !al16(zw))) return HQ_ERR_ALIGN;
     if (r > 0 && (reinterpret_cast<uintptr_t>(A) & 3u)) return HQ_ERR_ALIGN;
     return HQ_OK;
 }

@@ -10,8 +10,12 @@
 // Quantization by Offsetting", Methodology 3 (group-wise scale and zero point).
 //
 // Design (one CTA per SM, persistent over 128 x BN output tiles):
-//  * tcgen05 has no int4 MMA, so 7 producer warps read the packed codes with
-//    16-byte loads (prefetched one stage ahead in registers), expand them to
+//  * one thread moves the packed codes of each K-block into a ring of packed
+//    slots with the tensor memory accelerator: a 2D tensor-map load of the 128
+//    activation rows (64 bytes each; rows past M read as zero) and 8 KB bulk
+//    copies of the tile-major weight blocks (plus the zero points of the
+//    block's group for group weights).
+//  * tcgen05 has no int4 MMA, so 6 producer warps expand the packed codes to
 //    int8 in registers (16*q for activations and symmetric weights, u - z for
 //    asymmetric weights) and store them into 128-byte-swizzled K-major smem
 //    tiles: A = 128 activation rows x 128 K, B = BN weight rows x 128 K.
@@ -28,6 +32,9 @@
 //    HQ_ERR_TIMEOUT and the roles skip to teardown, which waits for in-flight
 //    MMAs before freeing tensor memory.
 #include <cstdint>
+#include <mutex>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -41,16 +48,23 @@ namespace pf {
 constexpr int BM = 128;
 constexpr int BK = 128;               // int8 K per stage = one 128-byte swizzle row
 constexpr int THREADS = 512;
-constexpr int MMA_WARP = 4;
-constexpr int EPI_WARP0 = 8;
-constexpr int NPROD = 7 * 32;         // producer threads: warps 0-3 and 5-7
-constexpr int RQ_LD = 64;             // bytes per unpacked Rq row (r <= 64) in the per-warp scratch
+constexpr int TMA_WARP = 0;           // lane 0 issues the packed-code copies
+constexpr int MMA_WARP = 1;           // lane 0 issues tcgen05.mma; the warp owns TMEM
+constexpr int PROD_WARP0 = 2;         // warps 2-7 expand codes to int8
+constexpr int NPROD_WARPS = 6;
+constexpr int NPROD = NPROD_WARPS * 32;
+constexpr int EPI_WARP0 = 8;          // warps 8-15: epilogue
+constexpr int PK_ROW = 64;            // packed bytes of one row of a K-block
+constexpr int RQ_LD = 64;             // bytes per unpacked Rq row (r <= 64) in the per-tile staging
+constexpr int EPI_THREADS = 256;
+constexpr uint32_t EPI_BAR = 1;       // named barrier of the epilogue warps
 }  // namespace pf
 
 // Shared memory: an int8 operand ring read by the tensor core (STAGES deep) and
-// a packed-code ring (PD deep) that each producer thread fills with cp.async
-// for its own 16-byte chunks (and, for group weights, the zero-point pair of
-// its weight row), PD stages ahead of their use.
+// a ring of packed slots (PD deep) filled by the copy engine.  A packed slot
+// holds the 128 activation rows (64 bytes each), the BN weight rows in the
+// order of the tile-major layout (128-row blocks of 8 KB) and, for group
+// weights, the BN fp16 zero points of the block's group.
 template <int BN, bool ASYM>
 struct PfSmem {
     static constexpr int STAGES = (BN == 256) ? 2 : 3;
@@ -60,65 +74,29 @@ struct PfSmem {
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int NCHUNK = (pf::BM + BN) * 4;                   // 16-byte packed chunks per stage
     static constexpr int NCH = (NCHUNK + pf::NPROD - 1) / pf::NPROD;  // per producer thread
-    static constexpr int PK_DATA = NCHUNK * 16;
-    static constexpr int PK_Z = ASYM ? BN * 4 * 4 : 0;                 // zero-point pair per weight chunk
-    static constexpr int PK_STAGE = ((PK_DATA + PK_Z) + 127) / 128 * 128;
+    static constexpr int PK_A = pf::BM * pf::PK_ROW;
+    static constexpr int PK_B = BN * pf::PK_ROW;
+    static constexpr int PK_Z = ASYM ? BN * 2 : 0;
+    static constexpr int PK_STAGE = ((PK_A + PK_B + PK_Z) + 127) / 128 * 128;
     static constexpr int OFF_PK = STAGES * STAGE;
-    static constexpr int OFF_RQ = OFF_PK + PD * PK_STAGE;              // 8 warps x 32 rows x RQ_LD
-    static constexpr int OFF_SAL = OFF_RQ + 8 * 32 * pf::RQ_LD;        // int32[128]
+    static constexpr int OFF_RQ = OFF_PK + PD * PK_STAGE;              // tile's Rq rows, BN x RQ_LD int8
+    static constexpr int OFF_SW = OFF_RQ + BN * pf::RQ_LD;             // float [2][BN]: sw of the tile (of a group)
+    static constexpr int OFF_SR = OFF_SW + 2 * BN * 4;                 // float [BN]
+    static constexpr int OFF_SAL = OFF_SR + BN * 4;                    // int32[128]
     static constexpr int OFF_BAR = OFF_SAL + 128 * 4;
-    static constexpr int NBAR = 2 * STAGES + 4 + 1;
+    static constexpr int NBAR = 2 * STAGES + 2 * PD + 4 + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16;
     static constexpr int ALLOC = BYTES + 1024;                         // 1024-byte alignment slack
+    static_assert(ALLOC <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ uint32_t swz_chunk(int row, int chunk) { return static_cast<uint32_t>(chunk ^ (row & 7)); }
 
-// 16-byte (4-byte) async copies that zero-fill when `valid` is false.
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
-                 "r"(valid ? 4 : 0)
-                 : "memory");
-}
-
-// Producer thread `pi`: issue the async copies of its chunks of one stage
-// (tile m0/n0, K-block kb) into packed slot `pk` (smem address).
-template <int BN, bool ASYM>
-__device__ __forceinline__ void prod_issue(const GemmArgs& p, int m0, int n0, int kb, int pi, uint32_t pk) {
-    using L = PfSmem<BN, ASYM>;
-    const int64_t kbytes = static_cast<int64_t>(p.K) / 2;
-#pragma unroll
-    for (int j = 0; j < L::NCH; ++j) {
-        const int ci = pi + j * pf::NPROD;
-        if (ci >= L::NCHUNK) continue;
-        if (ci < pf::BM * 4) {
-            const int row = ci >> 2, c = ci & 3;
-            const int m = m0 + row;
-            const bool ok = m < p.M;
-            cp_async16_zfill(pk + ci * 16, ok ? p.Xq + m * kbytes + kb * 64 + c * 16 : p.Xq, ok);
-        } else {
-            const int cj = ci - pf::BM * 4;
-            const int row = cj >> 2, c = cj & 3;
-            const int n = n0 + row;
-            const bool ok = n < p.N;
-            cp_async16_zfill(pk + ci * 16, ok ? p.Wq + wq_offset(n, kb * 64 + c * 16, p.K / 128) : p.Wq, ok);
-            if constexpr (ASYM) {
-                const int b = (kb * pf::BK) / p.gw;
-                cp_async4_zfill(pk + L::PK_DATA + cj * 4, ok ? p.zw + static_cast<int64_t>(b) * p.N + (n & ~1) : p.zw,
-                                ok);
-            }
-        }
-    }
-}
-
 // Producer thread `pi`: its packed chunks of one stage (slot `pk`, generic
-// pointer) -> int8 operand tiles of the stage.
+// pointer) -> int8 operand tiles of the stage.  Chunk ci covers packed bytes
+// [16 ci, 16 ci + 16) of the slot: activation row ci / 4 for ci < 512, else
+// weight row (ci - 512) / 4, K bytes 16 (ci % 4) onwards.
 template <int BN, bool ASYM>
 __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, int pi) {
     using L = PfSmem<BN, ASYM>;
@@ -134,10 +112,9 @@ __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, i
         uint32_t o[8];
         const uint32_t w[4] = {d.x, d.y, d.z, d.w};
         if (!isA && ASYM) {
-            // zero point of weight row n = (n0 + row): half (row & 1) of the copied pair
-            const uint32_t zp = *reinterpret_cast<const uint32_t*>(pk + L::PK_DATA + cl * 4);
-            const uint16_t zh = static_cast<uint16_t>((row & 1) ? (zp >> 16) : (zp & 0xFFFFu));
-            const uint32_t z4 = static_cast<uint32_t>(__half2float(__ushort_as_half(zh))) * 0x01010101u;
+            // zero point of weight row n0 + row, an integer in [0, 15] stored as fp16
+            const uint16_t zh = *reinterpret_cast<const uint16_t*>(pk + L::PK_A + L::PK_B + row * 2);
+            const uint32_t z4 = (static_cast<uint32_t>(__half2float(__ushort_as_half(zh))) & 0xFu) * 0x01010101u;
 #pragma unroll
             for (int e = 0; e < 4; ++e) unpack_u4x8_minus_z(w[e], z4, o[2 * e], o[2 * e + 1]);
         } else {
@@ -150,41 +127,55 @@ __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, i
 }
 
 // Gathered salient activation codes of row m as int8 words in the lo/hi
-// permutation of unpack_s4x8_times16 (plain codes, not scaled by 16).
+// permutation of unpack_s4x8_times16 (plain codes, not scaled by 16):
+// position j = 8 i + 2 e + h -> word 2 i + h, byte e.  Eight loads in flight
+// per batch of eight positions (r is a multiple of 8).
 __device__ __forceinline__ void gather_xs(const GemmArgs& p, const int32_t* sal_s, int m, uint32_t (&xs)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) xs[i] = 0;
-    if (m >= p.M) return;
+    if (m >= p.M || p.r == 0) return;
     const uint8_t* row = p.Xq + static_cast<int64_t>(m) * (p.K / 2);
-    for (int j = 0; j < p.r; ++j) {
-        const int k = sal_s[j];
-        const int nib = (__ldg(row + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
-        const uint32_t code = static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu;
-        // position j = 8*i + 2*e + h  ->  word 2*i + h, byte e
-        const int i = j >> 3, e = (j >> 1) & 3, h = j & 1;
-        const uint32_t sh = 8u * e;
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-            if (q == 2 * i + h) xs[q] |= code << sh;
+    for (int i = 0; i < 8; ++i) {
+        if (8 * i >= p.r) break;
+        uint32_t nib[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int k = sal_s[8 * i + t];
+            nib[t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const uint32_t code = static_cast<uint32_t>(static_cast<int>(nib[t] ^ 8u) - 8) & 0xFFu;
+            xs[2 * i + (t & 1)] |= code << (8 * (t >> 1));
+        }
     }
 }
 
-// Unpacks Rq rows of the warp's 32 columns into the warp's smem scratch:
-// lane l -> row l, r/8 words -> r/4 words (16 * code), lo/hi permutation.
-__device__ __forceinline__ void stage_rq(const GemmArgs& p, uint8_t* scratch, int n_first, int lane) {
-    const int n = n_first + lane;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(scratch + lane * pf::RQ_LD);
-    const int words = p.r / 8;
-    if (n < p.N) {
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(p.Rq + static_cast<int64_t>(n) * (p.r / 2));
-        for (int i = 0; i < words; ++i) {
-            uint32_t lo, hi;
-            unpack_s4x8_times16(__ldg(src + i), lo, hi);
-            dst[2 * i] = lo;
-            dst[2 * i + 1] = hi;
-        }
-    } else {
-        for (int i = 0; i < 2 * words; ++i) dst[i] = 0;
+// Column data of output column n for one tile, staged by one epilogue thread:
+// sw (per channel, or of group 0) and sr as float, and the SERQ row Rq[n]
+// unpacked to r int8 values (16 * code, lo/hi permutation).  Columns past N
+// stage zeros.
+template <int OUT>
+__device__ __forceinline__ void stage_column(const GemmArgs& p, int n, float* sw_d, float* sr_d, uint8_t* rq_d) {
+    const bool nv = n < p.N;
+    if constexpr (OUT != OUT_DEBUG) {
+        *sw_d = nv ? __half2float(__ushort_as_half(__ldg(p.sw + n))) : 0.f;
+        *sr_d = (nv && p.r > 0) ? __half2float(__ushort_as_half(__ldg(p.sr + n))) : 0.f;
+    }
+    if (p.r == 0) return;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.Rq + static_cast<int64_t>(nv ? n : 0) * (p.r / 2));
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = (nv && 8 * i < p.r) ? __ldg(src + i) : 0u;
+    uint4* dst = reinterpret_cast<uint4*>(rq_d);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (16 * i >= p.r) break;   // words 2i and 2i+1 hold codes 16i .. 16i+15
+        uint32_t a0, a1, b0, b1;
+        unpack_s4x8_times16(w[2 * i], a0, a1);
+        unpack_s4x8_times16(w[2 * i + 1], b0, b1);
+        dst[i] = make_uint4(a0, a1, b0, b1);
     }
 }
 
@@ -283,7 +274,7 @@ __device__ __forceinline__ void load_h32(const uint16_t* src, float (&o)[32]) {
 
 // OUT: HQ_F16 / HQ_BF16 / HQ_F32, or OUT_DEBUG for raw accumulators.
 template <int BN, bool ASYM, int OUT>
-__global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
+__global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, const __grid_constant__ CUtensorMap tmX) {
     using L = PfSmem<BN, ASYM>;
     constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -292,11 +283,14 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     const uint32_t bar0 = smem_u32(bars);
+    constexpr int PD = L::PD;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
-    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
-    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+    auto pkfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+    auto pkempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + PD + s); };
+    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * PD + b); };
+    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * PD + 2 + b); };
+    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 2 * PD + 4);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
     int32_t* sal_s = reinterpret_cast<int32_t*>(smem + L::OFF_SAL);
 
@@ -310,8 +304,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), pf::NPROD);
+            mbar_init(full_bar(s), pf::NPROD_WARPS);
             mbar_init(empty_bar(s), 1);
+        }
+        for (int s = 0; s < PD; ++s) {
+            mbar_init(pkfull_bar(s), 1);
+            mbar_init(pkempty_bar(s), pf::NPROD_WARPS);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf_bar(b), 1);
@@ -330,33 +328,64 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp < pf::EPI_WARP0 && warp != pf::MMA_WARP) {
-        // ======================= producers
-        const int pi = (warp < pf::MMA_WARP ? warp : warp - 1) * 32 + lane;
-        const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-        const int items = my_tiles * KB;
-        const uint32_t pk0 = smem_u32(smem + L::OFF_PK);
-        auto issue = [&](int item) {
-            if (item < items) {
+    const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int items = my_tiles * KB;   // (tile, K-block) pairs of this CTA, in order
+    const uint32_t pk0 = smem_u32(smem + L::OFF_PK);
+
+    if (warp == pf::TMA_WARP) {
+        // ======================= packed-code copies
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            const int npad = (p.N + 127) / 128 * 128;   // rows present in the tile-major weight buffer
+            int slot = 0;
+            uint32_t ph = 0;
+            int issued = 0;
+            for (int item = 0; item < items; ++item) {
                 const int tile = blockIdx.x + (item / KB) * gridDim.x;
-                prod_issue<BN, ASYM>(p, (tile % MT) * pf::BM, (tile / MT) * BN, item % KB, pi,
-                                     pk0 + (item % L::PD) * L::PK_STAGE);
+                const int kb = item % KB;
+                const int m0 = (tile % MT) * pf::BM, n0 = (tile / MT) * BN;
+                if (!mbar_wait(pkempty_bar(slot), ph ^ 1u, p.limit_ns)) break;
+                const uint32_t dst = pk0 + slot * L::PK_STAGE;
+                const int nb = (npad - n0) < BN ? (npad - n0) : BN;
+                const int zb = ASYM ? ((p.N - n0) < BN ? (p.N - n0) : BN) * 2 : 0;
+                mbar_arrive_expect_tx(pkfull_bar(slot), static_cast<uint32_t>(L::PK_A + nb * pf::PK_ROW + zb));
+                tma_load_2d(dst, &tmX, kb * pf::PK_ROW, m0, pkfull_bar(slot));
+                for (int h = 0; h < nb / 128; ++h)
+                    bulk_copy_g2s(dst + L::PK_A + h * 128 * pf::PK_ROW, p.Wq + wq_offset(n0 + 128 * h, kb * 64, KB),
+                                  128 * pf::PK_ROW, pkfull_bar(slot));
+                if constexpr (ASYM)
+                    bulk_copy_g2s(dst + L::PK_A + L::PK_B,
+                                  p.zw + static_cast<int64_t>(kb / GPK) * p.N + n0, static_cast<uint32_t>(zb),
+                                  pkfull_bar(slot));
+                ++issued;
+                if (++slot == PD) { slot = 0; ph ^= 1u; }
             }
-            cp_async_commit();   // one group per stage (possibly empty)
-        };
-        for (int d = 0; d < L::PD; ++d) issue(d);
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int item = 0; item < items; ++item) {
-            cp_async_wait_group<L::PD - 1>();      // this thread's chunks of `item` have landed
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, p.limit_ns))) break;
-            prod_unpack<BN, ASYM>(smem + L::OFF_PK + (item % L::PD) * L::PK_STAGE, smem + stage * L::STAGE, pi);
-            issue(item + L::PD);                   // refill the packed slot just read
-            fence_proxy_async_smem();
-            mbar_arrive(full_bar(stage));
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            // no copy may still be landing when the CTA exits: wait for the
+            // last phase of every slot that was written (immediate unless a
+            // consumer gave up)
+            for (int i = issued > PD ? issued - PD : 0; i < issued; ++i)
+                mbar_wait(pkfull_bar(i % PD), static_cast<uint32_t>(i / PD) & 1u, p.limit_ns);
         }
-        cp_async_wait_all();   // nothing in flight when the CTA exits
+        __syncwarp();
+    } else if (warp >= pf::PROD_WARP0 && warp < pf::PROD_WARP0 + pf::NPROD_WARPS) {
+        // ======================= producers: packed codes -> int8 operand tiles
+        const int pi = (warp - pf::PROD_WARP0) * 32 + lane;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, ph = 0;
+        for (int item = 0; item < items; ++item) {
+            bool ok = mbar_wait(pkfull_bar(slot), ph, p.limit_ns);
+            ok = ok && mbar_wait(empty_bar(stage), phase ^ 1u, p.limit_ns);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            prod_unpack<BN, ASYM>(smem + L::OFF_PK + slot * L::PK_STAGE, smem + stage * L::STAGE, pi);
+            fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(pkempty_bar(slot));
+                mbar_arrive(full_bar(stage));
+            }
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            if (++slot == PD) { slot = 0; ph ^= 1u; }
+        }
     } else if (warp == pf::MMA_WARP) {
         // ======================= MMA issuer
         if (lane == 0) {
@@ -398,138 +427,134 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
         __syncwarp();
     } else {
         // ======================= epilogue
-        const int q = warp & 3;                 // TMEM lane quarter
-        const int hcol = (warp - pf::EPI_WARP0) >> 2;   // column half
+        // All 8 warps run every tile and group in lockstep through the named
+        // barrier EPI_BAR; a warp whose accumulator wait gave up keeps taking
+        // the barriers (skipping the work) so that no warp is left waiting.
+        const int et = threadIdx.x - pf::EPI_WARP0 * 32;     // 0 .. 255
+        const int q = warp & 3;                              // TMEM lane quarter
+        const int hcol = (warp - pf::EPI_WARP0) >> 2;        // column half
         const int row = 32 * q + lane;
-        uint8_t* rq_scr = smem + L::OFF_RQ + (warp - pf::EPI_WARP0) * 32 * pf::RQ_LD;
+        float* sw_s = reinterpret_cast<float*>(smem + L::OFF_SW);
+        float* sr_s = reinterpret_cast<float*>(smem + L::OFF_SR);
+        uint8_t* rq_s = smem + L::OFF_RQ;
         const int rwords = p.r / 4;
         uint32_t aphase = 0;   // bit b: phase parity of accumulator buffer b
         int abuf = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int m0 = (tile % MT) * pf::BM, n0 = (tile / MT) * BN;
             const int m = m0 + row;
             const bool mvalid = m < p.M;
+            // ---- stage the tile's column data while its MMAs run
+            named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);   // previous tile's readers are done
+            if (et < BN) stage_column<OUT>(p, n0 + et, sw_s + et, sr_s + et, rq_s + et * pf::RQ_LD);
             float sxm = 0.f;
-            if constexpr (OUT != OUT_DEBUG) sxm = mvalid ? p.sx[m] : 0.f;
+            if constexpr (OUT != OUT_DEBUG) sxm = mvalid ? __ldg(p.sx + m) : 0.f;
             uint32_t xs[16];
-            if (p.r > 0) gather_xs(p, sal_s, m, xs);
+            gather_xs(p, sal_s, m, xs);
+            named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
             constexpr int NCHUNK = BN / 2 / 32;
             float ypart[ASYM ? NCHUNK * 32 : 1];
             if constexpr (ASYM) {
-                // correction first: ypart = sr[n] * (X[m,S] . R[n,:])
+                // SERQ term first: ypart = sr[n] * (X[m,S] . R[n,:])
 #pragma unroll
                 for (int c = 0; c < NCHUNK; ++c) {
-                    const int nb = n0 + hcol * (BN / 2) + c * 32;
+                    const int col = hcol * (BN / 2) + c * 32;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) ypart[c * 32 + j] = 0.f;
-                    if (p.r > 0 && nb < p.N) {
-                        __syncwarp();
-                        stage_rq(p, rq_scr, nb, lane);
-                        __syncwarp();
+                    for (int j = 0; j < 32; ++j) {
+                        const int cc = (p.r > 0) ? corr_dot(xs, rq_s + (col + j) * pf::RQ_LD, rwords) : 0;
                         if constexpr (OUT == OUT_DEBUG) {
-                            for (int j = 0; j < 32; ++j) {
-                                const int cc = corr_dot(xs, rq_scr + j * pf::RQ_LD, rwords);
-                                if (mvalid && nb + j < p.N) p.dbg_acc_c[static_cast<int64_t>(m) * p.N + nb + j] = cc;
-                            }
+                            if (p.r > 0 && mvalid && n0 + col + j < p.N)
+                                p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n0 + col + j] = cc;
+                            ypart[c * 32 + j] = 0.f;
                         } else {
-                            float srv[32];
-                            load_h32(p.sr + nb, srv);
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const int cc = corr_dot(xs, rq_scr + j * pf::RQ_LD, rwords);
-                                ypart[c * 32 + j] = __fmul_rn(srv[j], static_cast<float>(cc));
-                            }
+                            ypart[c * 32 + j] = (p.r > 0) ? __fmul_rn(sr_s[col + j], static_cast<float>(cc)) : 0.f;
                         }
                     }
                 }
             }
-            for (int g = 0; ok && g < NG; ++g) {
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(accf_bar(abuf), (aphase >> abuf) & 1u, p.limit_ns))) {
-                    ok = false;
-                    break;
+            for (int g = 0; g < NG; ++g) {
+                float swn = 0.f;   // sw of group g + 1, column n0 + et (group weights)
+                if constexpr (ASYM && OUT != OUT_DEBUG) {
+                    if (g + 1 < NG && et < BN && n0 + et < p.N)
+                        swn = __half2float(__ushort_as_half(__ldg(p.sw + static_cast<int64_t>(g + 1) * p.N + n0 + et)));
                 }
-                tc_fence_after();
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(accf_bar(abuf), (aphase >> abuf) & 1u, p.limit_ns));
+                if (ok) {
+                    tc_fence_after();
+                    const float* swg = sw_s + (ASYM ? (g & 1) * BN : 0);
 #pragma unroll
-                for (int c = 0; c < NCHUNK; ++c) {
-                    const int col = hcol * (BN / 2) + c * 32;
-                    const int nb = n0 + col;
-                    uint32_t acc[32];
-                    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                                           static_cast<uint32_t>(abuf * BN + col), acc);
-                    tmem_wait_ld();
-                    if (nb >= p.N) continue;
-                    const int nvalid = p.N - nb;
-                    if constexpr (OUT == OUT_DEBUG) {
-                        if (mvalid) {
-                            const int sh = ASYM ? 4 : 8;
-                            for (int j = 0; j < 32 && j < nvalid; ++j)
-                                p.dbg_acc[(static_cast<int64_t>(m) * p.N + nb + j) * NG + g] =
-                                    static_cast<int32_t>(acc[j]) >> sh;
-                        }
-                        if constexpr (!ASYM) {
-                            if (p.r > 0) {
-                                __syncwarp();
-                                stage_rq(p, rq_scr, nb, lane);
-                                __syncwarp();
-                                for (int j = 0; j < 32; ++j) {
-                                    const int cc = corr_dot(xs, rq_scr + j * pf::RQ_LD, rwords);
-                                    if (mvalid && j < nvalid) p.dbg_acc_c[static_cast<int64_t>(m) * p.N + nb + j] = cc;
+                    for (int c = 0; c < NCHUNK; ++c) {
+                        const int col = hcol * (BN / 2) + c * 32;
+                        const int nb = n0 + col;
+                        uint32_t acc[32];
+                        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                               static_cast<uint32_t>(abuf * BN + col), acc);
+                        tmem_wait_ld();
+                        if (nb >= p.N) continue;
+                        const int nvalid = p.N - nb;
+                        if constexpr (OUT == OUT_DEBUG) {
+                            if (mvalid) {
+                                const int sh = ASYM ? 4 : 8;
+                                for (int j = 0; j < 32 && j < nvalid; ++j)
+                                    p.dbg_acc[(static_cast<int64_t>(m) * p.N + nb + j) * NG + g] =
+                                        static_cast<int32_t>(acc[j]) >> sh;
+                                if constexpr (!ASYM) {
+                                    if (p.r > 0) {
+                                        for (int j = 0; j < 32 && j < nvalid; ++j)
+                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + nb + j] =
+                                                corr_dot(xs, rq_s + (col + j) * pf::RQ_LD, rwords);
+                                    }
                                 }
                             }
-                        }
-                    } else if constexpr (ASYM) {
+                        } else if constexpr (ASYM) {
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            float swv[8];
-                            load_h8(p.sw + static_cast<int64_t>(g) * p.N + nb + 8 * v, swv);
+                            for (int v = 0; v < 4; ++v) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int j = 8 * v + e;
-                                ypart[c * 32 + j] = __fmaf_rn(
-                                    swv[e], static_cast<float>(static_cast<int32_t>(acc[j]) >> 4), ypart[c * 32 + j]);
+                                for (int e = 0; e < 8; ++e) {
+                                    const int j = 8 * v + e;
+                                    ypart[c * 32 + j] = __fmaf_rn(swg[col + j],
+                                                                  static_cast<float>(static_cast<int32_t>(acc[j]) >> 4),
+                                                                  ypart[c * 32 + j]);
+                                }
+                                if (g == NG - 1 && mvalid && 8 * v < nvalid) {
+                                    float y[8];
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(sxm, ypart[c * 32 + 8 * v + e]);
+                                    store_out8<OUT>(p.Y, static_cast<int64_t>(m) * p.N + nb + 8 * v, y);
+                                }
                             }
-                            if (g == NG - 1 && mvalid && 8 * v < nvalid) {
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                if (8 * v >= nvalid) break;
                                 float y[8];
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(sxm, ypart[c * 32 + 8 * v + e]);
-                                store_out8<OUT>(p.Y, static_cast<int64_t>(m) * p.N + nb + 8 * v, y);
+                                for (int e = 0; e < 8; ++e) {
+                                    const int j = 8 * v + e;
+                                    const int cc = (p.r > 0) ? corr_dot(xs, rq_s + (col + j) * pf::RQ_LD, rwords) : 0;
+                                    const float a = static_cast<float>(static_cast<int32_t>(acc[j]) >> 8);
+                                    const float t = __fmaf_rn(sr_s[col + j], static_cast<float>(cc), __fmul_rn(swg[col + j], a));
+                                    y[e] = __fmul_rn(sxm, t);
+                                }
+                                if (mvalid) store_out8<OUT>(p.Y, static_cast<int64_t>(m) * p.N + nb + 8 * v, y);
                             }
-                        }
-                    } else {
-                        if (p.r > 0) {
-                            __syncwarp();
-                            stage_rq(p, rq_scr, nb, lane);
-                            __syncwarp();
-                        }
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            if (8 * v >= nvalid) break;
-                            float swv[8], srv[8], y[8];
-                            load_h8(p.sw + nb + 8 * v, swv);
-                            if (p.r > 0) {
-                                load_h8(p.sr + nb + 8 * v, srv);
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) srv[e] = 0.f;
-                            }
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int j = 8 * v + e;
-                                const int cc = (p.r > 0) ? corr_dot(xs, rq_scr + j * pf::RQ_LD, rwords) : 0;
-                                const float a = static_cast<float>(static_cast<int32_t>(acc[j]) >> 8);
-                                const float t = __fmaf_rn(srv[e], static_cast<float>(cc), __fmul_rn(swv[e], a));
-                                y[e] = __fmul_rn(sxm, t);
-                            }
-                            if (mvalid) store_out8<OUT>(p.Y, static_cast<int64_t>(m) * p.N + nb + 8 * v, y);
                         }
                     }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acce_bar(abuf));
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acce_bar(abuf));
                 aphase ^= 1u << abuf;
                 abuf ^= 1;
+                if constexpr (ASYM) {
+                    // hand the next group's sw to every warp; the buffer written
+                    // here was last read in group g - 1, before the previous barrier
+                    if constexpr (OUT != OUT_DEBUG) {
+                        if (et < BN) sw_s[((g + 1) & 1) * BN + et] = swn;
+                    }
+                    named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
+                }
             }
         }
     }
@@ -543,15 +568,48 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p) {
     }
 }
 
+// cuTensorMapEncodeTiled from the driver, found once through the runtime (the
+// library links only the CUDA runtime).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// Tensor map of the packed activations Xq[M][K/2] (bytes): boxes of 64 bytes x
+// 128 rows, rows past M filled with zero.
+static hq_status xq_tensor_map(const GemmArgs& a, CUtensorMap* map) {
+    const auto encode = encode_tiled();
+    if (!encode) return HQ_ERR_CUDA;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 2), static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 2)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::PK_ROW), static_cast<cuuint32_t>(pf::BM)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.Xq), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
 template <int BN, bool ASYM, int OUT>
 static hq_status launch_pf_t(const GemmArgs& a, cudaStream_t st, int nsm) {
     auto kern = k_gemm_pf<BN, ASYM, OUT>;
     const int smem = PfSmem<BN, ASYM>::ALLOC;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
+    CUtensorMap tmX;
+    const hq_status s = xq_tensor_map(a, &tmX);
+    if (s != HQ_OK) return s;
     const int tiles = ((a.M + pf::BM - 1) / pf::BM) * ((a.N + BN - 1) / BN);
     const int grid = tiles < nsm ? tiles : nsm;
-    kern<<<grid, pf::THREADS, smem, st>>>(a);
+    kern<<<grid, pf::THREADS, smem, st>>>(a, tmX);
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
