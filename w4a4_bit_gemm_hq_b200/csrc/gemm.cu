@@ -9,25 +9,33 @@
 // no intermediate quantisation); "OffQ: Taming Structured Outliers in LLM
 // Quantization by Offsetting", Methodology 3 (group-wise scale and zero point).
 //
-// Design (one CTA per SM, persistent over 128 x BN output tiles):
-//  * one thread moves the packed codes of each K-block into a ring of packed
-//    slots with the tensor memory accelerator: a 2D tensor-map load of the 128
-//    activation rows (64 bytes each; rows past M read as zero) and 8 KB bulk
-//    copies of the tile-major weight blocks (plus the zero points of the
-//    block's group for group weights).
-//  * tcgen05 has no int4 MMA, so 6 producer warps expand the packed codes to
-//    int8 in registers (16*q for activations and symmetric weights, u - z for
-//    asymmetric weights) and store them into 128-byte-swizzled K-major smem
-//    tiles: A = 128 activation rows x 128 K, B = BN weight rows x 128 K.
-//  * one thread issues tcgen05.mma (M=128, N=BN, K=32) x 4 per stage into a
-//    double-buffered int32 accumulator in tensor memory; tcgen05.commit frees
-//    the smem stage and, at the end of a tile (per-channel weights) or of a
-//    weight group (group weights), hands the accumulator to the epilogue.
-//  * 8 epilogue warps (2 per TMEM lane quarter, splitting the columns) load
-//    the accumulator with tcgen05.ld, dequantise with sx[m] * sw[n] (or sum the
-//    per-group sw[b][n] * acc_b), add sr[n] * (X[m,S] . Rq[n,:]) computed with
-//    dp4a (the SERQ term as an epilogue add: no second launch), round once and
-//    store.
+// Design (CTA pairs, one CTA per SM, persistent over 256 x BN output tiles):
+//  * the two CTAs of a cluster form a pair; the even CTA issues pair-wide
+//    tcgen05.mma (M = 256, N = BN, K = 32): A rows 0-127 come from its own
+//    shared memory and rows 128-255 from its partner's, and each CTA holds
+//    half of the BN weight rows of B, so each SM stages only its own 128
+//    activation rows and BN/2 weight rows.  Each CTA's tensor memory receives
+//    its 128 rows x BN of the int32 accumulator.
+//  * in each CTA, one thread moves the packed codes of each K-block into a ring
+//    of packed slots with the tensor memory accelerator: a 2D tensor-map load
+//    of its 128 activation rows (64 bytes each; rows past M read as zero) and a
+//    bulk copy of its half of the tile-major weight block (plus the zero points
+//    of the block's group for group weights).
+//  * tcgen05 has no int4 MMA, so 6 producer warps per CTA expand the packed
+//    codes to int8 in registers (16*q for activations and symmetric weights,
+//    u - z for asymmetric weights) and store them into 128-byte-swizzled
+//    K-major smem tiles; they signal the even CTA's stage barrier, and the
+//    pair MMA's commit frees the stage in both CTAs.
+//  * the even CTA's MMA thread issues 4 pair MMAs per stage into one of
+//    512 / BN int32 accumulator buffers; at the end of a tile (per-channel
+//    weights) or of a weight group (group weights) a multicast commit hands the
+//    buffer to the epilogues of both CTAs.
+//  * 8 epilogue warps per CTA (2 per TMEM lane quarter, splitting the
+//    columns) stage the tile's sw, sr and unpacked Rq rows in smem while the
+//    tile's MMAs run, then load the accumulator with tcgen05.ld, dequantise
+//    with sx[m] * sw[n] (or sum the per-group sw[b][n] * acc_b), add
+//    sr[n] * (X[m,S] . Rq[n,:]) computed with dp4a (the SERQ term as an
+//    epilogue add: no second launch), round once and store.
 //  * every mbarrier wait is bounded; on timeout the status word records
 //    HQ_ERR_TIMEOUT and the roles skip to teardown, which waits for in-flight
 //    MMAs before freeing tensor memory.
@@ -60,23 +68,25 @@ constexpr int EPI_THREADS = 256;
 constexpr uint32_t EPI_BAR = 1;       // named barrier of the epilogue warps
 }  // namespace pf
 
-// Shared memory: an int8 operand ring read by the tensor core (STAGES deep) and
-// a ring of packed slots (PD deep) filled by the copy engine.  A packed slot
-// holds the 128 activation rows (64 bytes each), the BN weight rows in the
-// order of the tile-major layout (128-row blocks of 8 KB) and, for group
-// weights, the BN fp16 zero points of the block's group.
+// Shared memory of one CTA of a pair: an int8 operand ring read by the tensor
+// core (STAGES deep: 128 activation rows, then BH = BN/2 weight rows, 128 K
+// bytes each) and a ring of packed slots (PD deep) filled by the copy engine:
+// the 128 activation rows (64 bytes each), the BH weight rows in tile-major
+// order and, for group weights, their BH fp16 zero points of the block's group.
 template <int BN, bool ASYM>
 struct PfSmem {
-    static constexpr int STAGES = (BN == 256) ? 2 : 3;
-    static constexpr int PD = (BN == 256) ? 4 : 5;
+    static constexpr int BH = BN / 2;                                  // weight rows per CTA
+    static constexpr int NACC = 512 / BN;                              // accumulator buffers
+    static constexpr int STAGES = 4;
+    static constexpr int PD = ASYM ? 6 : 4;
     static constexpr int A_BYTES = pf::BM * pf::BK;
-    static constexpr int B_BYTES = BN * pf::BK;
+    static constexpr int B_BYTES = BH * pf::BK;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NCHUNK = (pf::BM + BN) * 4;                   // 16-byte packed chunks per stage
+    static constexpr int NCHUNK = (pf::BM + BH) * 4;                   // 16-byte packed chunks per stage
     static constexpr int NCH = (NCHUNK + pf::NPROD - 1) / pf::NPROD;  // per producer thread
     static constexpr int PK_A = pf::BM * pf::PK_ROW;
-    static constexpr int PK_B = BN * pf::PK_ROW;
-    static constexpr int PK_Z = ASYM ? BN * 2 : 0;
+    static constexpr int PK_B = BH * pf::PK_ROW;
+    static constexpr int PK_Z = ASYM ? BH * 2 : 0;
     static constexpr int PK_STAGE = ((PK_A + PK_B + PK_Z) + 127) / 128 * 128;
     static constexpr int OFF_PK = STAGES * STAGE;
     static constexpr int OFF_RQ = OFF_PK + PD * PK_STAGE;              // tile's Rq rows, BN x RQ_LD int8
@@ -84,11 +94,12 @@ struct PfSmem {
     static constexpr int OFF_SR = OFF_SW + 2 * BN * 4;                 // float [BN]
     static constexpr int OFF_SAL = OFF_SR + BN * 4;                    // int32[128]
     static constexpr int OFF_BAR = OFF_SAL + 128 * 4;
-    static constexpr int NBAR = 2 * STAGES + 2 * PD + 4 + 1;
+    static constexpr int NBAR = 2 * STAGES + 2 * PD + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16;
     static constexpr int ALLOC = BYTES + 1024;                         // 1024-byte alignment slack
     static_assert(ALLOC <= 227 * 1024, "shared memory budget");
+    static_assert(BN * NACC == 512, "accumulator buffers fill the tensor memory");
 };
 
 __device__ __forceinline__ uint32_t swz_chunk(int row, int chunk) { return static_cast<uint32_t>(chunk ^ (row & 7)); }
@@ -273,67 +284,71 @@ __device__ __forceinline__ void load_h32(const uint16_t* src, float (&o)[32]) {
 }
 
 // OUT: HQ_F16 / HQ_BF16 / HQ_F32, or OUT_DEBUG for raw accumulators.
+// Launched as clusters of 2 CTAs (an even number of CTAs).
 template <int BN, bool ASYM, int OUT>
 __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, const __grid_constant__ CUtensorMap tmX) {
     using L = PfSmem<BN, ASYM>;
     constexpr int STAGES = L::STAGES;
+    constexpr int PD = L::PD;
+    constexpr int NACC = L::NACC;
+    constexpr int BH = L::BH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t crank = cluster_ctarank();   // 0: issues the pair MMAs
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     const uint32_t bar0 = smem_u32(bars);
-    constexpr int PD = L::PD;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };                       // even CTA: both CTAs' producers
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };           // each CTA: pair MMA commit
     auto pkfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
     auto pkempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + PD + s); };
-    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * PD + b); };
-    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * PD + 2 + b); };
-    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 2 * PD + 4);
+    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * PD + b); };          // each CTA
+    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * PD + NACC + b); };   // even CTA
+    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 2 * PD + 2 * NACC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
     int32_t* sal_s = reinterpret_cast<int32_t*>(smem + L::OFF_SAL);
 
-    const int MT = (p.M + pf::BM - 1) / pf::BM;
+    const int MT = (p.M + 2 * pf::BM - 1) / (2 * pf::BM);
     const int NT = (p.N + BN - 1) / BN;
     const int num_tiles = MT * NT;
     const int KB = p.K / pf::BK;
     const int GPK = ASYM ? p.gw / pf::BK : KB;   // K-blocks per accumulation group
     const int NG = KB / GPK;
-    constexpr uint32_t TMEM_COLS = 2 * BN;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), pf::NPROD_WARPS);
+            mbar_init(full_bar(s), 2 * pf::NPROD_WARPS);
             mbar_init(empty_bar(s), 1);
         }
         for (int s = 0; s < PD; ++s) {
             mbar_init(pkfull_bar(s), 1);
             mbar_init(pkempty_bar(s), pf::NPROD_WARPS);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NACC; ++b) {
             mbar_init(accf_bar(b), 1);
-            mbar_init(acce_bar(b), 8);
+            mbar_init(acce_bar(b), 2 * 8);
         }
         mbar_init(done_bar, 1);
         fence_mbar_init();
     }
     for (int j = threadIdx.x; j < p.r; j += blockDim.x) sal_s[j] = p.sal[j];
     if (warp == pf::MMA_WARP) {
-        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(tmem_slot), 512);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int items = my_tiles * KB;   // (tile, K-block) pairs of this CTA, in order
+    const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
+    const int items = my_tiles * KB;   // (tile, K-block) pairs of this CTA pair, in order
     const uint32_t pk0 = smem_u32(smem + L::OFF_PK);
 
     if (warp == pf::TMA_WARP) {
-        // ======================= packed-code copies
+        // ======================= packed-code copies (this CTA's rows)
         if (lane == 0) {
             prefetch_tmap(&tmX);
             const int npad = (p.N + 127) / 128 * 128;   // rows present in the tile-major weight buffer
@@ -341,22 +356,25 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
             uint32_t ph = 0;
             int issued = 0;
             for (int item = 0; item < items; ++item) {
-                const int tile = blockIdx.x + (item / KB) * gridDim.x;
+                const int tile = pair + (item / KB) * npairs;
                 const int kb = item % KB;
-                const int m0 = (tile % MT) * pf::BM, n0 = (tile / MT) * BN;
+                const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM;
+                const int nr = (tile / MT) * BN + static_cast<int>(crank) * BH;   // first weight row of this CTA
                 if (!mbar_wait(pkempty_bar(slot), ph ^ 1u, p.limit_ns)) break;
                 const uint32_t dst = pk0 + slot * L::PK_STAGE;
-                const int nb = (npad - n0) < BN ? (npad - n0) : BN;
-                const int zb = ASYM ? ((p.N - n0) < BN ? (p.N - n0) : BN) * 2 : 0;
-                mbar_arrive_expect_tx(pkfull_bar(slot), static_cast<uint32_t>(L::PK_A + nb * pf::PK_ROW + zb));
+                const bool has_b = nr < npad;
+                const int zrows = ASYM ? ((p.N - nr) < BH ? (p.N - nr) : BH) : 0;
+                const int zb = zrows > 0 ? zrows * 2 : 0;
+                mbar_arrive_expect_tx(pkfull_bar(slot),
+                                      static_cast<uint32_t>(L::PK_A + (has_b ? L::PK_B : 0) + zb));
                 tma_load_2d(dst, &tmX, kb * pf::PK_ROW, m0, pkfull_bar(slot));
-                for (int h = 0; h < nb / 128; ++h)
-                    bulk_copy_g2s(dst + L::PK_A + h * 128 * pf::PK_ROW, p.Wq + wq_offset(n0 + 128 * h, kb * 64, KB),
-                                  128 * pf::PK_ROW, pkfull_bar(slot));
-                if constexpr (ASYM)
-                    bulk_copy_g2s(dst + L::PK_A + L::PK_B,
-                                  p.zw + static_cast<int64_t>(kb / GPK) * p.N + n0, static_cast<uint32_t>(zb),
-                                  pkfull_bar(slot));
+                if (has_b)
+                    bulk_copy_g2s(dst + L::PK_A, p.Wq + wq_offset(nr, kb * 64, KB), L::PK_B, pkfull_bar(slot));
+                if constexpr (ASYM) {
+                    if (zb > 0)
+                        bulk_copy_g2s(dst + L::PK_A + L::PK_B, p.zw + static_cast<int64_t>(kb / GPK) * p.N + nr,
+                                      static_cast<uint32_t>(zb), pkfull_bar(slot));
+                }
                 ++issued;
                 if (++slot == PD) { slot = 0; ph ^= 1u; }
             }
@@ -370,39 +388,43 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
     } else if (warp >= pf::PROD_WARP0 && warp < pf::PROD_WARP0 + pf::NPROD_WARPS) {
         // ======================= producers: packed codes -> int8 operand tiles
         const int pi = (warp - pf::PROD_WARP0) * 32 + lane;
+        const uint32_t full_remote0 = mapa_shared(full_bar(0), 0);
         int stage = 0, slot = 0;
         uint32_t phase = 0, ph = 0;
         for (int item = 0; item < items; ++item) {
             bool ok = mbar_wait(pkfull_bar(slot), ph, p.limit_ns);
-            ok = ok && mbar_wait(empty_bar(stage), phase ^ 1u, p.limit_ns);
+            ok = ok && mbar_wait_cluster(empty_bar(stage), phase ^ 1u, p.limit_ns);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
             prod_unpack<BN, ASYM>(smem + L::OFF_PK + slot * L::PK_STAGE, smem + stage * L::STAGE, pi);
             fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(pkempty_bar(slot));
-                mbar_arrive(full_bar(stage));
+                mbar_arrive_cluster(full_remote0 + 8u * static_cast<uint32_t>(stage));
             }
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             if (++slot == PD) { slot = 0; ph ^= 1u; }
         }
     } else if (warp == pf::MMA_WARP) {
-        // ======================= MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_i8(pf::BM, BN);
+        // ======================= pair MMA issuer (even CTA)
+        if (lane == 0 && crank == 0) {
+            constexpr uint32_t IDESC = idesc_i8(2 * pf::BM, BN);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t aphase = 0;   // bit b: phase parity of accumulator buffer b
             int abuf = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
                 for (int kb = 0; ok && kb < KB; ++kb) {
                     const bool first = (kb % GPK) == 0;
                     if (first) {
-                        if (!mbar_wait(acce_bar(abuf), ((aphase >> abuf) & 1u) ^ 1u, p.limit_ns)) { ok = false; break; }
+                        if (!mbar_wait_cluster(acce_bar(abuf), ((aphase >> abuf) & 1u) ^ 1u, p.limit_ns)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
                     }
-                    if (!mbar_wait(full_bar(stage), phase, p.limit_ns)) { ok = false; break; }
+                    if (!mbar_wait_cluster(full_bar(stage), phase, p.limit_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * L::STAGE);
                     const uint64_t adesc = sw128_kmajor_desc(sa);
@@ -410,23 +432,23 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                     const uint32_t dcol = tmem_base + static_cast<uint32_t>(abuf * BN);
 #pragma unroll
                     for (int kk = 0; kk < pf::BK / 32; ++kk)
-                        mma_i8_ss(dcol, adesc + 2u * kk, bdesc + 2u * kk, IDESC, (first && kk == 0) ? 0u : 1u);
-                    tc_commit(empty_bar(stage));
+                        mma_i8_ss_pair(dcol, adesc + 2u * kk, bdesc + 2u * kk, IDESC, (first && kk == 0) ? 0u : 1u);
+                    tc_commit_pair_mc(empty_bar(stage), 0x3);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     if ((kb % GPK) == GPK - 1) {
-                        tc_commit(accf_bar(abuf));
+                        tc_commit_pair_mc(accf_bar(abuf), 0x3);
                         aphase ^= 1u << abuf;
-                        abuf ^= 1;
+                        abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
                     }
                 }
             }
             // all MMAs issued by this thread have completed before teardown
-            tc_commit(done_bar);
+            tc_commit_pair(done_bar);
             mbar_wait(done_bar, 0, p.limit_ns);
         }
         __syncwarp();
     } else {
-        // ======================= epilogue
+        // ======================= epilogue (this CTA's 128 rows, all BN columns)
         // All 8 warps run every tile and group in lockstep through the named
         // barrier EPI_BAR; a warp whose accumulator wait gave up keeps taking
         // the barriers (skipping the work) so that no warp is left waiting.
@@ -438,11 +460,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
         float* sr_s = reinterpret_cast<float*>(smem + L::OFF_SR);
         uint8_t* rq_s = smem + L::OFF_RQ;
         const int rwords = p.r / 4;
+        const uint32_t acce_remote0 = mapa_shared(acce_bar(0), 0);
         uint32_t aphase = 0;   // bit b: phase parity of accumulator buffer b
         int abuf = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int m0 = (tile % MT) * pf::BM, n0 = (tile / MT) * BN;
+        for (int tile = pair; tile < num_tiles; tile += npairs) {
+            const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM, n0 = (tile / MT) * BN;
             const int m = m0 + row;
             const bool mvalid = m < p.M;
             // ---- stage the tile's column data while its MMAs run
@@ -543,10 +566,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(acce_bar(abuf));
+                    if (lane == 0) mbar_arrive_cluster(acce_remote0 + 8u * static_cast<uint32_t>(abuf));
                 }
                 aphase ^= 1u << abuf;
-                abuf ^= 1;
+                abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
                 if constexpr (ASYM) {
                     // hand the next group's sw to every warp; the buffer written
                     // here was last read in group g - 1, before the previous barrier
@@ -559,12 +582,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
         }
     }
 
+    // Teardown: neither CTA leaves while its partner may still read its shared
+    // memory or arrive on its barriers, or while pair MMAs are in flight (the
+    // even CTA's MMA thread waited for them above).
     __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     if (warp == pf::MMA_WARP) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, 512);
     }
 }
 
@@ -607,12 +633,35 @@ static hq_status launch_pf_t(const GemmArgs& a, cudaStream_t st, int nsm) {
     CUtensorMap tmX;
     const hq_status s = xq_tensor_map(a, &tmX);
     if (s != HQ_OK) return s;
-    const int tiles = ((a.M + pf::BM - 1) / pf::BM) * ((a.N + BN - 1) / BN);
-    const int grid = tiles < nsm ? tiles : nsm;
-    kern<<<grid, pf::THREADS, smem, st>>>(a, tmX);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(pf::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // CTA pairs that fit on the device at once (a pair needs two SMs of one
+    // cluster-capable group, so this can be below nsm / 2); queried once per
+    // device and kernel variant
+    static int max_pairs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HQ_ERR_CUDA;
+    if (max_pairs[dev] == 0) {
+        cfg.gridDim = dim3(2 * (nsm / 2), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return HQ_ERR_CUDA;
+        max_pairs[dev] = n;
+    }
+    const int tiles = ((a.M + 2 * pf::BM - 1) / (2 * pf::BM)) * ((a.N + BN - 1) / BN);
+    const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, a, tmX) != cudaSuccess) return HQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
-
 hq_status launch_gemm_prefill(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
     if (a.gw == 0) {
         switch (out) {
