@@ -60,7 +60,8 @@ constexpr int TMA_WARP = 0;           // lane 0 issues the packed-code copies
 constexpr int MMA_WARP = 1;           // lane 0 issues tcgen05.mma; the warp owns TMEM
 constexpr int PROD_WARP0 = 2;         // warps 2-7 expand codes to int8
 constexpr int NPROD_WARPS = 6;
-constexpr int NPROD = NPROD_WARPS * 32;
+constexpr int NGROUP_WARPS = 3;       // two producer groups take alternate K-blocks
+constexpr int NGROUP = NGROUP_WARPS * 32;
 constexpr int EPI_WARP0 = 8;          // warps 8-15: epilogue
 constexpr int PK_ROW = 64;            // packed bytes of one row of a K-block
 constexpr int RQ_LD = 64;             // bytes per unpacked Rq row (r <= 64) in the per-tile staging
@@ -83,7 +84,7 @@ struct PfSmem {
     static constexpr int B_BYTES = BH * pf::BK;
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int NCHUNK = (pf::BM + BH) * 4;                   // 16-byte packed chunks per stage
-    static constexpr int NCH = (NCHUNK + pf::NPROD - 1) / pf::NPROD;  // per producer thread
+    static constexpr int NCH = (NCHUNK + pf::NGROUP - 1) / pf::NGROUP;  // per producer thread and stage
     static constexpr int PK_A = pf::BM * pf::PK_ROW;
     static constexpr int PK_B = BH * pf::PK_ROW;
     static constexpr int PK_Z = ASYM ? BH * 2 : 0;
@@ -113,7 +114,7 @@ __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, i
     using L = PfSmem<BN, ASYM>;
 #pragma unroll
     for (int j = 0; j < L::NCH; ++j) {
-        const int ci = pi + j * pf::NPROD;
+        const int ci = pi + j * pf::NGROUP;
         if (ci >= L::NCHUNK) continue;
         const bool isA = ci < pf::BM * 4;
         const int cl = isA ? ci : ci - pf::BM * 4;
@@ -293,7 +294,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
     constexpr int NACC = L::NACC;
     constexpr int BH = L::BH;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived by pointer arithmetic on the __shared__
+    // array so that every access through it compiles to a shared-memory
+    // instruction (a pointer rebuilt from an integer is generic)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t crank = cluster_ctarank();   // 0: issues the pair MMAs
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -319,12 +323,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 2 * pf::NPROD_WARPS);
+            mbar_init(full_bar(s), 2 * pf::NGROUP_WARPS);
             mbar_init(empty_bar(s), 1);
         }
         for (int s = 0; s < PD; ++s) {
             mbar_init(pkfull_bar(s), 1);
-            mbar_init(pkempty_bar(s), pf::NPROD_WARPS);
+            mbar_init(pkempty_bar(s), pf::NGROUP_WARPS);
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(accf_bar(b), 1);
@@ -387,11 +391,17 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
         __syncwarp();
     } else if (warp >= pf::PROD_WARP0 && warp < pf::PROD_WARP0 + pf::NPROD_WARPS) {
         // ======================= producers: packed codes -> int8 operand tiles
-        const int pi = (warp - pf::PROD_WARP0) * 32 + lane;
+        // Two groups of 3 warps take alternate K-blocks, so one group's
+        // barrier waits overlap the other's unpacking (STAGES and PD are even:
+        // each group keeps to its own stages and slots).
+        static_assert(STAGES % 2 == 0 && PD % 2 == 0, "groups alternate over the rings");
+        const int grp = (warp - pf::PROD_WARP0) / pf::NGROUP_WARPS;
+        const int pi = ((warp - pf::PROD_WARP0) % pf::NGROUP_WARPS) * 32 + lane;
         const uint32_t full_remote0 = mapa_shared(full_bar(0), 0);
-        int stage = 0, slot = 0;
-        uint32_t phase = 0, ph = 0;
-        for (int item = 0; item < items; ++item) {
+        for (int item = grp; item < items; item += 2) {
+            const int stage = item % STAGES, slot = item % PD;
+            const uint32_t phase = static_cast<uint32_t>(item / STAGES) & 1u;
+            const uint32_t ph = static_cast<uint32_t>(item / PD) & 1u;
             bool ok = mbar_wait(pkfull_bar(slot), ph, p.limit_ns);
             ok = ok && mbar_wait_cluster(empty_bar(stage), phase ^ 1u, p.limit_ns);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -402,8 +412,6 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 mbar_arrive(pkempty_bar(slot));
                 mbar_arrive_cluster(full_remote0 + 8u * static_cast<uint32_t>(stage));
             }
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            if (++slot == PD) { slot = 0; ph ^= 1u; }
         }
     } else if (warp == pf::MMA_WARP) {
         // ======================= pair MMA issuer (even CTA)

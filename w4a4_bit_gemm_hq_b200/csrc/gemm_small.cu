@@ -147,7 +147,10 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
     using L = SkSmem<NT>;
     constexpr int SB = L::SB;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived by pointer arithmetic on the __shared__
+    // array so that every access through it compiles to a shared-memory
+    // instruction (a pointer rebuilt from an integer is generic)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_u32(smem + L::OFF_BAR);
     auto fulla = [&](int s) { return bar0 + 8u * s; };          // A stage s written (producer set s)
