@@ -64,7 +64,8 @@ constexpr int NGROUP_WARPS = 3;       // two producer groups take alternate K-bl
 constexpr int NGROUP = NGROUP_WARPS * 32;
 constexpr int EPI_WARP0 = 8;          // warps 8-15: epilogue
 constexpr int PK_ROW = 64;            // packed bytes of one row of a K-block
-constexpr int RQ_LD = 64;             // bytes per unpacked Rq row (r <= 64) in the per-tile staging
+constexpr int RQ_LD = 80;             // bytes per staged int8 row of r <= 64 codes (padded: the
+                                      // mma.sync fragment loads of 8 rows x 4 words hit 32 banks)
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t EPI_BAR = 1;       // named barrier of the epilogue warps
 }  // namespace pf
@@ -93,7 +94,8 @@ struct PfSmem {
     static constexpr int OFF_RQ = OFF_PK + PD * PK_STAGE;              // tile's Rq rows, BN x RQ_LD int8
     static constexpr int OFF_SW = OFF_RQ + BN * pf::RQ_LD;             // float [2][BN]: sw of the tile (of a group)
     static constexpr int OFF_SR = OFF_SW + 2 * BN * 4;                 // float [BN]
-    static constexpr int OFF_SAL = OFF_SR + BN * 4;                    // int32[128]
+    static constexpr int OFF_XS = OFF_SR + BN * 4;                     // tile's X[m,S] rows, 128 x RQ_LD int8
+    static constexpr int OFF_SAL = OFF_XS + pf::BM * pf::RQ_LD;        // int32[128]
     static constexpr int OFF_BAR = OFF_SAL + 128 * 4;
     static constexpr int NBAR = 2 * STAGES + 2 * PD + 2 * NACC + 1;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
@@ -188,6 +190,127 @@ __device__ __forceinline__ void stage_column(const GemmArgs& p, int n, float* sw
         unpack_s4x8_times16(w[2 * i], a0, a1);
         unpack_s4x8_times16(w[2 * i + 1], b0, b1);
         dst[i] = make_uint4(a0, a1, b0, b1);
+    }
+}
+
+// Salient activation codes of row m for the staged int8 row `xs_w` (words):
+// position j = 8 i + 2 e + h -> word 2 i + h, byte e (the lo/hi permutation of
+// unpack_s4x8_times16).  This thread writes the blocks i with i % 2 == half
+// (words 2i, 2i+1) of the first `nblk` blocks; blocks past r and rows past M
+// are zero.  All loads of the thread are in flight together.
+__device__ __forceinline__ void gather_xs_smem(const GemmArgs& p, const int32_t* sal_s, int m, uint32_t* xs_w,
+                                               int half, int nblk) {
+    const bool mv = m < p.M;
+    const uint8_t* row = p.Xq + static_cast<int64_t>(mv ? m : 0) * (p.K / 2);
+    uint32_t nib[4][8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const int i = 2 * b + half;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            nib[b][t] = 0u;
+            if (mv && 8 * i < p.r) {
+                const int k = sal_s[8 * i + t];
+                nib[b][t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
+            }
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const int i = 2 * b + half;
+        if (i >= nblk) break;
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const uint32_t code = (8 * i < p.r) ? static_cast<uint32_t>(static_cast<int>(nib[b][t] ^ 8u) - 8) & 0xFFu : 0u;
+            if (t & 1) hi |= code << (8 * (t >> 1));
+            else lo |= code << (8 * (t >> 1));
+        }
+        xs_w[2 * i] = lo;
+        xs_w[2 * i + 1] = hi;
+    }
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_out2(void* Y, int64_t off, float a, float b) {
+    if constexpr (OUT == HQ_F32) {
+        *reinterpret_cast<float2*>(static_cast<float*>(Y) + off) = make_float2(a, b);
+    } else if constexpr (OUT == HQ_BF16) {
+        *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(Y) + off) = __floats2bfloat162_rn(a, b);
+    } else {
+        *reinterpret_cast<__half2*>(static_cast<uint16_t*>(Y) + off) = __floats2half2_rn(a, b);
+    }
+}
+
+// Symmetric-weight epilogue of one 32-column chunk for the warp's 32 rows.
+// The accumulator comes from tensor memory in the mma.sync m16n8 fragment
+// layout (two 16-lane halves); the SERQ term acc_c = X[m,S] . Rq[n,:] is
+// computed on the staged int8 codes with mma.sync m16n8k32 in the same layout;
+// then Y = sx[m] * (sr[n] * acc_c + sw[n] * acc), rounded once.
+//  tm     tensor-memory address of lane 32q, chunk column 0
+//  mq0    first output row of the warp;  n0c  first output column of the chunk
+//  scol   column of the chunk within the tile (index into the staged columns)
+//  afr    A fragments [row half][K step] of the warp's X[m,S] rows
+template <int OUT>
+__device__ __forceinline__ void drain_sym_chunk(const GemmArgs& p, uint32_t tm, int mq0, int n0c, int scol,
+                                                const float* sw_s, const float* sr_s, const uint8_t* rq_s,
+                                                const uint32_t (&afr)[2][2][4], int ksteps, const float (&sxr)[2][2],
+                                                int g, int t) {
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        uint32_t v[16];
+        tmem_ld_16x256b_x4(tm + (static_cast<uint32_t>(16 * mt) << 16), v);
+        tmem_wait_ld();
+        int32_t cc[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cc[nt][i] = 0;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            if (ks < ksteps) {
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const uint32_t* rw =
+                        reinterpret_cast<const uint32_t*>(rq_s + (scol + 8 * nt + g) * pf::RQ_LD) + 8 * ks;
+                    mma_s8_16x8x32(cc[nt], afr[mt][ks], rw[t], rw[4 + t]);
+                }
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            if (n0c + 8 * nt >= p.N) continue;   // N % 8 == 0: whole groups of 8 columns
+            const int cl = scol + 8 * nt + 2 * t;
+            const int64_t n = n0c + 8 * nt + 2 * t;
+            float2 swv = make_float2(0.f, 0.f), srv = make_float2(0.f, 0.f);
+            if constexpr (OUT != OUT_DEBUG) {
+                swv = *reinterpret_cast<const float2*>(sw_s + cl);
+                srv = *reinterpret_cast<const float2*>(sr_s + cl);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int m = mq0 + 16 * mt + g + 8 * h;
+                if (m >= p.M) continue;
+                const int32_t a0 = static_cast<int32_t>(v[4 * nt + 2 * h]) >> 8;
+                const int32_t a1 = static_cast<int32_t>(v[4 * nt + 2 * h + 1]) >> 8;
+                const int32_t c0 = cc[nt][2 * h] >> 4, c1 = cc[nt][2 * h + 1] >> 4;   // Rq codes carry 16
+                const int64_t off = static_cast<int64_t>(m) * p.N + n;
+                if constexpr (OUT == OUT_DEBUG) {
+                    p.dbg_acc[off] = a0;
+                    p.dbg_acc[off + 1] = a1;
+                    if (p.r > 0) {
+                        p.dbg_acc_c[off] = c0;
+                        p.dbg_acc_c[off + 1] = c1;
+                    }
+                } else {
+                    const float y0 = __fmul_rn(sxr[mt][h], __fmaf_rn(srv.x, static_cast<float>(c0),
+                                                                     __fmul_rn(swv.x, static_cast<float>(a0))));
+                    const float y1 = __fmul_rn(sxr[mt][h], __fmaf_rn(srv.y, static_cast<float>(c1),
+                                                                     __fmul_rn(swv.y, static_cast<float>(a1))));
+                    store_out2<OUT>(p.Y, off, y0, y1);
+                }
+            }
+        }
     }
 }
 
@@ -467,11 +590,69 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
         float* sw_s = reinterpret_cast<float*>(smem + L::OFF_SW);
         float* sr_s = reinterpret_cast<float*>(smem + L::OFF_SR);
         uint8_t* rq_s = smem + L::OFF_RQ;
-        const int rwords = p.r / 4;
         const uint32_t acce_remote0 = mapa_shared(acce_bar(0), 0);
         uint32_t aphase = 0;   // bit b: phase parity of accumulator buffer b
         int abuf = 0;
         bool ok = true;
+        if constexpr (!ASYM) {
+            // per-channel weights: one accumulator per tile, drained in the
+            // mma.sync fragment layout with the SERQ term on mma.sync
+            const uint32_t* xs_w = reinterpret_cast<const uint32_t*>(smem + L::OFF_XS);
+            const int g8 = lane >> 2, t4 = lane & 3;
+            const int ksteps = (p.r + 31) / 32;
+            for (int tile = pair; tile < num_tiles; tile += npairs) {
+                const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM, n0 = (tile / MT) * BN;
+                const int mq0 = m0 + 32 * q;
+                // ---- stage the tile's column data and X[m,S] rows while its MMAs run
+                named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);   // previous tile's readers are done
+                if (et < BN) stage_column<OUT>(p, n0 + et, sw_s + et, sr_s + et, rq_s + et * pf::RQ_LD);
+                if (p.r > 0)
+                    gather_xs_smem(p, sal_s, m0 + row,
+                                   reinterpret_cast<uint32_t*>(smem + L::OFF_XS + row * pf::RQ_LD), hcol, 4 * ksteps);
+                float sxr[2][2];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int m = mq0 + 16 * mt + g8 + 8 * h;
+                        sxr[mt][h] = 0.f;
+                        if constexpr (OUT != OUT_DEBUG) sxr[mt][h] = m < p.M ? __ldg(p.sx + m) : 0.f;
+                    }
+                named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
+                uint32_t afr[2][2][4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const uint32_t* r0 = xs_w + (32 * q + 16 * mt + g8) * (pf::RQ_LD / 4) + 8 * ks;
+                        const uint32_t* r1 = r0 + 8 * (pf::RQ_LD / 4);
+                        const bool on = ks < ksteps;
+                        afr[mt][ks][0] = on ? r0[t4] : 0u;
+                        afr[mt][ks][1] = on ? r1[t4] : 0u;
+                        afr[mt][ks][2] = on ? r0[4 + t4] : 0u;
+                        afr[mt][ks][3] = on ? r1[4 + t4] : 0u;
+                    }
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(accf_bar(abuf), (aphase >> abuf) & 1u, p.limit_ns));
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < BN / 2 / 32; ++c) {
+                        const int col = hcol * (BN / 2) + c * 32;
+                        if (n0 + col >= p.N) break;
+                        drain_sym_chunk<OUT>(p,
+                                             tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                                 static_cast<uint32_t>(abuf * BN + col),
+                                             mq0, n0 + col, col, sw_s, sr_s, rq_s, afr, ksteps, sxr, g8, t4);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(acce_remote0 + 8u * static_cast<uint32_t>(abuf));
+                }
+                aphase ^= 1u << abuf;
+                abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
+            }
+        } else {
+        const int rwords = p.r / 4;
         for (int tile = pair; tile < num_tiles; tile += npairs) {
             const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM, n0 = (tile / MT) * BN;
             const int m = m0 + row;
@@ -587,6 +768,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                     named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
                 }
             }
+        }
         }
     }
 

@@ -231,6 +231,30 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)
         : "r"(taddr));
 }
 
+// 16 lanes x (8 columns x 4): thread i of the warp receives lanes base + i/4
+// and base + i/4 + 8, columns 2 (i%4) and 2 (i%4) + 1 of each group of 8
+// columns: v[4g + 0,1] = lane base + i/4, v[4g + 2,3] = lane base + i/4 + 8
+// for column group g (the accumulator layout of mma.sync m16n8).
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+// Warp-level int8 MMA, 16 x 8 x 32, int32 accumulate in registers:
+// a = rows g, g+8 (g = lane/4) x K bytes 4 (lane%4) .. +3 and 16 + 4 (lane%4) .. +3;
+// b = K bytes 4 (lane%4) .. +3 and 16 + .. of column g; c as tmem_ld_16x256b.
+__device__ __forceinline__ void mma_s8_16x8x32(int32_t (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // 32 lanes x 16 columns.
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
     asm volatile(
