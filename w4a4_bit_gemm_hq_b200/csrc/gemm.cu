@@ -652,123 +652,180 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
             }
         } else {
-        const int rwords = p.r / 4;
-        for (int tile = pair; tile < num_tiles; tile += npairs) {
-            const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM, n0 = (tile / MT) * BN;
-            const int m = m0 + row;
-            const bool mvalid = m < p.M;
-            // ---- stage the tile's column data while its MMAs run
-            named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);   // previous tile's readers are done
-            if (et < BN) stage_column<OUT>(p, n0 + et, sw_s + et, sr_s + et, rq_s + et * pf::RQ_LD);
-            float sxm = 0.f;
-            if constexpr (OUT != OUT_DEBUG) sxm = mvalid ? __ldg(p.sx + m) : 0.f;
-            uint32_t xs[16];
-            gather_xs(p, sal_s, m, xs);
-            named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
-            constexpr int NCHUNK = BN / 2 / 32;
-            float ypart[ASYM ? NCHUNK * 32 : 1];
-            if constexpr (ASYM) {
-                // SERQ term first: ypart = sr[n] * (X[m,S] . R[n,:])
+            // group weights: one accumulator per (tile, group); per-thread fp32
+            // partial sums in the mma.sync fragment layout, 64 columns x the
+            // warp's 32 rows: ypart[chunk][row half][8-col group][4]
+            const uint32_t* xs_w = reinterpret_cast<const uint32_t*>(smem + L::OFF_XS);
+            const int g8 = lane >> 2, t4 = lane & 3;
+            const int ksteps = (p.r + 31) / 32;
+            constexpr int NC = BN / 2 / 32;   // 32-column chunks per warp
+            for (int tile = pair; tile < num_tiles; tile += npairs) {
+                const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM, n0 = (tile / MT) * BN;
+                const int mq0 = m0 + 32 * q;
+                named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);   // previous tile's readers are done
+                if (et < BN) stage_column<OUT>(p, n0 + et, sw_s + et, sr_s + et, rq_s + et * pf::RQ_LD);
+                if (p.r > 0)
+                    gather_xs_smem(p, sal_s, m0 + row,
+                                   reinterpret_cast<uint32_t*>(smem + L::OFF_XS + row * pf::RQ_LD), hcol, 4 * ksteps);
+                float sxr[2][2];
 #pragma unroll
-                for (int c = 0; c < NCHUNK; ++c) {
-                    const int col = hcol * (BN / 2) + c * 32;
+                for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int cc = (p.r > 0) ? corr_dot(xs, rq_s + (col + j) * pf::RQ_LD, rwords) : 0;
-                        if constexpr (OUT == OUT_DEBUG) {
-                            if (p.r > 0 && mvalid && n0 + col + j < p.N)
-                                p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n0 + col + j] = cc;
-                            ypart[c * 32 + j] = 0.f;
-                        } else {
-                            ypart[c * 32 + j] = (p.r > 0) ? __fmul_rn(sr_s[col + j], static_cast<float>(cc)) : 0.f;
-                        }
+                    for (int h = 0; h < 2; ++h) {
+                        const int m = mq0 + 16 * mt + g8 + 8 * h;
+                        sxr[mt][h] = 0.f;
+                        if constexpr (OUT != OUT_DEBUG) sxr[mt][h] = m < p.M ? __ldg(p.sx + m) : 0.f;
                     }
-                }
-            }
-            for (int g = 0; g < NG; ++g) {
-                float swn = 0.f;   // sw of group g + 1, column n0 + et (group weights)
-                if constexpr (ASYM && OUT != OUT_DEBUG) {
-                    if (g + 1 < NG && et < BN && n0 + et < p.N)
-                        swn = __half2float(__ushort_as_half(__ldg(p.sw + static_cast<int64_t>(g + 1) * p.N + n0 + et)));
-                }
-                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(accf_bar(abuf), (aphase >> abuf) & 1u, p.limit_ns));
-                if (ok) {
-                    tc_fence_after();
-                    const float* swg = sw_s + (ASYM ? (g & 1) * BN : 0);
+                named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
+                // ---- SERQ term first: ypart = sr[n] * (X[m,S] . Rq[n,:])
+                float ypart[NC][2][4][4];
+                {
+                    uint32_t afr[2][2][4];
 #pragma unroll
-                    for (int c = 0; c < NCHUNK; ++c) {
-                        const int col = hcol * (BN / 2) + c * 32;
-                        const int nb = n0 + col;
-                        uint32_t acc[32];
-                        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                                               static_cast<uint32_t>(abuf * BN + col), acc);
-                        tmem_wait_ld();
-                        if (nb >= p.N) continue;
-                        const int nvalid = p.N - nb;
-                        if constexpr (OUT == OUT_DEBUG) {
-                            if (mvalid) {
-                                const int sh = ASYM ? 4 : 8;
-                                for (int j = 0; j < 32 && j < nvalid; ++j)
-                                    p.dbg_acc[(static_cast<int64_t>(m) * p.N + nb + j) * NG + g] =
-                                        static_cast<int32_t>(acc[j]) >> sh;
-                                if constexpr (!ASYM) {
-                                    if (p.r > 0) {
-                                        for (int j = 0; j < 32 && j < nvalid; ++j)
-                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + nb + j] =
-                                                corr_dot(xs, rq_s + (col + j) * pf::RQ_LD, rwords);
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const uint32_t* r0 = xs_w + (32 * q + 16 * mt + g8) * (pf::RQ_LD / 4) + 8 * ks;
+                            const uint32_t* r1 = r0 + 8 * (pf::RQ_LD / 4);
+                            const bool on = ks < ksteps;
+                            afr[mt][ks][0] = on ? r0[t4] : 0u;
+                            afr[mt][ks][1] = on ? r1[t4] : 0u;
+                            afr[mt][ks][2] = on ? r0[4 + t4] : 0u;
+                            afr[mt][ks][3] = on ? r1[4 + t4] : 0u;
+                        }
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) {
+                        const int scol = hcol * (BN / 2) + 32 * c;
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) {
+                            int32_t cc[4][4];
+#pragma unroll
+                            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) cc[nt][i] = 0;
+#pragma unroll
+                            for (int ks = 0; ks < 2; ++ks) {
+                                if (ks < ksteps) {
+#pragma unroll
+                                    for (int nt = 0; nt < 4; ++nt) {
+                                        const uint32_t* rw = reinterpret_cast<const uint32_t*>(
+                                                                 rq_s + (scol + 8 * nt + g8) * pf::RQ_LD) + 8 * ks;
+                                        mma_s8_16x8x32(cc[nt], afr[mt][ks], rw[t4], rw[4 + t4]);
                                     }
                                 }
                             }
-                        } else if constexpr (ASYM) {
 #pragma unroll
-                            for (int v = 0; v < 4; ++v) {
+                            for (int nt = 0; nt < 4; ++nt) {
+                                const int cl = scol + 8 * nt + 2 * t4;
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const int j = 8 * v + e;
-                                    ypart[c * 32 + j] = __fmaf_rn(swg[col + j],
-                                                                  static_cast<float>(static_cast<int32_t>(acc[j]) >> 4),
-                                                                  ypart[c * 32 + j]);
+                                for (int i = 0; i < 4; ++i) {
+                                    const int32_t cv = cc[nt][i] >> 4;   // Rq codes carry 16
+                                    if constexpr (OUT == OUT_DEBUG) {
+                                        const int m = mq0 + 16 * mt + g8 + 8 * (i >> 1);
+                                        const int n = n0 + cl + (i & 1);
+                                        if (p.r > 0 && m < p.M && n < p.N)
+                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n] = cv;
+                                        ypart[c][mt][nt][i] = 0.f;
+                                    } else {
+                                        ypart[c][mt][nt][i] =
+                                            (p.r > 0) ? __fmul_rn(sr_s[cl + (i & 1)], static_cast<float>(cv)) : 0.f;
+                                    }
                                 }
-                                if (g == NG - 1 && mvalid && 8 * v < nvalid) {
-                                    float y[8];
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(sxm, ypart[c * 32 + 8 * v + e]);
-                                    store_out8<OUT>(p.Y, static_cast<int64_t>(m) * p.N + nb + 8 * v, y);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                if (8 * v >= nvalid) break;
-                                float y[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const int j = 8 * v + e;
-                                    const int cc = (p.r > 0) ? corr_dot(xs, rq_s + (col + j) * pf::RQ_LD, rwords) : 0;
-                                    const float a = static_cast<float>(static_cast<int32_t>(acc[j]) >> 8);
-                                    const float t = __fmaf_rn(sr_s[col + j], static_cast<float>(cc), __fmul_rn(swg[col + j], a));
-                                    y[e] = __fmul_rn(sxm, t);
-                                }
-                                if (mvalid) store_out8<OUT>(p.Y, static_cast<int64_t>(m) * p.N + nb + 8 * v, y);
                             }
                         }
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acce_remote0 + 8u * static_cast<uint32_t>(abuf));
                 }
-                aphase ^= 1u << abuf;
-                abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
-                if constexpr (ASYM) {
-                    // hand the next group's sw to every warp; the buffer written
-                    // here was last read in group g - 1, before the previous barrier
-                    if constexpr (OUT != OUT_DEBUG) {
-                        if (et < BN) sw_s[((g + 1) & 1) * BN + et] = swn;
+                // ---- sw of group 0 for this thread's columns (fp16 pairs)
+                uint32_t swc[NC][4];
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const int n = n0 + hcol * (BN / 2) + 32 * c + 8 * nt + 2 * t4;
+                        swc[c][nt] = 0u;
+                        if constexpr (OUT != OUT_DEBUG)
+                            if (n < p.N) swc[c][nt] = __ldg(reinterpret_cast<const uint32_t*>(p.sw + n));
                     }
-                    named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
+                for (int g = 0; g < NG; ++g) {
+                    // next group's sw, in flight while this group's accumulator is awaited
+                    uint32_t swn[NC][4];
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+#pragma unroll
+                        for (int nt = 0; nt < 4; ++nt) {
+                            const int n = n0 + hcol * (BN / 2) + 32 * c + 8 * nt + 2 * t4;
+                            swn[c][nt] = 0u;
+                            if constexpr (OUT != OUT_DEBUG)
+                                if (g + 1 < NG && n < p.N)
+                                    swn[c][nt] = __ldg(reinterpret_cast<const uint32_t*>(
+                                        p.sw + static_cast<int64_t>(g + 1) * p.N + n));
+                        }
+                    if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(accf_bar(abuf), (aphase >> abuf) & 1u, p.limit_ns));
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < NC; ++c) {
+                            const int scol = hcol * (BN / 2) + 32 * c;
+#pragma unroll
+                            for (int mt = 0; mt < 2; ++mt) {
+                                uint32_t v[16];
+                                tmem_ld_16x256b_x4(tmem_base + (static_cast<uint32_t>(32 * q + 16 * mt) << 16) +
+                                                       static_cast<uint32_t>(abuf * BN + scol),
+                                                   v);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int nt = 0; nt < 4; ++nt) {
+                                    const float2 swf = __half22float2(*reinterpret_cast<const __half2*>(&swc[c][nt]));
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) {
+                                        const int32_t av = static_cast<int32_t>(v[4 * nt + i]) >> 4;
+                                        if constexpr (OUT == OUT_DEBUG) {
+                                            const int m = mq0 + 16 * mt + g8 + 8 * (i >> 1);
+                                            const int n = n0 + scol + 8 * nt + 2 * t4 + (i & 1);
+                                            if (m < p.M && n < p.N)
+                                                p.dbg_acc[(static_cast<int64_t>(m) * p.N + n) * NG + g] = av;
+                                        } else {
+                                            ypart[c][mt][nt][i] = __fmaf_rn((i & 1) ? swf.y : swf.x,
+                                                                            static_cast<float>(av), ypart[c][mt][nt][i]);
+                                        }
+                                    }
+                                }
+                            }
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acce_remote0 + 8u * static_cast<uint32_t>(abuf));
+                    }
+                    aphase ^= 1u << abuf;
+                    abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+#pragma unroll
+                        for (int nt = 0; nt < 4; ++nt) swc[c][nt] = swn[c][nt];
+                }
+                // ---- Y = sx[m] * ypart
+                if constexpr (OUT != OUT_DEBUG) {
+                    if (ok) {
+#pragma unroll
+                        for (int c = 0; c < NC; ++c)
+#pragma unroll
+                            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                                for (int nt = 0; nt < 4; ++nt) {
+                                    const int64_t n = n0 + hcol * (BN / 2) + 32 * c + 8 * nt + 2 * t4;
+                                    if (n >= p.N) continue;
+#pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        const int m = mq0 + 16 * mt + g8 + 8 * h;
+                                        if (m >= p.M) continue;
+                                        store_out2<OUT>(p.Y, static_cast<int64_t>(m) * p.N + n,
+                                                        __fmul_rn(sxr[mt][h], ypart[c][mt][nt][2 * h]),
+                                                        __fmul_rn(sxr[mt][h], ypart[c][mt][nt][2 * h + 1]));
+                                    }
+                                }
+                    }
                 }
             }
-        }
         }
     }
 
