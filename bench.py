@@ -416,7 +416,7 @@ def main():
     decode_like = M <= 64
     if t_k2 >= t_k1:
         if decode_like:
-            roof = {"kernel": "k_gemm (w4a4_linear)", "bound": "hbm", "achieved": b2 / (t_k2 * 1e-3) / 1e9,
+            roof = {"kernel": "k_gemm_small (w4a4_linear)", "bound": "hbm", "achieved": b2 / (t_k2 * 1e-3) / 1e9,
                     "peak": peaks["hbm"], "unit": "GB/s", "bytes_per_launch": b2}
         else:
             roof = {"kernel": "k_gemm_pf (w4a4_linear)", "bound": "tensor",
