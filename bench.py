@@ -464,18 +464,21 @@ def committed_traffic(workload, M, kernel):
     try:
         d = json.load(open(p))
         e = d.get("%s:M=%d" % (workload, M))
-        if not e or e.get("sources_sha") != sources_sha():
+        if not e or e.get("sources_sha") != sources_sha(e.get("sources")):
             return None
         return e["dram_bytes_per_launch"]
     except (ValueError, KeyError):
         return None
 
 
-def sources_sha():
+def sources_sha(files=None):
+    """Hash of the CUDA sources a captured kernel is built from (all of csrc/
+    when the entry names none): a committed traffic figure is used only while
+    they are unchanged."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "w4a4_bit_gemm_hq_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files if files else os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
     constexpr int HREG = (G < EPT) ? G : EPT;        // in-register stages: h < HREG
     constexpr int TSHFL = (TPG < 32) ? TPG : 32;     // shuffle stages: s < TSHFL
     extern __shared__ float xch[];                   // [EPT][blockDim] exchange (G >= 2048)
-    __shared__ float red[32];
+    __shared__ float red[2][32];   // per-warp maxima, double-buffered by row parity
 
     // a kernel launched after this one with programmatic stream serialization
     // (the small-M GEMM) may start now: it waits for this grid's completion
@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
         }
     };
     load_row(blockIdx.x, raw);
-    for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    int par = 0;
+    for (int64_t m = blockIdx.x; m < M; m += gridDim.x, par ^= 1) {
         load_row(m + gridDim.x, raw_next);
         float2 v[EPT / 2];
         if (active) {
@@ -225,11 +226,13 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             const int nw = nthr >> 5;
             if (nw > 1) {
-                if ((t & 31) == 0) red[t >> 5] = amax;
+                // one barrier per row: the other buffer is written by the next
+                // row, and the one after it only once every thread has passed
+                // the next row's barrier (so has finished reading this one)
+                if ((t & 31) == 0) red[par][t >> 5] = amax;
                 __syncthreads();
                 amax = 0.f;
-                for (int w = 0; w < nw; ++w) amax = fmaxf(amax, red[w]);
-                __syncthreads();  // red is rewritten by the next row
+                for (int w = 0; w < nw; ++w) amax = fmaxf(amax, red[par][w]);
             }
             // ---- scale, round half to even, pack
             uint32_t words[EPT / 8];
