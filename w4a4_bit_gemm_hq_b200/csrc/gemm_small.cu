@@ -518,22 +518,41 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
                 float* part = ws_part + (static_cast<int64_t>(t) * plan.maxc + slot) * NT * sk::BMW;
 #pragma unroll
                 for (int j = 0; j < NT; ++j) part[j * sk::BMW + row] = y[j];
-                __threadfence();
+                // one thread publishes the CTA's partial (the barrier orders every
+                // thread's stores before its fence) and counts the arrival; the
+                // last arriver's thread fences again before the CTA reads the
+                // other contributors' partials
                 named_bar_sync(1, 128);
                 if (ethr == 0) {
+                    __threadfence();
                     const uint32_t old = atomicAdd(ws_cnt + t, 1u);
-                    misc[2] = (old == static_cast<uint32_t>(last - first)) ? 1u : 0u;
+                    const bool last_one = old == static_cast<uint32_t>(last - first);
+                    if (last_one) __threadfence();
+                    misc[2] = last_one ? 1u : 0u;
                 }
                 named_bar_sync(1, 128);
                 finish = misc[2] != 0;
                 if (finish) {
-                    __threadfence();
 #pragma unroll
                     for (int j = 0; j < NT; ++j) y[j] = 0.f;
-                    for (int c = 0; c <= last - first; ++c) {
-                        const float* pc = ws_part + (static_cast<int64_t>(t) * plan.maxc + c) * NT * sk::BMW;
+                    // all contributors' partials, CB at a time in flight, summed in slot order
+                    constexpr int CB = NT <= 16 ? 4 : (NT <= 32 ? 2 : 1);
+                    const int nc = last - first + 1;
+                    for (int c0 = 0; c0 < nc; c0 += CB) {
+                        float pv[CB][NT];
 #pragma unroll
-                        for (int j = 0; j < NT; ++j) y[j] = __fadd_rn(y[j], __ldcg(pc + j * sk::BMW + row));
+                        for (int cc = 0; cc < CB; ++cc) {
+                            const float* pc = ws_part + (static_cast<int64_t>(t) * plan.maxc + c0 + cc) * NT * sk::BMW;
+#pragma unroll
+                            for (int j = 0; j < NT; ++j) pv[cc][j] = (c0 + cc < nc) ? __ldcg(pc + j * sk::BMW + row) : 0.f;
+                        }
+#pragma unroll
+                        for (int cc = 0; cc < CB; ++cc) {
+                            if (c0 + cc < nc) {
+#pragma unroll
+                                for (int j = 0; j < NT; ++j) y[j] = __fadd_rn(y[j], pv[cc][j]);
+                            }
+                        }
                     }
                     if (ethr == 0) ws_cnt[t] = 0u;   // ready for the next call
                 }
