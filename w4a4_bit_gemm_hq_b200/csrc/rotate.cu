@@ -169,103 +169,237 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 }
             }
         }
-        // ---- shuffle stages: partner thread t ^ s holds channels +-32s
+        if constexpr (G == 4096) {
+            // ---- groups of 4096 (128 threads each): the remaining 7 stages run
+            // in registers between two shared-memory transposes.
+            // Channel i of the group = 1024 ah + 32 al + b.  So far thread
+            // (warp ah, lane al) holds b = 0..31.
+            const int tg = t & 127, wg = tg >> 5, ln = t & 31;
+            float* ta = xch + (t >> 7) * 4096 + wg * 1024;                          // this warp's 32 x 32 block
+            float* tb = xch + static_cast<size_t>(EPT) * nthr + (t >> 7) * 4096;    // the group's 4096 channels
+            // T1, within the warp: lane al writes row al (16-byte chunk k of the
+            // row at chunk k ^ (al & 7)), then lane b reads column b.
 #pragma unroll
-        for (int s = 1; s < TSHFL; s <<= 1) {
-            const bool upper = (t & s) != 0;
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4*>(ta + ln * 32 + 4 * (k ^ (ln & 7))) =
+                    make_float4(v[2 * k].x, v[2 * k].y, v[2 * k + 1].x, v[2 * k + 1].y);
+            __syncwarp();
+            float2 u[EPT / 2];   // u[j] = channels al = 2j, 2j+1 of column b = lane
 #pragma unroll
-            for (int i = 0; i < EPT / 2; ++i) {
-                float2 p;
-                p.x = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, s);
-                p.y = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, s);
-                v[i] = upper ? f2sub(p, v[i]) : f2add_rn(v[i], p);
+            for (int j = 0; j < EPT / 2; ++j) {
+                u[j].x = ta[(2 * j) * 32 + 4 * ((ln >> 2) ^ ((2 * j) & 7)) + (ln & 3)];
+                u[j].y = ta[(2 * j + 1) * 32 + 4 * ((ln >> 2) ^ ((2 * j + 1) & 7)) + (ln & 3)];
             }
-        }
-        // ---- cross-warp stages through shared memory (G >= 2048)
-        if constexpr (TPG > 32) {
+            // stages h = 32 .. 512: pairs (al, al + h/32), in registers
 #pragma unroll
-            for (int s = 32; s < TPG; s <<= 1) {
-                const bool upper = (t & s) != 0;
-#pragma unroll
-                for (int i = 0; i < EPT / 2; ++i) {
-                    xch[(2 * i) * nthr + t] = v[i].x;
-                    xch[(2 * i + 1) * nthr + t] = v[i].y;
-                }
-                __syncthreads();
-#pragma unroll
-                for (int i = 0; i < EPT / 2; ++i) {
-                    float2 p = make_float2(xch[(2 * i) * nthr + (t ^ s)], xch[(2 * i + 1) * nthr + (t ^ s)]);
-                    v[i] = upper ? f2sub(p, v[i]) : f2add_rn(v[i], p);
-                }
-                __syncthreads();
+            for (int j = 0; j < EPT / 2; ++j) {
+                const float a0 = u[j].x, b0 = u[j].y;
+                u[j].x = __fadd_rn(a0, b0);
+                u[j].y = __fsub_rn(a0, b0);
             }
-        }
-
-        if constexpr (MODE == MODE_ROTATE) {
-            if (active) {
-                float4* dst = reinterpret_cast<float4*>(out + m * K + col0);
-                const float2 c2 = make_float2(cg, cg);
 #pragma unroll
-                for (int j = 0; j < EPT / 4; ++j) {
-                    const float2 a = f2mul_rn(v[2 * j], c2), b = f2mul_rn(v[2 * j + 1], c2);
-                    dst[j] = make_float4(a.x, a.y, b.x, b.y);
+            for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+                for (int i = 0; i < EPT; i += 2) {
+                    if ((i & h) == 0) {
+                        const float2 a0 = u[i / 2], b0 = u[(i + h) / 2];
+                        u[i / 2] = f2add_rn(a0, b0);
+                        u[(i + h) / 2] = f2sub(a0, b0);
+                    }
                 }
             }
-        } else if constexpr (MODE == MODE_SQNORM) {
+            // T2, across the group's 4 warps: channel i stored at
+            // i ^ (4 (al & 1)); thread (al = tg / 4, c = tg % 4) then reads
+            // channels 1024 ah + 32 al + 8 c + e for ah = 0..3, e = 0..7.
 #pragma unroll
-            for (int i = 0; i < EPT / 2; ++i) {
-                accsq[2 * i] = __fmaf_rn(v[i].x, v[i].x, accsq[2 * i]);
-                accsq[2 * i + 1] = __fmaf_rn(v[i].y, v[i].y, accsq[2 * i + 1]);
+            for (int j = 0; j < EPT / 2; ++j) {
+                tb[wg * 1024 + (2 * j) * 32 + ln] = u[j].x;
+                tb[wg * 1024 + (2 * j + 1) * 32 + (ln ^ 4)] = u[j].y;
             }
-        } else {
-            // ---- per-token absmax over the whole row
-            float amax = 0.f;
+            __syncthreads();
+            const int al = tg >> 2, c4 = tg & 3;
+            float w[4][8];
 #pragma unroll
-            for (int i = 0; i < EPT / 2; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+            for (int ah = 0; ah < 4; ++ah) {
+                const float* src = tb + ah * 1024 + al * 32;
+                const float4 p0 = *reinterpret_cast<const float4*>(src + 4 * ((2 * c4) ^ (al & 1)));
+                const float4 p1 = *reinterpret_cast<const float4*>(src + 4 * ((2 * c4 + 1) ^ (al & 1)));
+                w[ah][0] = p0.x; w[ah][1] = p0.y; w[ah][2] = p0.z; w[ah][3] = p0.w;
+                w[ah][4] = p1.x; w[ah][5] = p1.y; w[ah][6] = p1.z; w[ah][7] = p1.w;
+            }
+            // stages h = 1024 (ah ^ 1), then 2048 (ah ^ 2)
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-            const int nw = nthr >> 5;
-            if (nw > 1) {
-                // one barrier per row: the other buffer is written by the next
-                // row, and the one after it only once every thread has passed
-                // the next row's barrier (so has finished reading this one)
+            for (int hb = 1; hb <= 2; hb <<= 1) {
+#pragma unroll
+                for (int ah = 0; ah < 4; ++ah) {
+                    if ((ah & hb) == 0) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float a0 = w[ah][e], b0 = w[ah + hb][e];
+                            w[ah][e] = __fadd_rn(a0, b0);
+                            w[ah + hb][e] = __fsub_rn(a0, b0);
+                        }
+                    }
+                }
+            }
+            // channel of w[ah][e] within the row: grp0 + 1024 ah + e
+            const int64_t grp0 = static_cast<int64_t>(t >> 7) * 4096 + 32 * al + 8 * c4;
+            if constexpr (MODE == MODE_ROTATE) {
+#pragma unroll
+                for (int ah = 0; ah < 4; ++ah) {
+                    float4* dst = reinterpret_cast<float4*>(out + m * K + grp0 + 1024 * ah);
+                    const float2 c2 = make_float2(cg, cg);
+                    const float2 a0 = f2mul_rn(make_float2(w[ah][0], w[ah][1]), c2);
+                    const float2 a1 = f2mul_rn(make_float2(w[ah][2], w[ah][3]), c2);
+                    const float2 a2 = f2mul_rn(make_float2(w[ah][4], w[ah][5]), c2);
+                    const float2 a3 = f2mul_rn(make_float2(w[ah][6], w[ah][7]), c2);
+                    dst[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
+                    dst[1] = make_float4(a2.x, a2.y, a3.x, a3.y);
+                }
+            } else if constexpr (MODE == MODE_SQNORM) {
+#pragma unroll
+                for (int ah = 0; ah < 4; ++ah)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) accsq[8 * ah + e] = __fmaf_rn(w[ah][e], w[ah][e], accsq[8 * ah + e]);
+            }
+            if constexpr (MODE != MODE_QUANT) {
+                __syncthreads();   // the next row rewrites the cross-warp buffer
+            } else {
+                float amax = 0.f;
+#pragma unroll
+                for (int ah = 0; ah < 4; ++ah)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(w[ah][e]));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+                const int nw = nthr >> 5;
                 if ((t & 31) == 0) red[par][t >> 5] = amax;
                 __syncthreads();
                 amax = 0.f;
-                for (int w = 0; w < nw; ++w) amax = fmaxf(amax, red[par][w]);
-            }
-            // ---- scale, round half to even, pack
-            uint32_t words[EPT / 8];
-            if (amax == 0.f) {
+                for (int wi = 0; wi < nw; ++wi) amax = fmaxf(amax, red[par][wi]);
+                uint32_t words[4] = {0u, 0u, 0u, 0u};
+                if (amax != 0.f) {
+                    const float inv = __fdiv_rn(7.0f, amax);
+                    const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
 #pragma unroll
-                for (int j = 0; j < EPT / 8; ++j) words[j] = 0u;
-            } else {
-                const float inv = __fdiv_rn(7.0f, amax);
-                const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+                    for (int ah = 0; ah < 4; ++ah) {
+                        uint32_t wd = 0;
 #pragma unroll
-                for (int j = 0; j < EPT / 8; ++j) {
-                    uint32_t w = 0;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        // |u * inv| <= 7 (1 + 2^-23): adding 1.5*2^23 rounds it to an
-                        // integer with ties to even; the low nibble of the sum's bits is
-                        // that integer in two's complement.
-                        // __fmul_rn is never merged into an fma, so fl32(u * inv) is
-                        // rounded before the rounding add, as the codes are defined.
-                        const float2 t = make_float2(__fmul_rn(v[4 * j + e].x, inv), __fmul_rn(v[4 * j + e].y, inv));
-                        const float2 r = f2add_rn(t, magic);
-                        const uint32_t b0 = __float_as_uint(r.x) & 0xFu;
-                        const uint32_t b1 = __float_as_uint(r.y) & 0xFu;
-                        w |= (b0 | (b1 << 4)) << (8 * e);
+                        for (int e = 0; e < 8; e += 2) {
+                            // fl32(u * inv) rounded (never merged into an fma), then the
+                            // round-half-even add; the low nibble is the code
+                            const float2 tq = make_float2(__fmul_rn(w[ah][e], inv), __fmul_rn(w[ah][e + 1], inv));
+                            const float2 r = f2add_rn(tq, magic);
+                            wd |= ((__float_as_uint(r.x) & 0xFu) | ((__float_as_uint(r.y) & 0xFu) << 4)) << (4 * e);
+                        }
+                        words[ah] = wd;
                     }
-                    words[j] = w;
+                }
+                uint8_t* qrow = Xq + m * (K / 2);
+#pragma unroll
+                for (int ah = 0; ah < 4; ++ah)
+                    *reinterpret_cast<uint32_t*>(qrow + (grp0 + 1024 * ah) / 2) = words[ah];
+                if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+            }
+        } else {
+            // ---- shuffle stages: partner thread t ^ s holds channels +-32s
+    #pragma unroll
+            for (int s = 1; s < TSHFL; s <<= 1) {
+                const bool upper = (t & s) != 0;
+    #pragma unroll
+                for (int i = 0; i < EPT / 2; ++i) {
+                    float2 p;
+                    p.x = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, s);
+                    p.y = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, s);
+                    v[i] = upper ? f2sub(p, v[i]) : f2add_rn(v[i], p);
                 }
             }
-            if (active) {
-                uint4* dst = reinterpret_cast<uint4*>(Xq + m * (K / 2) + col0 / 2);
-                *dst = make_uint4(words[0], words[1], words[2], words[3]);
+            // ---- cross-warp stages through shared memory (G >= 2048)
+            if constexpr (TPG > 32) {
+    #pragma unroll
+                for (int s = 32; s < TPG; s <<= 1) {
+                    const bool upper = (t & s) != 0;
+    #pragma unroll
+                    for (int i = 0; i < EPT / 2; ++i) {
+                        xch[(2 * i) * nthr + t] = v[i].x;
+                        xch[(2 * i + 1) * nthr + t] = v[i].y;
+                    }
+                    __syncthreads();
+    #pragma unroll
+                    for (int i = 0; i < EPT / 2; ++i) {
+                        float2 p = make_float2(xch[(2 * i) * nthr + (t ^ s)], xch[(2 * i + 1) * nthr + (t ^ s)]);
+                        v[i] = upper ? f2sub(p, v[i]) : f2add_rn(v[i], p);
+                    }
+                    __syncthreads();
+                }
             }
-            if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+
+            if constexpr (MODE == MODE_ROTATE) {
+                if (active) {
+                    float4* dst = reinterpret_cast<float4*>(out + m * K + col0);
+                    const float2 c2 = make_float2(cg, cg);
+    #pragma unroll
+                    for (int j = 0; j < EPT / 4; ++j) {
+                        const float2 a = f2mul_rn(v[2 * j], c2), b = f2mul_rn(v[2 * j + 1], c2);
+                        dst[j] = make_float4(a.x, a.y, b.x, b.y);
+                    }
+                }
+            } else if constexpr (MODE == MODE_SQNORM) {
+    #pragma unroll
+                for (int i = 0; i < EPT / 2; ++i) {
+                    accsq[2 * i] = __fmaf_rn(v[i].x, v[i].x, accsq[2 * i]);
+                    accsq[2 * i + 1] = __fmaf_rn(v[i].y, v[i].y, accsq[2 * i + 1]);
+                }
+            } else {
+                // ---- per-token absmax over the whole row
+                float amax = 0.f;
+    #pragma unroll
+                for (int i = 0; i < EPT / 2; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+    #pragma unroll
+                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+                const int nw = nthr >> 5;
+                if (nw > 1) {
+                    // one barrier per row: the other buffer is written by the next
+                    // row, and the one after it only once every thread has passed
+                    // the next row's barrier (so has finished reading this one)
+                    if ((t & 31) == 0) red[par][t >> 5] = amax;
+                    __syncthreads();
+                    amax = 0.f;
+                    for (int w = 0; w < nw; ++w) amax = fmaxf(amax, red[par][w]);
+                }
+                // ---- scale, round half to even, pack
+                uint32_t words[EPT / 8];
+                if (amax == 0.f) {
+    #pragma unroll
+                    for (int j = 0; j < EPT / 8; ++j) words[j] = 0u;
+                } else {
+                    const float inv = __fdiv_rn(7.0f, amax);
+                    const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    #pragma unroll
+                    for (int j = 0; j < EPT / 8; ++j) {
+                        uint32_t w = 0;
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            // |u * inv| <= 7 (1 + 2^-23): adding 1.5*2^23 rounds it to an
+                            // integer with ties to even; the low nibble of the sum's bits is
+                            // that integer in two's complement.
+                            // __fmul_rn is never merged into an fma, so fl32(u * inv) is
+                            // rounded before the rounding add, as the codes are defined.
+                            const float2 t = make_float2(__fmul_rn(v[4 * j + e].x, inv), __fmul_rn(v[4 * j + e].y, inv));
+                            const float2 r = f2add_rn(t, magic);
+                            const uint32_t b0 = __float_as_uint(r.x) & 0xFu;
+                            const uint32_t b1 = __float_as_uint(r.y) & 0xFu;
+                            w |= (b0 | (b1 << 4)) << (8 * e);
+                        }
+                        words[j] = w;
+                    }
+                }
+                if (active) {
+                    uint4* dst = reinterpret_cast<uint4*>(Xq + m * (K / 2) + col0 / 2);
+                    *dst = make_uint4(words[0], words[1], words[2], words[3]);
+                }
+                if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+            }
         }
 #pragma unroll
         for (int j = 0; j < NRAW; ++j) raw[j] = raw_next[j];
@@ -273,8 +407,17 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
 
     if constexpr (MODE == MODE_SQNORM) {
         if (active) {
+            if constexpr (G == 4096) {
+                const int tg = t & 127;
+                const int64_t grp0 = static_cast<int64_t>(t >> 7) * 4096 + 32 * (tg >> 2) + 8 * (tg & 3);
 #pragma unroll
-            for (int i = 0; i < EPT; ++i) atomicAdd(out + col0 + i, accsq[i]);
+                for (int ah = 0; ah < 4; ++ah)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) atomicAdd(out + grp0 + 1024 * ah + e, accsq[8 * ah + e]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < EPT; ++i) atomicAdd(out + col0 + i, accsq[i]);
+            }
         }
     }
 }
@@ -285,7 +428,9 @@ static hq_status launch_g(int group, const void* X, int64_t M, int64_t K, int64_
                           float* sx, float* out, cudaStream_t st) {
     const int threads = static_cast<int>(((K / EPT) + 31) / 32 * 32);
     const float cg = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(group)));
-    const size_t shm = (group >= 2048) ? static_cast<size_t>(EPT) * threads * sizeof(float) : 0;
+    // G >= 2048: exchange area of EPT floats per thread; G == 4096 uses two
+    // (the warp transposes and the cross-warp transpose)
+    const size_t shm = (group >= 2048) ? static_cast<size_t>(EPT) * threads * sizeof(float) * (group == 4096 ? 2 : 1) : 0;
     int nsm = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
