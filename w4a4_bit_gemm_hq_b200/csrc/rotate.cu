@@ -435,7 +435,7 @@ static hq_status launch_g(int group, const void* X, int64_t M, int64_t K, int64_
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     auto run = [&](auto kern) -> hq_status {
-        if (shm > 48 * 1024) {
+        if (shm > 32 * 1024) {   // with the static smem, anything near 48 KB needs the opt-in
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shm)) !=
                 cudaSuccess)
                 return HQ_ERR_CUDA;
