@@ -262,6 +262,10 @@ GEMM_CASES = [
     (300, 512, 2048, 256, 64),
     (129, 1032, 384, 0, 24),
     (64, 384, 4096, 128, 16),
+    # per-channel weights with r > 32: the epilogue's SERQ term takes two
+    # 32-wide mma.sync K steps (the second one ragged for r = 40)
+    (256, 512, 1024, 0, 64),
+    (300, 264, 512, 0, 40),
 ]
 
 
