@@ -31,11 +31,13 @@
 //    weights) or of a weight group (group weights) a multicast commit hands the
 //    buffer to the epilogues of both CTAs.
 //  * 8 epilogue warps per CTA (2 per TMEM lane quarter, splitting the
-//    columns) stage the tile's sw, sr and unpacked Rq rows in smem while the
-//    tile's MMAs run, then load the accumulator with tcgen05.ld, dequantise
-//    with sx[m] * sw[n] (or sum the per-group sw[b][n] * acc_b), add
-//    sr[n] * (X[m,S] . Rq[n,:]) computed with dp4a (the SERQ term as an
-//    epilogue add: no second launch), round once and store.
+//    columns) stage the tile's sw, sr, unpacked Rq rows and salient
+//    activation codes X[m,S] in smem while the tile's MMAs run, then load the
+//    accumulator with tcgen05.ld 16x256b (the mma.sync m16n8 fragment
+//    layout), compute the SERQ term X[m,S] . Rq[n,:] with mma.sync m16n8k32
+//    on the staged int8 codes in the same layout (an epilogue add: no second
+//    launch), dequantise with sx[m] * sw[n] (or sum the per-group
+//    sw[b][n] * acc_b), round once and store.
 //  * every mbarrier wait is bounded; on timeout the status word records
 //    HQ_ERR_TIMEOUT and the roles skip to teardown, which waits for in-flight
 //    MMAs before freeing tensor memory.
@@ -137,32 +139,6 @@ __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, i
         }
         *reinterpret_cast<uint4*>(base + swz_chunk(row, 2 * c) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(base + swz_chunk(row, 2 * c + 1) * 16) = make_uint4(o[4], o[5], o[6], o[7]);
-    }
-}
-
-// Gathered salient activation codes of row m as int8 words in the lo/hi
-// permutation of unpack_s4x8_times16 (plain codes, not scaled by 16):
-// position j = 8 i + 2 e + h -> word 2 i + h, byte e.  Eight loads in flight
-// per batch of eight positions (r is a multiple of 8).
-__device__ __forceinline__ void gather_xs(const GemmArgs& p, const int32_t* sal_s, int m, uint32_t (&xs)[16]) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) xs[i] = 0;
-    if (m >= p.M || p.r == 0) return;
-    const uint8_t* row = p.Xq + static_cast<int64_t>(m) * (p.K / 2);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        if (8 * i >= p.r) break;
-        uint32_t nib[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const int k = sal_s[8 * i + t];
-            nib[t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const uint32_t code = static_cast<uint32_t>(static_cast<int>(nib[t] ^ 8u) - 8) & 0xFFu;
-            xs[2 * i + (t & 1)] |= code << (8 * (t >> 1));
-        }
     }
 }
 
@@ -310,99 +286,6 @@ __device__ __forceinline__ void drain_sym_chunk(const GemmArgs& p, uint32_t tm, 
                     store_out2<OUT>(p.Y, off, y0, y1);
                 }
             }
-        }
-    }
-}
-
-__device__ __forceinline__ int corr_dot(const uint32_t (&xs)[16], const uint8_t* rq_row, int nwords) {
-    int acc = 0;
-    const uint4* rv = reinterpret_cast<const uint4*>(rq_row);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (4 * i < nwords) {
-            const uint4 q = rv[i];
-            acc = __dp4a(static_cast<int>(xs[4 * i + 0]), static_cast<int>(q.x), acc);
-            acc = __dp4a(static_cast<int>(xs[4 * i + 1]), static_cast<int>(q.y), acc);
-            acc = __dp4a(static_cast<int>(xs[4 * i + 2]), static_cast<int>(q.z), acc);
-            acc = __dp4a(static_cast<int>(xs[4 * i + 3]), static_cast<int>(q.w), acc);
-        }
-    }
-    return acc >> 4;  // Rq entries carry a factor 16
-}
-
-template <int OUT>
-__device__ __forceinline__ void store_out32(void* Y, int64_t off, const float (&y)[32], int nvalid) {
-    if constexpr (OUT == HQ_F32) {
-        float4* d = reinterpret_cast<float4*>(static_cast<float*>(Y) + off);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-            if (8 * (v / 2) < nvalid) d[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
-    } else {
-        uint4* d = reinterpret_cast<uint4*>(static_cast<uint16_t*>(Y) + off);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            if (8 * v >= nvalid) break;
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a = y[8 * v + 2 * e], b = y[8 * v + 2 * e + 1];
-                if constexpr (OUT == HQ_BF16) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-                    w[e] = *reinterpret_cast<uint32_t*>(&h);
-                } else {
-                    __half2 h = __floats2half2_rn(a, b);
-                    w[e] = *reinterpret_cast<uint32_t*>(&h);
-                }
-            }
-            d[v] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    }
-}
-
-template <int OUT>
-__device__ __forceinline__ void store_out8(void* Y, int64_t off, const float (&y)[8]) {
-    if constexpr (OUT == HQ_F32) {
-        float4* d = reinterpret_cast<float4*>(static_cast<float*>(Y) + off);
-        d[0] = make_float4(y[0], y[1], y[2], y[3]);
-        d[1] = make_float4(y[4], y[5], y[6], y[7]);
-    } else {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if constexpr (OUT == HQ_BF16) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * e], y[2 * e + 1]);
-                w[e] = *reinterpret_cast<uint32_t*>(&h);
-            } else {
-                __half2 h = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
-                w[e] = *reinterpret_cast<uint32_t*>(&h);
-            }
-        }
-        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(Y) + off) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-__device__ __forceinline__ void load_h8(const uint16_t* src, float (&o)[8]) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(src));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-        o[2 * e] = f.x;
-        o[2 * e + 1] = f.y;
-    }
-}
-
-__device__ __forceinline__ void load_h32(const uint16_t* src, float (&o)[32]) {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        const uint4 q = __ldg(s + v);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-            o[8 * v + 2 * e] = f.x;
-            o[8 * v + 2 * e + 1] = f.y;
         }
     }
 }
