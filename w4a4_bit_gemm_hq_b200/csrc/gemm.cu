@@ -41,6 +41,7 @@
 //  * every mbarrier wait is bounded; on timeout the status word records
 //    HQ_ERR_TIMEOUT and the roles skip to teardown, which waits for in-flight
 //    MMAs before freeing tensor memory.
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 #include <cuda.h>
@@ -777,17 +778,19 @@ static hq_status launch_pf_t(const GemmArgs& a, cudaStream_t st, int nsm) {
     // CTA pairs that fit on the device at once (a pair needs two SMs of one
     // cluster-capable group, so this can be below nsm / 2); queried once per
     // device and kernel variant
-    static int max_pairs[64] = {};
+    // (host threads may launch concurrently: the cache entries are atomic, and
+    // a race only repeats the query)
+    static std::atomic<int> max_pairs[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HQ_ERR_CUDA;
-    if (max_pairs[dev] == 0) {
+    int mp = max_pairs[dev].load(std::memory_order_relaxed);
+    if (mp == 0) {
         cfg.gridDim = dim3(2 * (nsm / 2), 1, 1);
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return HQ_ERR_CUDA;
-        max_pairs[dev] = n;
+        if (cudaOccupancyMaxActiveClusters(&mp, kern, &cfg) != cudaSuccess || mp <= 0) return HQ_ERR_CUDA;
+        max_pairs[dev].store(mp, std::memory_order_relaxed);
     }
     const int tiles = ((a.M + 2 * pf::BM - 1) / (2 * pf::BM)) * ((a.N + BN - 1) / BN);
-    const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    const int pairs = tiles < mp ? tiles : mp;
     cfg.gridDim = dim3(2 * pairs, 1, 1);
     if (cudaLaunchKernelEx(&cfg, kern, a, tmX) != cudaSuccess) return HQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
