@@ -193,7 +193,8 @@ hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* 
  *           multiple of 128
  *  A, B     device, serq_prepare outputs Rq [N][ceil(r/2)] and sr [N] (NULL if r == 0)
  *  sal_idx  device, [r] int32 (NULL if r == 0)
- *  r        0 <= r <= 128
+ *  r        0 <= r <= K (HQ_ERR_ARG otherwise); the kernels implement r <= 64
+ *           with r % 8 == 0 (HQ_ERR_UNSUPPORTED otherwise)
  *  Y        device, [M][N] of type yt (HQ_F16, HQ_BF16 or HQ_F32) (output)
  *  workspace, ws_bytes   device scratch of at least
  *           hq_linear_workspace_size(M, N, K, group) bytes (may be NULL when
