@@ -230,6 +230,31 @@ def config_dict(wl, M, pool, n):
     return c
 
 
+# ----------------------------------------------------------------- ranks
+# One process per GPU, each a full replica of the layer on its own token
+# batches (the layer has no exchange step); these helpers are the only
+# cross-rank logic and work with any torch.distributed backend.
+def max_over_ranks(ms, pg, device):
+    """The slowest rank's duration: the job is done when every replica is."""
+    if pg is None:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(ops_per_unit, units_per_rank, world, ms):
+    """Whole-job throughput: the work all ranks did over the slowest rank's time."""
+    return ops_per_unit * units_per_rank * world / (ms * 1e-3) / 1e12
+
+
+def replica_seed(rank, i):
+    """Seed of token batch i of rank `rank`: replicas process different batches."""
+    return 1000 * rank + i
+
+
 # ----------------------------------------------------------------- main
 def main():
     args = parse()
@@ -274,7 +299,7 @@ def main():
         return torch.from_numpy(a).to(dev)
 
     # ---- one prepared layer, then a pool of distinct copies
-    X0 = synth.activations(wl, seed=rank, M=M)
+    X0 = synth.activations(wl, seed=replica_seed(rank, 0), M=M)
     W0 = synth.weights(wl, seed=rank)
     d = torch.from_numpy(synth.hadamard_signs(wl.g, seed=rank)).to(dev)
     Xd0 = to_dev(X0, wl.xdtype)
@@ -287,7 +312,7 @@ def main():
         clone = lambda t: None if t is None else t.clone()
         layers.append(hq.W4A4Linear(base.group, base.gw, base.H_signs, clone(base.Wq), clone(base.sw),
                                     clone(base.zw), clone(base.Rq), clone(base.sr), base.sal_idx, wl.K, wl.N, xdt))
-        Xs.append(Xd0 if i == 0 else torch.from_numpy(synth.activations(wl, seed=1000 * rank + i, M=M).view(
+        Xs.append(Xd0 if i == 0 else torch.from_numpy(synth.activations(wl, seed=replica_seed(rank, i), M=M).view(
             np.int16 if wl.xdtype == "bf16" else np.float16)).view(xdt).to(dev))
         Xqs.append(torch.empty((M, wl.K // 2), dtype=torch.uint8, device=dev))
         sxs.append(torch.empty((M,), dtype=torch.float32, device=dev))
@@ -350,11 +375,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clocks = clk.stop()
-    ms = e0.elapsed_time(e1)
-    if pg is not None:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
     assert hq.hq_last_device_status() == 0
 
     # ---- per-kernel launch durations (graphs of one kernel kind, CUDA events)
@@ -397,17 +418,13 @@ def main():
         b.record()
         torch.cuda.synchronize()
         barrier()
-        e_ms = a.elapsed_time(b)
-        if pg is not None:
-            t = torch.tensor([e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": k2_ops(M, wl.N, wl.K) * r * P * world / (e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        e_ms = max_over_ranks(a.elapsed_time(b), pg, dev)
+        e2e = {"value": job_tops(k2_ops(M, wl.N, wl.K), r * P, world, e_ms), "unit": "TOPS",
                "h2d_bytes_per_step": M * wl.K * 2, "d2h_bytes_per_step": M * wl.N * 2,
                "ms_per_step": e_ms / (r * P)}
 
     ops = k2_ops(M, wl.N, wl.K)
-    value = ops * steps * world / (ms * 1e-3) / 1e12
+    value = job_tops(ops, steps, world, ms)
     # ---- roofline of the dominant kernel
     b1 = k1_bytes(M, wl.K)
     b2 = k2_bytes(M, wl.N, wl.K, wl.gw, wl.r)
