@@ -284,7 +284,7 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
-// 2D tiled TMA load (no multicast) of box {x..x+bx, y..y+by} into smem,
+// 2D tiled TMA load of box {x..x+bx, y..y+by} into this CTA's shared memory,
 // completing `bytes` of transaction on the mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void* tmap, int x, int y, uint32_t bar) {
     asm volatile(
