@@ -53,10 +53,12 @@ _sig("hqo_pack_s4", [_P, _I64, _I64, _P])
 _sig("hqo_unpack_s4", [_P, _I64, _I64, _P])
 _sig("hqo_unpack_u4", [_P, _I64, _I64, _P])
 _sig("hqo_rotate_quant", [_P, _ct.c_int, _I64, _I64, _I32, _P, _P, _P, _P])
+_sig("hqo_rotate_quant8", [_P, _ct.c_int, _I64, _I64, _I32, _P, _P, _P])
 _sig("hqo_w4_pack", [_P, _ct.c_int, _I64, _I64, _I32, _P, _P, _P])
 _sig("hqo_w4_dequant", [_P, _P, _P, _I64, _I64, _I32, _P])
 _sig("hqo_serq_prepare", [_P, _I64, _I64, _P, _P, _P, _I32, _P, _I32, _P, _P, _P])
 _sig("hqo_accum", [_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P], _ct.c_int)
+_sig("hqo_accum8", [_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P], _ct.c_int)
 _sig("hqo_epilogue_f64", [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P])
 _sig("hqo_linear_rows_f64", [_P, _P, _I64, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _P, _I64, _P])
 _sig("hqo_linear_fp64", [_P, _ct.c_int, _I64, _I64, _P, _ct.c_int, _I64, _P])
@@ -172,6 +174,18 @@ def rotate_quant(X, xdtype, g, d=None, return_u=False):
     return (Xq, sx, u) if return_u else (Xq, sx)
 
 
+def rotate_quant8(X, xdtype, g, d=None):
+    """W4A8 activations (DynamicPTQ, Methodology 2): (Xq8 [M, K] int8, sx [M]
+    fp32) -- the same rotation with per-token symmetric 8-bit codes in
+    [-127, 127]."""
+    X = _raw(X, xdtype)
+    M, K = X.shape
+    Xq8 = _np.empty((M, K), _np.int8)
+    sx = _np.empty((M,), _np.float32)
+    _lib.hqo_rotate_quant8(_ptr(X), _DT[xdtype], M, K, g, _ptr(_signs(d, g)), _ptr(Xq8), _ptr(sx))
+    return Xq8, sx
+
+
 def w4_pack(W, wdtype, gw):
     """(Wq, sw, zw): per-channel symmetric (gw = 0; sw [N]) or group asymmetric
     int4 (sw, zw group-major [K/gw, N])."""
@@ -226,6 +240,25 @@ def accum(Xq, K, Wq, zw, gw, Rq=None, sal=None):
     Rqp = None if r == 0 else _c(Rq, _np.uint8)
     ovf = _lib.hqo_accum(_ptr(Xq), M, K, _ptr(Wq), _ptr(zp), N, gw, _ptr(Rqp), _ptr(salp), r,
                          _ptr(acc), _ptr(acc_c))
+    assert ovf == 0, "accumulator exceeds int32"
+    return acc, acc_c
+
+
+def accum8(Xq8, K, Wq, zw, gw, Rq=None, sal=None):
+    """W4A8 integer accumulators from 8-bit activation codes Xq8 [M, K] int8:
+    acc [M, N, G] int64 and acc_c [M, N] int64 (same definitions as accum)."""
+    Xq8 = _c(Xq8, _np.int8)
+    Wq = _c(Wq, _np.uint8)
+    M, N = Xq8.shape[0], Wq.shape[0]
+    G = K // gw if gw else 1
+    r = 0 if sal is None else len(sal)
+    acc = _np.empty((M, N, G), _np.int64)
+    acc_c = _np.zeros((M, N), _np.int64)
+    zp = None if zw is None else _c(zw, _np.float16)
+    salp = None if r == 0 else _c(sal, _np.int32)
+    Rqp = None if r == 0 else _c(Rq, _np.uint8)
+    ovf = _lib.hqo_accum8(_ptr(Xq8), M, K, _ptr(Wq), _ptr(zp), N, gw, _ptr(Rqp), _ptr(salp), r,
+                          _ptr(acc), _ptr(acc_c))
     assert ovf == 0, "accumulator exceeds int32"
     return acc, acc_c
 

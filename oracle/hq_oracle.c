@@ -20,6 +20,9 @@
  *  [WaterSIC] "WaterSIC: information-theoretically (near) optimal linear
  *          layer quantization", Technical summary section 1 (a linear layer
  *          computes Y = W X).
+ *  [DynamicPTQ] "DynamicPTQ", Methodology 2 (8-bit activations on the
+ *          quantisation-sensitive layers, weights and everything else in 4
+ *          bit); SERQ section 4 evaluates the same layer at W4A8.
  *
  * Readings where the pages are silent (each one is listed in the design
  * notes): H = diag(d) * Sylvester(g), d a +-1 vector with d[0] = +1; the
@@ -256,6 +259,48 @@ void hqo_rotate_quant(const void* X, int dtype, int64_t M, int64_t K, int32_t g,
     if (!u_out) free(u);
 }
 
+/* W4A8 activations [DynamicPTQ Methodology 2; SERQ s4]: the same rotation
+ * and per-token symmetric quantiser with 8-bit codes.  Per row m: amax =
+ * max |u|; if amax == 0 the codes are 0 and sx = 0; else
+ * s = fl32(amax / 127), inv = fl32(127 / amax),
+ * q = clamp(rint(fl32(u * inv)), -127, 127), sx = fl32(s * fl32(1/sqrt(g))).
+ * Xq8 is [M][K] int8 (one code per byte); sx is [M]. */
+void hqo_rotate_quant8(const void* X, int dtype, int64_t M, int64_t K, int32_t g,
+                       const int8_t* d, int8_t* Xq8, float* sx)
+{
+    float cg = (float)(1.0 / sqrt((double)g));
+    float* u = (float*)malloc((size_t)(M * K) * sizeof(float));
+    hqo_rotate_rows(X, dtype, M, K, g, d, u);
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const float* row = u + m * K;
+        int8_t* qrow = Xq8 + m * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) amax = fmaxf(amax, fabsf(row[k]));
+        if (amax == 0.0f) {
+            sx[m] = 0.0f;
+            memset(qrow, 0, (size_t)K);
+            continue;
+        }
+        float s = amax / 127.0f;
+        float inv = 127.0f / amax;
+        sx[m] = s * cg;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = row[k] * inv;
+            qrow[k] = (int8_t)(int)clampf(rintf(t), -127.0f, 127.0f);
+        }
+    }
+    free(u);
+}
+
+/* The W4A8 integer GEMM: as hqo_accum with 8-bit activation codes
+ * (Xq8 [M][K] int8): acc[m][n][b] = sum_{k in group b} qx[m][k] *
+ * (qw[n][k] - z[b][n]), acc_c[m][n] = sum_{j<r} qx[m][S_j] * qr[n][j].
+ * Plain triple loop in int64; returns 1 if any value does not fit in int32. */
+int hqo_accum8(const int8_t* Xq8, int64_t M, int64_t K, const uint8_t* Wq, const uint16_t* zw,
+               int64_t N, int32_t gw, const uint8_t* Rq, const int32_t* sal, int32_t r,
+               int64_t* acc, int64_t* acc_c);
+
 /* ------------------------------------------------------------------------ */
 /* Weight quantiser w4_pack.                                                 */
 /* ------------------------------------------------------------------------ */
@@ -400,6 +445,38 @@ int hqo_accum(const uint8_t* Xq, int64_t M, int64_t K, const uint8_t* Wq, const 
             int64_t c = 0;
             for (int32_t j = 0; j < r; ++j)
                 c += (int64_t)get_nibble_s(xrow, sal[j]) * get_nibble_s(Rq + n * ldr, j);
+            if (acc_c) acc_c[m * N + n] = c;
+        }
+    }
+    return overflow;
+}
+
+int hqo_accum8(const int8_t* Xq8, int64_t M, int64_t K, const uint8_t* Wq, const uint16_t* zw,
+               int64_t N, int32_t gw, const uint8_t* Rq, const int32_t* sal, int32_t r,
+               int64_t* acc, int64_t* acc_c)
+{
+    int64_t G = gw ? K / gw : 1;
+    int64_t glen = gw ? gw : K;
+    int64_t ldr = (r + 1) / 2;
+    int overflow = 0;
+    #pragma omp parallel for schedule(static) reduction(|:overflow)
+    for (int64_t m = 0; m < M; ++m) {
+        const int8_t* xrow = Xq8 + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* wrow = Wq + n * (K / 2);
+            for (int64_t b = 0; b < G; ++b) {
+                int64_t s = 0;
+                int z = gw ? (int)hqo_f16_to_f32(zw[b * N + n]) : 0;
+                for (int64_t k = b * glen; k < (b + 1) * glen; ++k) {
+                    int wv = gw ? get_nibble_u(wrow, k) - z : get_nibble_s(wrow, k);
+                    s += (int64_t)xrow[k] * wv;
+                }
+                acc[(m * N + n) * G + b] = s;
+                if (s > INT32_MAX || s < INT32_MIN) overflow = 1;
+            }
+            int64_t c = 0;
+            for (int32_t j = 0; j < r; ++j)
+                c += (int64_t)xrow[sal[j]] * get_nibble_s(Rq + n * ldr, j);
             if (acc_c) acc_c[m * N + n] = c;
         }
     }

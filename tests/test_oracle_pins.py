@@ -402,3 +402,105 @@ def test_quantised_layer_approximates_float_layer(name):
     out0 = O.layer(X, wl.xdtype, W, wl.wdtype, wl.g, d, wl.gw, 0)
     rel0 = np.linalg.norm(out0["y"] - yf) / np.linalg.norm(yf)
     assert rel0 < 0.35
+
+
+# ---------------------------------------------------------------- W4A8 (next row)
+# DynamicPTQ, Methodology 2: 8-bit activations on the sensitive layers, weights
+# in 4 bit; SERQ section 4 evaluates the same layer at W4A8.  Reading: the same
+# rotation and per-token symmetric quantiser with codes in [-127, 127], one
+# code per byte.
+
+@pytest.mark.parametrize("name", ["tiny", "attn", "down"])
+def test_w4a8_activation_quant_round_trip(name):
+    wl = synth.WORKLOADS[name]
+    M = 16 if name == "tiny" else 6
+    X = synth.activations(wl, M=M)
+    d = synth.hadamard_signs(wl.g)
+    _, _, u = O.rotate_quant(X, wl.xdtype, wl.g, d, return_u=True)   # the pinned rotation
+    q8, sx8 = O.rotate_quant8(X, wl.xdtype, wl.g, d)
+    q = q8.astype(np.float64)
+    u = u.astype(np.float64)
+    amax = np.abs(u).max(axis=1)
+    s = amax / 127.0
+    assert np.all(np.abs(q) <= 127)
+    assert np.all(np.abs(u / s[:, None] - q) <= 0.5 + 1e-4)                  # |u - q s| <= s/2
+    idx = np.abs(u).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(M), idx]) == 127)                        # amax element -> +-127
+    assert np.allclose(sx8, s / np.sqrt(wl.g), rtol=2 ** -22)
+    # 8-bit codes resolve the rotated row 127/7 times finer than the 4-bit ones
+    q4 = O.unpack_s4(O.rotate_quant(X, wl.xdtype, wl.g, d)[0], wl.K).astype(np.float64)
+    err8 = np.abs(u - q * s[:, None]).max()
+    err4 = np.abs(u - q4 * (amax / 7.0)[:, None]).max()
+    assert err8 < err4 / 10
+
+
+def test_w4a8_codes_round_ties_to_even():
+    # one channel per group of 8 spreads as a constant over the group; group 1
+    # holds 127, so amax = 127, inv = fl32(127/127) = 1 and the codes are
+    # rint(u): 2.5 -> 2 and 3.5 -> 4 (ties to even)
+    X = np.zeros((2, 16), np.float16)
+    X[0, 0], X[0, 8] = 2.5, 127.0
+    X[1, 0], X[1, 8] = 3.5, 127.0
+    q8, sx8 = O.rotate_quant8(X, "f16", 8, None)
+    assert np.all(q8[0, :8] == 2) and np.all(q8[0, 8:] == 127)
+    assert np.all(q8[1, :8] == 4) and np.all(q8[1, 8:] == 127)
+    assert sx8[0] == np.float32(np.float32(127.0) / np.float32(127.0)) * np.float32(1 / np.sqrt(8))
+
+
+def test_w4a8_zero_row():
+    X = np.zeros((2, 256), np.float16)
+    X[1, 3] = 1.0
+    q8, sx8 = O.rotate_quant8(X, "f16", 128, None)
+    assert sx8[0] == 0 and np.all(q8[0] == 0) and sx8[1] > 0
+
+
+@pytest.mark.parametrize("gw", [0, 64])
+def test_accum8_brute_force_matches_numpy_matmul(gw):
+    rng = np.random.default_rng(16)
+    M, N, K = 5, 7, 256
+    qx = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    if gw:
+        Wq = O.pack_s4(rng.integers(0, 16, (N, K)).astype(np.int8))
+        z = rng.integers(0, 16, (K // gw, N)).astype(np.float16)
+        wv = O.unpack_u4(Wq, K).astype(np.int64) - np.repeat(z.astype(np.int64).T, gw, axis=1)
+    else:
+        qw = rng.integers(-8, 8, (N, K)).astype(np.int8)
+        Wq = O.pack_s4(qw)
+        z = None
+        wv = qw.astype(np.int64)
+    sal = np.array([0, 31, 128, 255], np.int32)
+    qr = rng.integers(-8, 8, (N, 4)).astype(np.int8)
+    acc, acc_c = O.accum8(qx, K, Wq, z, gw, O.pack_s4(qr), sal)
+    G = K // gw if gw else 1
+    L = K // G
+    for b in range(G):
+        assert np.array_equal(acc[:, :, b], qx[:, b * L:(b + 1) * L].astype(np.int64) @ wv[:, b * L:(b + 1) * L].T)
+    assert np.array_equal(acc_c, qx[:, sal].astype(np.int64) @ qr.astype(np.int64).T)
+
+
+def test_accum8_int32_worst_case_fits():
+    # K (at most 65536) * 127 * 15 (an 8-bit code times an asymmetric weight offset) < 2^31
+    assert 65536 * 127 * 15 < 2 ** 31
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_w4a8_layer_against_dequantised_matmul_and_closer_to_float(name):
+    wl = synth.WORKLOADS[name]
+    M, N = (16, 128) if name == "tiny" else (4, 192)
+    wl, X, W, d, Wrot, Wq, sw, zw, sal = _prepared(name, M=M, N=N)
+    Rq, sr = O.serq_prepare(Wrot, Wq, sw, zw, wl.gw, sal)
+    q8, sx8 = O.rotate_quant8(X, wl.xdtype, wl.g, d)
+    acc, acc_c = O.accum8(q8, wl.K, Wq, zw, wl.gw, Rq, sal)
+    y8 = O.epilogue_f64(acc, acc_c, sx8, sw, sr)
+    # independent formulation: dequantise both operands and multiply (numpy)
+    Xhat = q8.astype(np.float64) * sx8.astype(np.float64)[:, None]
+    What = O.w4_dequant(Wq, sw, zw, wl.K, wl.gw).astype(np.float64)
+    Rhat = O.unpack_s4(Rq, wl.r).astype(np.float64) * sr.astype(np.float64)[:, None]
+    ref = Xhat @ What.T + Xhat[:, sal] @ Rhat.T
+    assert np.allclose(y8, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # 8-bit activations lose less than 4-bit ones against the float layer
+    yf = O.linear_fp64(X, wl.xdtype, W, wl.wdtype)
+    y4 = O.layer(X, wl.xdtype, W, wl.wdtype, wl.g, d, wl.gw, wl.r)["y"]
+    rel8 = np.linalg.norm(y8 - yf) / np.linalg.norm(yf)
+    rel4 = np.linalg.norm(y4 - yf) / np.linalg.norm(yf)
+    assert rel8 < rel4, (rel8, rel4)
