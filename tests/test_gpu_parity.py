@@ -93,6 +93,9 @@ ROT_CASES = [
     ("attn", 48, None),
     ("down", 24, None),
     ("large", 12, None),
+    ("attn", 200, None),
+    ("down", 130, None),
+    ("large", 100, None),
 ]
 
 
@@ -157,6 +160,46 @@ def test_rotate_quant_edge_rows_and_strides():
     assert np.all(O.unpack_s4(host(Xq), K)[1, :g] == 7)
     Xq0, sx0 = hq.hq_rotate_quant(big[:0, :K], g, None)       # M == 0
     assert Xq0.shape == (0, K // 2)
+
+
+@pytest.mark.parametrize("K,g,dtype", [(11008, 128, "bf16"), (8192, 256, "bf16"), (4096, 4096, "bf16"),
+                                     (4096, 128, "f16"), (16384, 512, "f16"), (1152, 64, "bf16"), (3072, 1024, "f16")])
+def test_rotate_quant_many_rows_per_team(K, g, dtype):
+    # more rows than row teams on the device: every team of the streaming kernel
+    # walks several rows through its two shared-memory slots; K covers teams of
+    # 1 to 4 warps (and a partly idle last warp for 11008 = 86 x 128 channels)
+    rng = np.random.default_rng(K + g)
+    M = 2500
+    x = rng.standard_t(3, size=(M, K)).astype(np.float32)
+    x[::97, 3] = 400.0
+    x[5] = 0.0
+    X = x.astype(np.float16) if dtype == "f16" else synth.f32_to_bf16_bits(x)
+    d = synth.hadamard_signs(g, seed=K)
+    Xq_o, sx_o = O.rotate_quant(X, dtype, g, d)
+    Xq, sx = hq.hq_rotate_quant(dev(X, dtype), g, torch.from_numpy(d).cuda())
+    assert_same(host(Xq), Xq_o, "codes")
+    assert_same(host(sx), sx_o, "scales")
+    no_device_error()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_rotate_quant_ties_and_strides_on_128_multiples(dtype):
+    # rows of 256 channels (the streaming kernel): exact ties of fl32(u * inv)
+    # and a row stride larger than the row
+    X = np.zeros((6, 256), np.float32)
+    X[0, 0], X[0, 8] = 1.5, 3.0
+    X[1, 0], X[1, 8] = 2.75, 5.5
+    X[2, 0], X[2, 8] = 5.5, 11.0
+    X[3, :] = np.linspace(-3, 3, 256)
+    X[4, 200] = -9.0
+    Xr = X.astype(np.float16) if dtype == "f16" else synth.f32_to_bf16_bits(X)
+    Xq_o, sx_o = O.rotate_quant(Xr, dtype, 8, None)
+    big = torch.zeros((6, 256 + 128), dtype=torch.float16 if dtype == "f16" else torch.bfloat16, device="cuda")
+    big[:, :256] = dev(Xr, dtype)
+    Xq, sx = hq.hq_rotate_quant(big[:, :256], 8, None)
+    assert_same(host(Xq), Xq_o, "codes")
+    assert_same(host(sx), sx_o, "scales")
+    assert np.all(O.unpack_s4(Xq_o, 256)[:3, :8] == 4)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
