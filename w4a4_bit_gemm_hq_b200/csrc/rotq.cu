@@ -78,12 +78,24 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void sts128f(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ float2 lds64f(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+
 // Packed f32x2 arithmetic (sm_100): each lane is an IEEE round-to-nearest-
 // even add (or fma) like __fadd_rn (__fmaf_rn).
 __device__ __forceinline__ float2 rq_add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 rq_sub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
 // a * b + c with one rounding; with b = +-1 this is exactly c + a or c - a
 __device__ __forceinline__ float2 rq_fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// a - b, as fma(b, -1, a): the product is exact, so this is the one rounding
+// of the exact difference (a plain packed add of a negated operand would
+// first negate both lanes with separate instructions)
+__device__ __forceinline__ float2 rq_sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
 
 // max(|a|, |b|, |c|)
 __device__ __forceinline__ float rq_max3abs(float a, float b, float c) {
@@ -220,7 +232,7 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
                         }
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            v[j0 + e].x = __uint_as_float((wv[e] << 16) + mk[2 * e]);
+                            v[j0 + e].x = __uint_as_float(wv[e] * 65536u + mk[2 * e]);   // one integer multiply-add
                             v[j0 + e].y = __uint_as_float((wv[e] & 0xFFFF0000u) ^ mk[2 * e + 1]);
                         }
                     } else {
@@ -241,7 +253,7 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 64; ++j) v[j] = make_float2(0.f, 0.f);
         }
-        if (team_warps == 1) {
+        if (T < 32 && team_warps == 1) {
             // the team is this warp: every lane has read the slot, refill it now
             __syncwarp();
             if (leader && issued < nrows && !flags[team]) issue(issued++);
@@ -267,25 +279,80 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
                 }
             }
         }
-        // ---- stages h >= 128: partner lane (unit) u ^ (h / 128) of the same warp
+        // ---- stages h >= 128
+        // groups of 4096 (one warp each): two transposes through this warp's part
+        // of the row slot (8 KB, free once read) leave lane l with channels
+        // 128 a + 4 l + {0..3} of the group for a = 0..31; the five remaining
+        // stages pair a with a ^ (h / 128) in registers.  wq[p][a] holds
+        // channels 128 a + 4 l + 2 p + {0, 1}.
+        float2 wq[T == 32 ? 2 : 1][T == 32 ? 32 : 1];
+        if constexpr (T == 32) {
+            const uint32_t slot = ring + s * L.slot;
+            const uint32_t p0 = slot + static_cast<uint32_t>(wt * 32) * 128u;          // half-0 lines of the warp's units
+            const uint32_t p1 = slot + static_cast<uint32_t>(NU + wt * 32) * 128u;     // half-1 lines
 #pragma unroll
-        for (int sft = 1; sft < T; sft <<= 1) {
-            const float sg = (lane & sft) ? -1.0f : 1.0f;
-            const float2 sg2 = make_float2(sg, sg);
+            for (int ph = 0; ph < 2; ++ph) {
+                // lane l writes row l (256 bytes): channels 4 k + 2 ph + {0, 1}, k = 0..31,
+                // 16-byte chunk q stored at q ^ (l & 7)
+                const uint32_t rw = lane < 16 ? p0 + 256u * lane : p1 + 256u * (lane - 16);
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                float2 p;
-                p.x = __shfl_xor_sync(0xFFFFFFFFu, v[j].x, sft);
-                p.y = __shfl_xor_sync(0xFFFFFFFFu, v[j].y, sft);
-                // lower lane: own + partner = a + b; upper lane: partner - own = a - b
-                v[j] = rq_fma2(v[j], sg2, p);
+                for (int q = 0; q < 16; ++q) {
+                    const float2 a = v[4 * q + ph], bb = v[4 * q + 2 + ph];
+                    sts128f(rw + ((static_cast<uint32_t>(q) ^ (lane & 7u)) << 4), a.x, a.y, bb.x, bb.y);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int a = 0; a < 32; ++a) {
+                    const uint32_t ra = a < 16 ? p0 + 256u * a : p1 + 256u * (a - 16);
+                    wq[ph][a] = lds64f(ra + (((static_cast<uint32_t>(lane) >> 1) ^ (a & 7u)) << 4) + (lane & 1u) * 8u);
+                }
+                __syncwarp();
+            }
+            // the slot has been read and rewritten by this warp's generic stores:
+            // order them before the next row's copy into it
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (team_warps == 1 && leader && issued < nrows && !flags[team]) issue(issued++);
+#pragma unroll
+            for (int sb = 1; sb < 32; sb <<= 1) {
+#pragma unroll
+                for (int ph = 0; ph < 2; ++ph)
+#pragma unroll
+                    for (int a = 0; a < 32; ++a)
+                        if ((a & sb) == 0) {
+                            const float2 x0 = wq[ph][a], x1 = wq[ph][a + sb];
+                            wq[ph][a] = rq_add2(x0, x1);
+                            wq[ph][a + sb] = rq_sub2(x0, x1);
+                        }
+            }
+        } else {
+            // partner lane (unit) u ^ (h / 128) of the same warp
+#pragma unroll
+            for (int sft = 1; sft < T; sft <<= 1) {
+                const float sg = (lane & sft) ? -1.0f : 1.0f;
+                const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    float2 p;
+                    p.x = __shfl_xor_sync(0xFFFFFFFFu, v[j].x, sft);
+                    p.y = __shfl_xor_sync(0xFFFFFFFFu, v[j].y, sft);
+                    // lower lane: own + partner = a + b; upper lane: partner - own = a - b
+                    v[j] = rq_fma2(v[j], sg2, p);
+                }
             }
         }
 
         // ---- row absmax
         float am[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (T == 32) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) am[j & 3] = rq_max3abs(am[j & 3], v[j].x, v[j].y);
+            for (int ph = 0; ph < 2; ++ph)
+#pragma unroll
+                for (int a = 0; a < 32; ++a) am[a & 3] = rq_max3abs(am[a & 3], wq[ph][a].x, wq[ph][a].y);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) am[j & 3] = rq_max3abs(am[j & 3], v[j].x, v[j].y);
+        }
         float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -304,30 +371,47 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
         }
         if (abort_now) break;
 
-        // ---- scale, round half to even, pack, store (16 bytes at a time)
-        if (act) {
-            uint4* dst = reinterpret_cast<uint4*>(Xq + static_cast<int64_t>(m) * (K / 2) + 64 * u);
-            const float inv = amax == 0.f ? 0.f : __fdiv_rn(7.0f, amax);   // amax == 0: every code is 0
+        // ---- scale, round half to even, pack, store
+        const float inv = amax == 0.f ? 0.f : __fdiv_rn(7.0f, amax);   // amax == 0: every code is 0
+        if constexpr (T == 32) {
+            // lane l: 2 bytes (channels 128 a + 4 l .. + 3) per a, 64 contiguous bytes per warp store
+            if (act) {
+                uint16_t* dst = reinterpret_cast<uint16_t*>(Xq + static_cast<int64_t>(m) * (K / 2) + 2048 * wt) + lane;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t words[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    uint32_t P[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        // scalar __fmul_rn: the product is rounded before the rounding
-                        // add (a packed f32x2 multiply here was contracted with the
-                        // add into one fused operation, which rounds exact ties the
-                        // other way)
-                        const float2 x = v[16 * q + 4 * w + e];
-                        const float2 r = rq_add2(make_float2(__fmul_rn(x.x, inv), __fmul_rn(x.y, inv)), mg);
-                        P[e] = (__float_as_uint(r.y) << 4) + __float_as_uint(r.x);   // byte e of the word (low 16 bits)
-                    }
-                    const uint32_t q01 = (P[1] << 8) + P[0], q23 = (P[3] << 8) + P[2];
-                    words[w] = __byte_perm(q01, q23, 0x5410) ^ 0x88888888u;
+                for (int a = 0; a < 32; ++a) {
+                    const float2 x0 = wq[0][a], x1 = wq[1][a];
+                    const float2 r0 = rq_add2(make_float2(__fmul_rn(x0.x, inv), __fmul_rn(x0.y, inv)), mg);
+                    const float2 r1 = rq_add2(make_float2(__fmul_rn(x1.x, inv), __fmul_rn(x1.y, inv)), mg);
+                    const uint32_t b0 = (__float_as_uint(r0.y) << 4) + __float_as_uint(r0.x);
+                    const uint32_t b1 = (__float_as_uint(r1.y) << 4) + __float_as_uint(r1.x);
+                    dst[32 * a] = static_cast<uint16_t>(((b1 << 8) + b0) ^ 0x8888u);
                 }
-                dst[q] = make_uint4(words[0], words[1], words[2], words[3]);
+            }
+        } else {
+            // 64 bytes per thread, 16 at a time
+            if (act) {
+                uint4* dst = reinterpret_cast<uint4*>(Xq + static_cast<int64_t>(m) * (K / 2) + 64 * u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t words[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t P[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            // scalar __fmul_rn: the product is rounded before the rounding
+                            // add (a packed f32x2 multiply here was contracted with the
+                            // add into one fused operation, which rounds exact ties the
+                            // other way)
+                            const float2 x = v[16 * q + 4 * w + e];
+                            const float2 r = rq_add2(make_float2(__fmul_rn(x.x, inv), __fmul_rn(x.y, inv)), mg);
+                            P[e] = (__float_as_uint(r.y) << 4) + __float_as_uint(r.x);   // byte e (low 16 bits)
+                        }
+                        const uint32_t q01 = (P[1] << 8) + P[0], q23 = (P[3] << 8) + P[2];
+                        words[w] = __byte_perm(q01, q23, 0x5410) ^ 0x88888888u;
+                    }
+                    dst[q] = make_uint4(words[0], words[1], words[2], words[3]);
+                }
             }
         }
         if (leader) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
