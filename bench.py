@@ -6,18 +6,24 @@ grouped Hadamard rotation + per-token int4 quantisation) followed by
 w4a4_linear (K2: int4 x int4 GEMM with the fused SERQ term and dequantising
 epilogue).  Weights are prepared once, offline, by the library's own kernels.
 
-Default workload: the decode-shaped Llama-7B MLP up-projection, 16 tokens,
-K = 4096, N = 11008, group-128 asymmetric int4 weights, Hadamard group 128,
-rank-16 SERQ term, fp16 in/out.  Other workloads: --workload attn|down|large|tiny.
+The JSON line's headline (value, ms_per_step, roofline, e2e, cpu_baseline) is
+the Llama-7B MLP down-projection: 4096 tokens, K = 11008 (86 Hadamard groups
+of 128), N = 4096, group-128 asymmetric int4 weights, rank-32 SERQ term, bf16
+in/out.  The same run also measures every other layer shape of the suite and
+reports them under "workloads": decode (M = 1, 4, 16; 4096 -> 11008), the
+attention projection (M = 2048; 4096 -> 4096, one Hadamard group of 4096) and
+the Llama-70B MLP shape (M = 512, 2048, 8192; 8192 -> 28672), each with K1's
+HBM throughput and fraction of the HBM roofline and K2's TOP/s and fraction of
+the dense int8 tensor peak (of HBM for decode).  "serq_overhead" compares K2
+with and without the SERQ term on the same weights.
 
-Timing: the P steps of one pass over a rotating pool of layers (distinct
-weights and activations, more bytes than the 126 MB L2) are captured in a CUDA
-graph; the timed region replays it, bracketed by a barrier and a device
-synchronise, with CUDA events; the value is the max over ranks.  Per-kernel
-launch durations (for the roofline) come from graphs holding one kernel kind,
-timed with CUDA events on the launch stream.  SM clocks are sampled with
-nvidia-smi during the timed region.  With --gpus N (torchrun) every rank runs
-an independent replica (weak scaling; the layer has no exchange step).
+Timing: every layer shape runs over a rotating pool of layers and batches
+(distinct weights and activations) holding more bytes than 2x the 126 MB L2;
+steps are captured in CUDA graphs and timed with CUDA events on the launching
+stream; per-kernel launch durations come from graphs holding one kernel kind.
+SM clocks are sampled with nvidia-smi during the headline's timed region.
+With --gpus N (torchrun) every rank runs an independent replica (weak scaling;
+the layer has no exchange step), durations are the max over ranks.
 
 Prints ONE JSON line on rank 0.
 """
@@ -35,9 +41,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
-
-DEFAULT_STEPS = {"tiny": 20000, "decode": 100000, "attn": 20000, "down": 4000, "large": 400}
-DEFAULT_M = {"tiny": 16, "decode": 16, "attn": 2048, "down": 4096, "large": 8192}
+HEADLINE = ("down", 4096)
+# (workload, M) of the suite; the large Llama-70B shape is measured at three M
+SUITE = [("decode", 1), ("decode", 4), ("decode", 16), ("attn", 2048), ("down", 4096), ("large", 512),
+         ("large", 2048), ("large", 8192)]
+# shapes where K1 and the prefill GEMM have roofline targets (M >= 2048)
+TARGET_SHAPES = [("attn", 2048), ("down", 4096), ("large", 8192)]
+K1_TARGET, K2_TARGET = 0.70, 0.60
+DEFAULT_STEPS = 500
+NOMINAL_INT8_PER_BF16 = 2.0   # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PF nominal)
 
 
 def measured_peaks():
@@ -50,13 +62,17 @@ def measured_peaks():
 
 
 def parse():
+    from w4a4_bit_gemm_hq_b200 import synth
+
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(DEFAULT_M), default="decode")
-    ap.add_argument("--m", type=int, default=None, help="tokens per step (default: the workload's)")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=HEADLINE[0],
+                    help="headline workload (default: the down-projection)")
+    ap.add_argument("--m", type=int, default=None, help="tokens per step of the headline (default: the workload's)")
+    ap.add_argument("--headline-only", action="store_true", help="skip the other shapes (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -64,10 +80,12 @@ def parse():
 
 # ----------------------------------------------------------------- algorithmic work per launch
 def k1_bytes(M, K, xbytes=2):
+    """Read X (16-bit), write packed codes (0.5 B / element) and sx (4 B / row)."""
     return M * K * xbytes + M * K // 2 + 4 * M
 
 
 def k2_bytes(M, N, K, gw, r, ybytes=2):
+    """Every operand of w4a4_linear read once and Y written once."""
     b = N * K // 2                                  # packed weights
     b += (2 * (K // gw) * N * 2) if gw else 2 * N   # scales (+ zero points)
     b += N * r // 2 + 2 * N + 4 * r                 # Rq, sr, sal
@@ -77,6 +95,7 @@ def k2_bytes(M, N, K, gw, r, ybytes=2):
 
 
 def k2_ops(M, N, K):
+    """Main-term integer ops (the SERQ term's 2 M N r are not counted)."""
     return 2 * M * N * K
 
 
@@ -138,17 +157,16 @@ def oracle_step_sample(wl, M, seed, n_rows, n_cols, sample_seed=0):
     from w4a4_bit_gemm_hq_b200 import synth
 
     rng = np.random.default_rng(sample_seed)
-    X = synth.activations(wl, seed=seed, M=M)
-    W = synth.weights(wl, seed=seed)
-    d = synth.hadamard_signs(wl.g, seed=seed)
     rows = np.sort(rng.choice(M, size=min(n_rows, M), replace=False))
+    X = synth.activations(wl, seed=seed, M=M)[rows]
     cols = np.sort(rng.choice(wl.N, size=min(n_cols, wl.N), replace=False))
-    Wc = W[cols]
+    Wc = synth.weights(wl, seed=seed)[cols]
+    d = synth.hadamard_signs(wl.g, seed=seed)
     Wrot = O.rotate_normalised(Wc, wl.wdtype, wl.g, d)
     Wq, sw, zw = O.w4_pack(Wrot, "f32", wl.gw)
-    _, sal = O.salient_channels(X[rows], wl.xdtype, wl.g, d, wl.r)
+    _, sal = O.salient_channels(X, wl.xdtype, wl.g, d, wl.r)
     Rq, sr = O.serq_prepare(Wrot, Wq, sw, zw, wl.gw, sal)
-    Xs = np.ascontiguousarray(X[rows])
+    Xs = np.ascontiguousarray(X)
 
     def step():
         Xq, sx = O.rotate_quant(Xs, wl.xdtype, wl.g, d)
@@ -220,13 +238,16 @@ def metric_name():
     return "W4A4 linear TOPS & rotate/quant GB/s at Llama-7B shapes, % of B200 roofline"
 
 
+def describe(wl, M):
+    return "%s: W4A4 linear M=%d K=%d N=%d (Hadamard group %d, weight group %s, SERQ rank %d, %s in/out)" % (
+        wl.name, M, wl.K, wl.N, wl.g, wl.gw if wl.gw else "per-channel", wl.r, wl.xdtype)
+
+
 def config_dict(wl, M, pool, n):
-    c = {"workload": "%s: W4A4 linear M=%d K=%d N=%d (Hadamard group %d, weight group %s, SERQ rank %d, %s in/out)"
-                     % (wl.name, M, wl.K, wl.N, wl.g, wl.gw if wl.gw else "per-channel", wl.r, wl.xdtype),
-         "M": M, "K": wl.K, "N": wl.N, "hadamard_group": wl.g, "weight_group": wl.gw, "serq_rank": wl.r,
-         "parallelism": "replicas x%d" % n}
+    c = {"workload": describe(wl, M), "M": M, "K": wl.K, "N": wl.N, "hadamard_group": wl.g,
+         "weight_group": wl.gw, "serq_rank": wl.r, "parallelism": "replicas x%d" % n}
     if pool is not None:
-        c["l2"] = "rotating pool of %d layers and batches (%.0f MB > 126 MB L2)" % pool
+        c["l2"] = "rotating pool of %d layers and batches (%.0f MB > 2 x 126 MB L2)" % pool
     return c
 
 
@@ -255,25 +276,177 @@ def replica_seed(rank, i):
     return 1000 * rank + i
 
 
+# ----------------------------------------------------------------- GPU measurement
+class Runner:
+    """Device, peaks and helpers shared by every measured shape."""
+
+    def __init__(self, torch, hq, synth, rank, dev):
+        self.torch, self.hq, self.synth, self.rank, self.dev = torch, hq, synth, rank, dev
+        self.peaks = measured_peaks()
+        self.int8_peak = NOMINAL_INT8_PER_BF16 * self.peaks["bf16"]
+        self.int8_peak_sus = NOMINAL_INT8_PER_BF16 * self.peaks["bf16_sus"] if self.peaks["bf16_sus"] else None
+
+    def to_dev(self, a, dt):
+        import numpy as np
+
+        if dt == "bf16":
+            return self.torch.from_numpy(a.view(np.int16)).to(self.dev).view(self.torch.bfloat16)
+        return self.torch.from_numpy(a).to(self.dev)
+
+    def capture(self, fns):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for fn in fns:
+                fn()
+        torch.cuda.current_stream().wait_stream(s)
+        with torch.cuda.graph(g):
+            for fn in fns:
+                fn()
+        return g
+
+    def time_graph(self, g, reps):
+        torch = self.torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    def launch_ms(self, fn, P, budget_ms=25.0):
+        """Average duration of one launch of fn(i), from a graph of P launches
+        (one per pool entry) replayed until about budget_ms have passed."""
+        g = self.capture([lambda i=i: fn(i) for i in range(P)])
+        g.replay()
+        est = max(self.time_graph(g, 1), 1e-3)
+        reps = int(max(2, min(2000, budget_ms / est)))
+        ms = self.time_graph(g, reps) / (reps * P)
+        del g
+        return ms
+
+
+class Shape:
+    """One prepared layer shape: a pool of P layers (distinct weights) and P
+    token batches (distinct activations), all resident on the device."""
+
+    def __init__(self, R, wl, M, base=None, r=None):
+        torch, hq, synth = R.torch, R.hq, R.synth
+        self.R, self.wl, self.M = R, wl, M
+        self.r = wl.r if r is None else r
+        self.xdt = torch.float16 if wl.xdtype == "f16" else torch.bfloat16
+        X0 = R.to_dev(synth.activations(wl, seed=replica_seed(R.rank, 0), M=M), wl.xdtype)
+        if base is None:
+            W = R.to_dev(synth.weights(wl, seed=R.rank), wl.wdtype)
+            d = torch.from_numpy(synth.hadamard_signs(wl.g, seed=R.rank)).to(R.dev)
+            base = hq.W4A4Linear.prepare(W, wl.g, wl.gw, self.r, d, X_calib=X0, out_dtype=self.xdt)
+            del W
+        self.base = base
+        per_step = k1_bytes(M, wl.K) + k2_bytes(M, wl.N, wl.K, wl.gw, self.r) + M * wl.K * 2
+        self.per_step = per_step
+        self.P = int(min(16, max(1, math.ceil(2.2 * L2_BYTES / per_step))))
+        clone = lambda t: None if t is None else t.clone()
+        b = base
+        self.layers = [b] + [hq.W4A4Linear(b.group, b.gw, b.H_signs, clone(b.Wq), clone(b.sw), clone(b.zw),
+                                           clone(b.Rq), clone(b.sr), b.sal_idx, wl.K, wl.N, self.xdt)
+                             for _ in range(self.P - 1)]
+        # distinct batches: the seeded batch and row rotations of it (different
+        # bytes at different addresses; the values' statistics are unchanged)
+        self.X = [X0] + [X0.roll(i, 0).contiguous() for i in range(1, self.P)]
+        self.Xq = [torch.empty((M, wl.K // 2), dtype=torch.uint8, device=R.dev) for _ in range(self.P)]
+        self.sx = [torch.empty((M,), dtype=torch.float32, device=R.dev) for _ in range(self.P)]
+        self.Y = [torch.empty((M, wl.N), dtype=self.xdt, device=R.dev) for _ in range(self.P)]
+        self.ws = [L.workspace(M, R.dev) for L in self.layers]
+
+    def k1(self, i):
+        self.R.hq.hq_rotate_quant(self.X[i], self.wl.g, self.layers[i].H_signs, self.Xq[i], self.sx[i])
+
+    def k2(self, i):
+        L = self.layers[i]
+        self.R.hq.w4a4_linear(self.Xq[i], self.sx[i], L.Wq, L.sw, L.zw, L.gw, L.Rq, L.sr, L.sal_idx, self.xdt,
+                              self.Y[i], self.ws[i])
+
+    def step(self, i):
+        self.k1(i)
+        self.k2(i)
+
+    def record(self, decode_like):
+        """K1, K2 and whole-step measurements of this shape."""
+        R, wl, M, P = self.R, self.wl, self.M, self.P
+        for i in range(P):
+            self.step(i)
+        R.torch.cuda.synchronize()
+        assert R.hq.hq_last_device_status() == 0
+        t1 = R.launch_ms(self.k1, P)
+        t2 = R.launch_ms(self.k2, P)
+        ts = R.launch_ms(self.step, P)
+        b1, b2, ops = k1_bytes(M, wl.K), k2_bytes(M, wl.N, wl.K, wl.gw, self.r), k2_ops(M, wl.N, wl.K)
+        rec = {"workload": wl.name, "M": M, "K": wl.K, "N": wl.N, "hadamard_group": wl.g, "weight_group": wl.gw,
+               "serq_rank": self.r, "pool": P,
+               "k1_us": t1 * 1e3, "k1_bytes": b1, "k1_GBs": b1 / (t1 * 1e-3) / 1e9,
+               "k1_frac_hbm": b1 / (t1 * 1e-3) / 1e9 / R.peaks["hbm"],
+               "k2_us": t2 * 1e3, "k2_ops": ops, "k2_bytes": b2, "k2_TOPs": ops / (t2 * 1e-3) / 1e12,
+               "k2_GBs": b2 / (t2 * 1e-3) / 1e9,
+               "step_us": ts * 1e3, "step_TOPS": ops / (ts * 1e-3) / 1e12}
+        if decode_like:
+            rec["k2_bound"] = "hbm"
+            rec["k2_frac_hbm"] = rec["k2_GBs"] / R.peaks["hbm"]
+        else:
+            rec["k2_bound"] = "tensor (int8)"
+            rec["k2_frac_int8"] = rec["k2_TOPs"] / R.int8_peak
+        return rec
+
+    def free(self):
+        for name in ("layers", "X", "Xq", "sx", "Y", "ws", "base"):
+            setattr(self, name, None)
+
+
+def int8_gemm_crosscheck(R):
+    """cuBLASLt int8 GEMM (torch._int_mm) at 8192^3, best of 10: a cross-check
+    of the int8 denominator, which is 2 x the measured bf16 burst peak."""
+    torch = R.torch
+    try:
+        n = 8192
+        A = torch.randint(-8, 8, (n, n), dtype=torch.int8, device=R.dev)
+        B = torch.randint(-8, 8, (n, n), dtype=torch.int8, device=R.dev)
+        for _ in range(3):
+            torch._int_mm(A, B.t())
+        ts = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            torch._int_mm(A, B.t())
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        del A, B
+        return 2 * n ** 3 / min(ts) / 1e9
+    except Exception as e:  # noqa: BLE001 (report, never fail the bench on the cross-check)
+        return "unavailable: %s" % type(e).__name__
+
+
 # ----------------------------------------------------------------- main
 def main():
     args = parse()
-    wl0 = None
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     from w4a4_bit_gemm_hq_b200 import synth
 
-    wl0 = synth.WORKLOADS[args.workload]
-    M = args.m if args.m is not None else DEFAULT_M[args.workload]
-    wl = wl0.with_m(M)
+    head_name = args.workload
+    head_M = args.m if args.m is not None else (HEADLINE[1] if head_name == HEADLINE[0]
+                                                  else synth.WORKLOADS[head_name].M)
+    wl_head = synth.WORKLOADS[head_name].with_m(head_M)
 
     if args.impl == "reference":
-        run_reference(args, wl, M, rank, world)
+        run_reference(args, wl_head, head_M, rank, world)
         return
 
-    import numpy as np
     import torch
 
     torch.cuda.set_device(local)
@@ -288,80 +461,24 @@ def main():
     from w4a4_bit_gemm_hq_b200 import hq
 
     dev = torch.device("cuda", local)
-    steps = args.steps if args.steps is not None else DEFAULT_STEPS[args.workload]
+    R = Runner(torch, hq, synth, rank, dev)
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS
     warm = max(args.warmup, 3)
-    peaks = measured_peaks()
-    xdt = torch.float16 if wl.xdtype == "f16" else torch.bfloat16
 
-    def to_dev(a, dt):
-        if dt == "bf16":
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(a).to(dev)
-
-    # ---- one prepared layer, then a pool of distinct copies
-    X0 = synth.activations(wl, seed=replica_seed(rank, 0), M=M)
-    W0 = synth.weights(wl, seed=rank)
-    d = torch.from_numpy(synth.hadamard_signs(wl.g, seed=rank)).to(dev)
-    Xd0 = to_dev(X0, wl.xdtype)
-    base = hq.W4A4Linear.prepare(to_dev(W0, wl.wdtype), wl.g, wl.gw, wl.r, d, X_calib=Xd0, out_dtype=xdt)
-    del W0
-    per_step = k1_bytes(M, wl.K) + k2_bytes(M, wl.N, wl.K, wl.gw, wl.r) + M * wl.K * 2
-    P = int(min(16, max(1, math.ceil(2 * L2_BYTES / per_step))))
-    layers, Xs, Xqs, sxs, Ys = [], [], [], [], []
-    for i in range(P):
-        clone = lambda t: None if t is None else t.clone()
-        layers.append(hq.W4A4Linear(base.group, base.gw, base.H_signs, clone(base.Wq), clone(base.sw),
-                                    clone(base.zw), clone(base.Rq), clone(base.sr), base.sal_idx, wl.K, wl.N, xdt))
-        Xs.append(Xd0 if i == 0 else torch.from_numpy(synth.activations(wl, seed=replica_seed(rank, i), M=M).view(
-            np.int16 if wl.xdtype == "bf16" else np.float16)).view(xdt).to(dev))
-        Xqs.append(torch.empty((M, wl.K // 2), dtype=torch.uint8, device=dev))
-        sxs.append(torch.empty((M,), dtype=torch.float32, device=dev))
-        Ys.append(torch.empty((M, wl.N), dtype=xdt, device=dev))
-    pool_mb = P * per_step / 1e6
-
-    def k1(i):
-        hq.hq_rotate_quant(Xs[i], wl.g, layers[i].H_signs, Xqs[i], sxs[i])
-
-    def k2(i):
-        L = layers[i]
-        hq.w4a4_linear(Xqs[i], sxs[i], L.Wq, L.sw, L.zw, L.gw, L.Rq, L.sr, L.sal_idx, xdt, Ys[i],
-                       L.workspace(M, dev))
-
-    def step(i):
-        k1(i)
-        k2(i)
-
-    # ---- warm-up (eager), then graphs
+    # ---- the headline shape: timed region of exactly `steps` steps
+    S = Shape(R, wl_head, head_M)
+    P = S.P
     for w in range(warm):
-        step(w % P)
+        S.step(w % P)
     torch.cuda.synchronize()
     assert hq.hq_last_device_status() == 0
-
-    def capture(fn_list):
-        g = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            for fn in fn_list:
-                fn()
-        torch.cuda.current_stream().wait_stream(s)
-        with torch.cuda.graph(g):
-            for fn in fn_list:
-                fn()
-        return g
-
-    g_full = capture([lambda i=i: step(i) for i in range(P)])
+    g_full = R.capture([lambda i=i: S.step(i) for i in range(P)])
     rem = steps % P
-    g_rem = capture([lambda i=i: step(i) for i in range(rem)]) if rem else None
+    g_rem = R.capture([lambda i=i: S.step(i) for i in range(rem)]) if rem else None
     reps = steps // P
-
-    def barrier():
-        if pg is not None:
-            pg.barrier()
-
-    # ---- timed region
     torch.cuda.synchronize()
-    barrier()
+    if pg is not None:
+        pg.barrier()
     clk = ClockSampler(local)
     clk.start()
     time.sleep(0.3)
@@ -373,99 +490,129 @@ def main():
         g_rem.replay()
     e1.record()
     torch.cuda.synchronize()
-    barrier()
+    if pg is not None:
+        pg.barrier()
     clocks = clk.stop()
     ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
     assert hq.hq_last_device_status() == 0
-
-    # ---- per-kernel launch durations (graphs of one kernel kind, CUDA events)
-    def kernel_ms(fn):
-        g = capture([lambda i=i: fn(i) for i in range(P)])
-        r = max(1, min(reps, 2000))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        a.record()
-        for _ in range(r):
-            g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / (r * P)
-
-    t_k1 = kernel_ms(k1)
-    t_k2 = kernel_ms(k2)
+    del g_full, g_rem
+    decode_like = head_M <= 64
+    head = S.record(decode_like)
 
     # ---- end to end through the public call, host buffers, copies inside
     e2e = None
     if not args.no_e2e:
-        Xh = [torch.empty((M, wl.K), dtype=xdt, pin_memory=True) for _ in range(P)]
-        Yh = [torch.empty((M, wl.N), dtype=xdt, pin_memory=True) for _ in range(P)]
+        M, K, N = head_M, wl_head.K, wl_head.N
+        Xh = [torch.empty((M, K), dtype=S.xdt, pin_memory=True) for _ in range(P)]
+        Yh = [torch.empty((M, N), dtype=S.xdt, pin_memory=True) for _ in range(P)]
         for i in range(P):
-            Xh[i].copy_(Xs[i].cpu())
+            Xh[i].copy_(S.X[i].cpu())
 
         def e2e_step(i):
-            Xs[i].copy_(Xh[i], non_blocking=True)
-            layers[i](Xs[i], Ys[i], Xqs[i], sxs[i])
-            Yh[i].copy_(Ys[i], non_blocking=True)
+            S.X[i].copy_(Xh[i], non_blocking=True)
+            S.layers[i](S.X[i], S.Y[i], S.Xq[i], S.sx[i])
+            Yh[i].copy_(S.Y[i], non_blocking=True)
 
-        g_e2e = capture([lambda i=i: e2e_step(i) for i in range(P)])
-        r = max(1, min(reps, 20000))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        barrier()
-        a.record()
-        for _ in range(r):
-            g_e2e.replay()
-        b.record()
-        torch.cuda.synchronize()
-        barrier()
-        e_ms = max_over_ranks(a.elapsed_time(b), pg, dev)
-        e2e = {"value": job_tops(k2_ops(M, wl.N, wl.K), r * P, world, e_ms), "unit": "TOPS",
-               "h2d_bytes_per_step": M * wl.K * 2, "d2h_bytes_per_step": M * wl.N * 2,
-               "ms_per_step": e_ms / (r * P)}
+        g_e2e = R.capture([lambda i=i: e2e_step(i) for i in range(P)])
+        g_e2e.replay()
+        est = max(R.time_graph(g_e2e, 1), 1e-3)
+        r = int(max(2, min(20000, 400.0 / est)))
+        if pg is not None:
+            pg.barrier()
+        e_ms = max_over_ranks(R.time_graph(g_e2e, r), pg, dev)
+        e2e = {"value": job_tops(k2_ops(M, N, K), r * P, world, e_ms), "unit": "TOPS",
+               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e_ms / (r * P)}
+        del g_e2e, Xh, Yh
+    S.free()
+    del S
+    torch.cuda.empty_cache()
 
-    ops = k2_ops(M, wl.N, wl.K)
-    value = job_tops(ops, steps, world, ms)
-    # ---- roofline of the dominant kernel
-    b1 = k1_bytes(M, wl.K)
-    b2 = k2_bytes(M, wl.N, wl.K, wl.gw, wl.r)
-    k1_gbs = b1 / (t_k1 * 1e-3) / 1e9
-    int8_peak = 2.0 * peaks["bf16"]          # dense int8 = 2 x dense bf16 (nominal 4.5 vs 2.25 PF)
-    decode_like = M <= 64
-    if t_k2 >= t_k1:
+    # ---- every other shape of the suite
+    workloads = [head]
+    serq = []
+    if not args.headline_only:
+        base, prev = None, None
+        for name, M in SUITE:
+            if (name, M) == (head_name, head_M):
+                continue
+            if name != prev:   # the M values of one workload share one prepared layer
+                base, prev = None, name
+                torch.cuda.empty_cache()
+            wl = synth.WORKLOADS[name].with_m(M)
+            Sh = Shape(R, wl, M, base=base)
+            base = Sh.base
+            workloads.append(Sh.record(M <= 64))
+            Sh.free()
+            del Sh
+        base = None
+        torch.cuda.empty_cache()
+        # SERQ term's cost in K2: the same weights without the term (r = 0)
+        for name, M in [("attn", 2048), ("down", 4096), ("large", 8192)]:
+            wl = synth.WORKLOADS[name].with_m(M)
+            with_r = next(w for w in workloads if w["workload"] == name and w["M"] == M)
+            S0 = Shape(R, wl, M, r=0)
+            t0 = R.launch_ms(S0.k2, S0.P)
+            serq.append({"workload": name, "M": M, "serq_rank": wl.r, "k2_us_with_term": with_r["k2_us"],
+                         "k2_us_without_term": t0 * 1e3,
+                         "overhead_pct": 100.0 * (with_r["k2_us"] / (t0 * 1e3) - 1.0)})
+            S0.free()
+            del S0
+            torch.cuda.empty_cache()
+        workloads.sort(key=lambda w: [n for n, _ in SUITE].index(w["workload"]) * 100000 + w["M"])
+
+    targets = {}
+    for name, M in TARGET_SHAPES:
+        w = next((w for w in workloads if w["workload"] == name and w["M"] == M), None)
+        if w is not None:
+            targets["%s M=%d" % (name, M)] = {
+                "k1_frac_hbm": w["k1_frac_hbm"], "k1_target": K1_TARGET, "k1_met": w["k1_frac_hbm"] >= K1_TARGET,
+                "k2_frac_int8": w["k2_frac_int8"], "k2_target": K2_TARGET,
+                "k2_met": w["k2_frac_int8"] >= K2_TARGET}
+
+    # ---- roofline of the headline's dominant kernel
+    if head["k2_us"] >= head["k1_us"]:
         if decode_like:
-            roof = {"kernel": "k_gemm_small (w4a4_linear)", "bound": "hbm", "achieved": b2 / (t_k2 * 1e-3) / 1e9,
-                    "peak": peaks["hbm"], "unit": "GB/s", "bytes_per_launch": b2}
+            roof = {"kernel": "k_gemm_small (w4a4_linear)", "bound": "hbm", "achieved": head["k2_GBs"],
+                    "peak": R.peaks["hbm"], "unit": "GB/s", "bytes_per_launch": head["k2_bytes"]}
         else:
-            roof = {"kernel": "k_gemm_pf (w4a4_linear)", "bound": "tensor",
-                    "achieved": ops / (t_k2 * 1e-3) / 1e12, "peak": int8_peak, "unit": "TOP/s",
-                    "ops_per_launch": ops}
+            roof = {"kernel": "k_gemm_pf (w4a4_linear)", "bound": "tensor", "achieved": head["k2_TOPs"],
+                    "peak": R.int8_peak, "unit": "TOP/s", "ops_per_launch": head["k2_ops"]}
     else:
-        roof = {"kernel": "k_rotate (hq_rotate_quant)", "bound": "hbm", "achieved": k1_gbs, "peak": peaks["hbm"],
-                "unit": "GB/s", "bytes_per_launch": b1}
+        roof = {"kernel": "k_rotq (hq_rotate_quant)", "bound": "hbm", "achieved": head["k1_GBs"],
+                "peak": R.peaks["hbm"], "unit": "GB/s", "bytes_per_launch": head["k1_bytes"]}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["peak_source"] = peaks["src"] + (" (int8 = 2 x measured bf16 burst)" if roof["bound"] == "tensor" else
-                                          " HBM copy, burst")
-    roof["traffic"] = committed_traffic(args.workload, M, roof["kernel"])
+    roof["peak_source"] = (R.peaks["src"] + (" bf16 burst x %.0f (nominal dense int8 / bf16 ratio)" %
+                                             NOMINAL_INT8_PER_BF16 if roof["bound"] == "tensor" else " HBM copy"))
+    if roof["bound"] == "tensor" and R.int8_peak_sus:
+        roof["frac_of_sustained"] = roof["achieved"] / R.int8_peak_sus
+    roof["traffic"] = committed_traffic(head_name, head_M, roof["kernel"])
 
+    ops = k2_ops(head_M, wl_head.N, wl_head.K)
     out = {
-        "metric": metric_name(), "value": value, "unit": "TOPS", "n_gpus": world, "steps": steps, "warmup": warm,
-        "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4", "data": "synthetic", "config": config_dict(wl, M, (P, pool_mb), world),
+        "metric": metric_name(), "value": job_tops(ops, steps, world, ms), "unit": "TOPS", "n_gpus": world,
+        "steps": steps, "warmup": warm, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int4", "data": "synthetic (seeded; Llama-shaped activation statistics)",
+        "config": config_dict(wl_head, head_M, (P, P * head["k1_bytes"] / 1e6 + P * head["k2_bytes"] / 1e6), world),
         "roofline": roof,
-        "kernels": {"k1_rotate_quant": {"ms": t_k1, "GB/s": k1_gbs, "frac_hbm": k1_gbs / peaks["hbm"],
-                                        "bytes_per_launch": b1},
-                    "k2_linear": {"ms": t_k2, "TOP/s": ops / (t_k2 * 1e-3) / 1e12,
-                                  "GB/s": b2 / (t_k2 * 1e-3) / 1e9, "frac_int8": ops / (t_k2 * 1e-3) / 1e12 / int8_peak,
-                                  "frac_hbm": b2 / (t_k2 * 1e-3) / 1e9 / peaks["hbm"], "bytes_per_launch": b2}},
+        "kernels": {"k1_rotate_quant": {"ms": head["k1_us"] / 1e3, "GB/s": head["k1_GBs"],
+                                        "frac_hbm": head["k1_frac_hbm"], "bytes_per_launch": head["k1_bytes"]},
+                    "k2_linear": {"ms": head["k2_us"] / 1e3, "TOP/s": head["k2_TOPs"], "GB/s": head["k2_GBs"],
+                                  "frac_int8": head["k2_TOPs"] / R.int8_peak,
+                                  "frac_hbm": head["k2_GBs"] / R.peaks["hbm"], "bytes_per_launch": head["k2_bytes"]}},
+        "targets": targets,
+        "workloads": workloads,
+        "serq_overhead": serq,
+        "peaks": {"hbm_GBs": R.peaks["hbm"], "bf16_TFs_burst": R.peaks["bf16"], "bf16_TFs_sustained": R.peaks["bf16_sus"],
+                  "int8_TOPs_denominator": R.int8_peak, "source": R.peaks["src"],
+                  "int8_cublaslt_8192_TOPs_live": int8_gemm_crosscheck(R)},
         "gpu_launches": 2 * steps,
         "clocks": clocks,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, M)
+        out["cpu_baseline"] = cpu_baseline(wl_head, head_M)
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del g_full, g_rem
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()

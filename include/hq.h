@@ -88,8 +88,9 @@ size_t hq_packed_weight_bytes(int64_t N, int64_t K);
  *  ld_x    row stride of X in elements, >= K, ld_x*2 a multiple of 16
  *  group   power of two, 8 <= group <= 4096, K % group == 0, K % 32 == 0
  *  H_signs device, [group] int8 in {+1,-1} with H_signs[0] == +1, or NULL (d = 1).
- *          The sign of d[0] is not checked on the device; values other than
- *          -1 are treated as +1.
+ *          Entries other than -1 are treated as +1.  H_signs[0] == -1 is
+ *          reported as HQ_ERR_ARG in the device status word (read it with
+ *          hq_last_device_status()); the outputs are then those of the given d.
  *  Xq      device, [M][K/2] packed int4 codes (output)
  *  sx      device, [M] fp32 scales (output)
  * Errors: HQ_ERR_ARG (M < 0, K <= 0, bad group, K % group, K % 32, NULL
@@ -131,7 +132,7 @@ hq_status hq_channel_sqnorm(const void* X, hq_dtype xt, int64_t M, int64_t K, in
  * hq_select_salient -- host helper: the r largest entries of norm2 (ties to the
  * lower index), written in ascending index order to sal (host, [r] int32).
  *  norm2   host, [K] fp32
- * Errors: HQ_ERR_ARG (NULL, r < 0, r > K).
+ * Errors: HQ_ERR_ARG (NULL, r < 0, r > K, a NaN in norm2).
  */
 hq_status hq_select_salient(const float* norm2, int64_t K, int32_t r, int32_t* sal);
 
@@ -171,7 +172,9 @@ hq_status w4_pack(const void* W, hq_dtype wt, int64_t N, int64_t K, int32_t grou
  *  r       0 <= r <= 256
  *  Rq      device, [N][ceil(r/2)] packed codes (output), the "A" operand
  *  sr      device, [N] fp16 bits (output), the "B" operand
- * Errors: HQ_ERR_ARG, HQ_ERR_CUDA.  sal_idx is not range-checked on the device.
+ * Errors: HQ_ERR_ARG, HQ_ERR_CUDA.  An index outside [0, K) is never read
+ * through: its error term is taken as 0 and the device status word records
+ * HQ_ERR_ARG.
  */
 hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* Wq,
                        const uint16_t* sw, const uint16_t* zw, int32_t group,
@@ -192,15 +195,19 @@ hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* 
  *  Wq, sw, zw, group   device, w4_pack outputs (Wq tile-major); group is 0 or a
  *           multiple of 128
  *  A, B     device, serq_prepare outputs Rq [N][ceil(r/2)] and sr [N] (NULL if r == 0)
- *  sal_idx  device, [r] int32 (NULL if r == 0)
+ *  sal_idx  device, [r] int32 (NULL if r == 0).  An index outside [0, K) is
+ *           never read through: it contributes 0 and the device status word
+ *           records HQ_ERR_ARG.
  *  r        0 <= r <= K (HQ_ERR_ARG otherwise); the kernels implement r <= 64
  *           with r % 8 == 0 (HQ_ERR_UNSUPPORTED otherwise)
  *  Y        device, [M][N] of type yt (HQ_F16, HQ_BF16 or HQ_F32) (output)
  *  workspace, ws_bytes   device scratch of at least
  *           hq_linear_workspace_size(M, N, K, group) bytes (may be NULL when
  *           that size is 0).  Zero it once before its first use; every call
- *           leaves it zeroed again.  Calls that share a workspace must not
- *           overlap in time.
+ *           that completes leaves it zeroed again.  A call whose device status
+ *           reports HQ_ERR_TIMEOUT may leave counters behind: zero the
+ *           workspace again before its next use.  Calls that share a
+ *           workspace must not overlap in time.
  * Requirements: K % 128 == 0, 0 < K <= 65536, N % 8 == 0; Xq, Wq, sw, zw,
  * B, Y and workspace 16-byte aligned, A 4-byte aligned (HQ_ERR_ALIGN).
  * Errors: HQ_ERR_ARG, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA.
@@ -232,12 +239,14 @@ hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,
  *    call before any stream capture.
  *  - All calls share the one array and it keeps the previous call's contents:
  *    each call first clears the arrival counters (an asynchronous memset on
- *    `stream`).  Calls that overlap on the GPU (different streams, or several
- *    host threads) race on the array and must not be issued.
- *  - Shapes whose scratch would exceed 8 MiB (hq_linear_workspace_size(M, N,
- *    K, group) > 8 MiB) are rejected with HQ_ERR_UNSUPPORTED before anything
- *    is enqueued.  Large M (> 64) uses the large-M kernel, which needs no
- *    scratch.
+ *    `stream`), so a timeout of an earlier call leaves nothing behind.  Calls
+ *    that overlap on the GPU (different streams, or several host threads)
+ *    race on the array and must not be issued.
+ *  - Every argument check of w4a4_linear runs first; a rejected call enqueues
+ *    nothing.  Shapes whose scratch would exceed 8 MiB (hq_linear_workspace_
+ *    size(M, N, K, group) > 8 MiB) are rejected with HQ_ERR_UNSUPPORTED, also
+ *    before anything is enqueued.  Large M (> 64) uses the large-M kernel,
+ *    which needs no scratch.
  * Arguments, results and the other errors are those of w4a4_linear.
  */
 hq_status w4a4_linear_noalloc(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,

@@ -392,7 +392,7 @@ void hqo_serq_prepare(const float* Wrot, int64_t N, int64_t K, const uint8_t* Wq
     memset(Rq, 0, (size_t)(N * ld));
     #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
-        float e[4096];
+        float* e = (float*)malloc((size_t)(r > 0 ? r : 1) * sizeof(float));   /* any r */
         float amax = 0.0f;
         for (int32_t j = 0; j < r; ++j) {
             int64_t k = sal[j];
@@ -408,6 +408,7 @@ void hqo_serq_prepare(const float* Wrot, int64_t N, int64_t K, const uint8_t* Wq
             if (s != 0.0f) q = (int)clampf(rintf(e[j] / s), -8.0f, 7.0f);
             put_nibble(Rq + n * ld, j, q);
         }
+        free(e);
     }
 }
 

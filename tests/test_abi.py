@@ -111,3 +111,54 @@ def test_select_salient_matches_numpy(L, seed):
     ref = np.sort(np.argsort(-n, kind="stable")[:r])
     assert np.array_equal(out, ref)
     assert L.lib.hq_select_salient(n.ctypes.data, K, K + 1, out.ctypes.data) == L.HQ_ERR_ARG
+
+
+def _lin_na(L, M=16, K=256, N=128, g=0, r=8, yt=1, Xq=P, sx=P, A=P, B=P, sal=P, Y=P):
+    return L.lib.w4a4_linear_noalloc(Xq, sx, M, K, P, P, P, N, g, A, B, sal, r, Y, yt, None)
+
+
+def test_noalloc_rejects_arguments_before_touching_the_device(L):
+    # the same checks as w4a4_linear, all on the host: with no GPU in this
+    # process, a call that reached its scratch set-up or memset would report
+    # HQ_ERR_CUDA instead of these codes
+    assert _lin_na(L, K=192) == L.HQ_ERR_UNSUPPORTED
+    assert _lin_na(L, N=100) == L.HQ_ERR_UNSUPPORTED
+    assert _lin_na(L, r=12) == L.HQ_ERR_UNSUPPORTED
+    assert _lin_na(L, g=96) == L.HQ_ERR_ARG
+    assert _lin_na(L, A=None) == L.HQ_ERR_ARG
+    assert _lin_na(L, sx=None) == L.HQ_ERR_ARG
+    assert _lin_na(L, Y=ct.c_void_p(24)) == L.HQ_ERR_ALIGN
+    assert _lin_na(L, yt=9) == L.HQ_ERR_UNSUPPORTED
+    assert _lin_na(L, M=0) == L.HQ_OK
+
+
+def test_select_salient_rejects_nan_norms(L):
+    n = np.ones(64, np.float32)
+    n[7] = np.nan
+    out = np.zeros(4, np.int32)
+    assert L.lib.hq_select_salient(n.ctypes.data, 64, 4, out.ctypes.data) == L.HQ_ERR_ARG
+
+
+def test_binding_validates_salient_indices_and_signs():
+    # W4A4Linear.prepare checks caller-supplied salient channels and the
+    # Hadamard sign vector on the host before any device work (the tensors
+    # here are CPU tensors: a check that let them through would fail later
+    # with a different error)
+    import torch
+
+    from w4a4_bit_gemm_hq_b200 import hq
+    W = torch.zeros((16, 256))
+    ok_d = torch.ones(128, dtype=torch.int8)
+    for bad in ([3, 3, 7, 9], [9, 7, 3, 1], [0, 1, 2, 256], [-1, 0, 1, 2]):
+        with pytest.raises(ValueError):
+            hq.W4A4Linear.prepare(W, 128, 0, 4, ok_d, sal_idx=torch.tensor(bad, dtype=torch.int32))
+    with pytest.raises(ValueError):   # r disagrees with the given indices
+        hq.W4A4Linear.prepare(W, 128, 0, 8, ok_d, sal_idx=torch.tensor([0, 1, 2, 3], dtype=torch.int32))
+    bad_d = ok_d.clone()
+    bad_d[0] = -1                      # first row of H must stay all ones
+    with pytest.raises(ValueError):
+        hq.W4A4Linear.prepare(W, 128, 0, 0, bad_d)
+    with pytest.raises(ValueError):    # entries other than +-1
+        hq.W4A4Linear.prepare(W, 128, 0, 0, torch.full((128,), 2, dtype=torch.int8))
+    with pytest.raises(ValueError):    # one sign per channel of a group
+        hq.W4A4Linear.prepare(W, 128, 0, 0, torch.ones(64, dtype=torch.int8))

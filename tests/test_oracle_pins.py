@@ -364,10 +364,43 @@ def test_accum_brute_force_matches_numpy_matmul(gw):
     assert np.array_equal(acc_c, qx[:, sal].astype(np.int64) @ qr.astype(np.int64).T)
 
 
-def test_accum_int32_worst_case_fits():
-    # K * 7 * 15 (activation code times an asymmetric weight offset) < 2^31
-    K = 11008
-    assert K * 7 * 15 < 2 ** 31
+@pytest.mark.parametrize("gw", [0, 128])
+def test_accum_extreme_codes_closed_form(gw):
+    # every product at its extreme: activation codes -7 against weight values
+    # -8 (symmetric codes) or 0 - 15 (asymmetric code 0 with zero point 15);
+    # the integer accumulators must equal the closed forms K*56 / 128*105 per
+    # group exactly (no wrap-around, no lost term) and fit in int32, and the
+    # SERQ term with all codes -8 likewise
+    K, N, M = 11008 if gw else 8192, 3, 2
+    qx = np.full((M, K), -7, np.int8)
+    Xq = O.pack_s4(qx)
+    if gw:
+        Wq = O.pack_s4(np.zeros((N, K), np.int8))            # unsigned code 0
+        z = np.full((K // gw, N), 15.0, np.float16)
+        want = 7 * 15 * gw                                     # (-7) * (0 - 15) per element
+    else:
+        Wq = O.pack_s4(np.full((N, K), -8, np.int8))
+        z = None
+        want = 56 * K
+    sal = np.arange(0, 64, dtype=np.int32) * 7
+    Rq = O.pack_s4(np.full((N, 64), -8, np.int8))
+    acc, acc_c = O.accum(Xq, K, Wq, z, gw, Rq, sal)
+    assert np.all(acc == want) and acc.max() < 2 ** 31
+    assert np.all(acc_c == 56 * 64)
+
+
+def test_w4_pack_zero_point_zero_is_positive_zero():
+    # a group whose minimum is 0 has zero point 0, stored as +0 (bits 0x0000),
+    # never -0 (0x8000); other zero points are exact small integers
+    rng = np.random.default_rng(11)
+    K = 256
+    W = np.abs(rng.standard_normal((4, K))).astype(np.float32)
+    W[:, 0] = 0.0                                   # minimum 0 in group 0 of every row
+    W[:, 128:] = -W[:, 128:] - 0.1                  # group 1: all negative -> z = 15
+    _, sw, zw = O.w4_pack(W, "f32", 128)
+    zb = np.ascontiguousarray(zw).view(np.uint16)
+    assert np.all(zb[0] == 0x0000)
+    assert np.all(zw[1] == 15.0)
 
 
 def test_epilogue_against_dequantised_float_matmul():

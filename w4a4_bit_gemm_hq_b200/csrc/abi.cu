@@ -104,16 +104,29 @@ static hq_status run_gemm(GemmArgs& a, int out, bool small, void* ws, size_t ws_
     return launch_gemm_prefill(a, out, st, nsm);
 }
 
-extern "C" hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
-                                 const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
-                                 const uint16_t* B, const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt,
-                                 void* workspace, size_t ws_bytes, void* stream) {
+namespace hq {
+// Every check of w4a4_linear except the workspace's (shared with
+// w4a4_linear_noalloc, which must not enqueue anything for a rejected call).
+hq_status check_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
+                       const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
+                       const uint16_t* B, const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt) {
     hq_status s = check_gemm(Xq, M, K, Wq, zw, N, group, A, sal_idx, r);
     if (s != HQ_OK) return s;
     if (yt != HQ_F16 && yt != HQ_BF16 && yt != HQ_F32) return HQ_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return HQ_OK;
     if (!sx || !sw || !Y || (r > 0 && !B)) return HQ_ERR_ARG;
     if (!al16(sw) || !al16(Y) || (r > 0 && !al16(B))) return HQ_ERR_ALIGN;
+    return HQ_OK;
+}
+}  // namespace hq
+
+extern "C" hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
+                                 const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
+                                 const uint16_t* B, const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+    const hq_status s = check_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt);
+    if (s != HQ_OK) return s;
+    if (M == 0 || N == 0) return HQ_OK;
     GemmArgs a{};
     a.Xq = Xq; a.sx = sx; a.Wq = Wq; a.sw = sw; a.zw = zw; a.Rq = A; a.sr = B; a.sal = sal_idx;
     a.Y = Y;

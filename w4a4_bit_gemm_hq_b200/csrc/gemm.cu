@@ -188,7 +188,11 @@ __device__ __forceinline__ void gather_xs_smem(const GemmArgs& p, const int32_t*
             nib[b][t] = 0u;
             if (mv && 8 * i < p.r) {
                 const int k = sal_s[8 * i + t];
-                nib[b][t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
+                if (static_cast<unsigned>(k) < static_cast<unsigned>(p.K)) {
+                    nib[b][t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
+                } else {
+                    record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
+                }
             }
         }
     }

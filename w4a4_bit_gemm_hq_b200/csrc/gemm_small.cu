@@ -422,8 +422,12 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
                     const int j = 8 * i + 2 * e + h;
                     if (j < p.r) {
                         const int k = sal_s[j];
-                        const int nib = (__ldg(xrow + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
-                        word |= (static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu) << (8 * e);
+                        if (static_cast<unsigned>(k) < static_cast<unsigned>(p.K)) {
+                            const int nib = (__ldg(xrow + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
+                            word |= (static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu) << (8 * e);
+                        } else {
+                            record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
+                        }
                     }
                 }
             }
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
         int abuf = 0;
         uint32_t accph = 0;
         uint32_t* ws_cnt = static_cast<uint32_t*>(p.ws);
-        float* ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(p.ws) + ((plan.ntiles * 4 + 15) / 16) * 16);
+        float* ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(p.ws) + small_counter_bytes(plan.ntiles));
         const int sh = ASYM ? 4 : 8;
         const int G = ASYM ? p.K / p.gw : 1;
         int li = 0;
@@ -605,8 +609,7 @@ bool small_supported(int64_t M, int gw) {
 size_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int gw, int nsm) {
     if (!small_supported(M, gw) || N <= 0 || K < sk::BK) return 0;
     const SkPlan p = sk_plan(M, N, K, gw, nsm);
-    const size_t cnt = ((static_cast<size_t>(p.ntiles) * 4 + 15) / 16) * 16;
-    return cnt + static_cast<size_t>(p.ntiles) * p.maxc * nt_for(M) * sk::BMW * sizeof(float);
+    return small_counter_bytes(p.ntiles) + static_cast<size_t>(p.ntiles) * p.maxc * nt_for(M) * sk::BMW * sizeof(float);
 }
 
 template <int NT, bool ASYM, int OUT>

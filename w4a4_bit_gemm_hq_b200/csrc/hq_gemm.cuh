@@ -27,6 +27,17 @@ struct GemmArgs {
     uint64_t limit_ns;      // bounded-wait limit
 };
 
+// Bytes at the start of the small-M kernel's workspace holding its per-tile
+// arrival counters (one uint32 per 128-row weight tile, padded to 16 bytes);
+// the partial sums follow.  Every call leaves the counters at zero.
+__host__ __device__ inline size_t small_counter_bytes(int64_t ntiles) {
+    return static_cast<size_t>((ntiles * 4 + 15) / 16 * 16);
+}
+inline size_t small_counter_bytes_for_n(int64_t N) { return small_counter_bytes((N + 127) / 128); }
+
+hq_status check_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
+                       const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
+                       const uint16_t* B, const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt);
 hq_status launch_gemm_prefill(const GemmArgs& a, int out, cudaStream_t st, int nsm);
 hq_status launch_gemm_small(const GemmArgs& a, int out, cudaStream_t st, int nsm);
 size_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int gw, int nsm);

@@ -55,22 +55,21 @@ extern "C" hq_status w4a4_linear_noalloc(const uint8_t* Xq, const float* sx, int
                                          const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
                                          int32_t group, const uint8_t* A, const uint16_t* B,
                                          const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt, void* stream) {
-    if (M > 0 && N > 0 && K > 0 && group >= 0 && small_supported(M, group)) {
-        const size_t need = hq_linear_workspace_size(M, N, K, group);
-        if (need > kNoAllocScratchBytes) return HQ_ERR_UNSUPPORTED;   // beyond the fixed scratch
-        if (need > 0) {
-            void* ws = nullptr;
-            const hq_status s = scratch_for_current_device(&ws);
-            if (s != HQ_OK) return s;
-            // the per-tile arrival counters at the start of the scratch must be
-            // zero; the array keeps whatever the previous call left in it
-            const size_t counters = ((static_cast<size_t>((N + 127) / 128) * 4 + 15) / 16) * 16;
-            if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-                return HQ_ERR_CUDA;
-            return w4a4_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt, ws,
-                               kNoAllocScratchBytes, stream);
-        }
-    }
-    // the large-M kernel needs no scratch
-    return w4a4_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt, nullptr, 0, stream);
+    // every argument check first: a rejected call enqueues nothing
+    const hq_status chk = check_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt);
+    if (chk != HQ_OK) return chk;
+    if (M == 0 || N == 0) return HQ_OK;
+    const size_t need = small_supported(M, group) ? hq_linear_workspace_size(M, N, K, group) : 0;
+    if (need > kNoAllocScratchBytes) return HQ_ERR_UNSUPPORTED;   // beyond the fixed scratch
+    if (need == 0)   // the large-M kernel needs no scratch
+        return w4a4_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt, nullptr, 0, stream);
+    void* ws = nullptr;
+    const hq_status s = scratch_for_current_device(&ws);
+    if (s != HQ_OK) return s;
+    // the per-tile arrival counters at the start of the scratch must be zero;
+    // the array keeps whatever the previous call (of any shape) left in it
+    if (cudaMemsetAsync(ws, 0, small_counter_bytes_for_n(N), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return HQ_ERR_CUDA;
+    return w4a4_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt, ws, kNoAllocScratchBytes,
+                       stream);
 }

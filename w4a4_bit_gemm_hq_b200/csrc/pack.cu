@@ -134,7 +134,9 @@ __global__ void k_serq_prepare(const float* __restrict__ Wrot, int64_t N, int64_
         for (int h = 0; h < 2; ++h) {
             const int j = 2 * (lane + 32 * i) + h;
             float ev = 0.f;
-            if (j < r) {
+            if (j < r && (sal[j] < 0 || sal[j] >= K)) {
+                record_status(HQ_ERR_ARG);   // a salient index outside [0, K): its error term is 0
+            } else if (j < r) {
                 const int64_t k = sal[j];
                 const uint8_t byte = Wq[wq_offset(n, k / 2, K / 128)];
                 const int nib = (byte >> (4 * (k & 1))) & 0xF;
@@ -219,6 +221,8 @@ extern "C" hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, cons
 
 extern "C" hq_status hq_select_salient(const float* norm2, int64_t K, int32_t r, int32_t* sal) {
     if (!norm2 || !sal || K <= 0 || r < 0 || r > K) return HQ_ERR_ARG;
+    for (int64_t k = 0; k < K; ++k)
+        if (norm2[k] != norm2[k]) return HQ_ERR_ARG;   // a NaN norm has no order
     std::vector<int64_t> idx(static_cast<size_t>(K));
     for (int64_t k = 0; k < K; ++k) idx[static_cast<size_t>(k)] = k;
     // largest first; equal values keep the lower index first

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
     float accsq[MODE == MODE_SQNORM ? EPT : 1];
 #pragma unroll
     for (int i = 0; i < (MODE == MODE_SQNORM ? EPT : 1); ++i) accsq[i] = 0.f;
+    if (blockIdx.x == 0 && t == 0 && dsign != nullptr && dsign[0] == -1) record_status(HQ_ERR_ARG);   // d[0] must be +1
     if (active && dsign != nullptr) {
         const int p0 = static_cast<int>(col0 % G);
 #pragma unroll

@@ -164,6 +164,9 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
         fence_mbar_init();
     }
     if constexpr (SIGNED) {
+        // d[0] must be +1 (the first row of H all ones); the rotation still
+        // uses the given d, and the status word reports the violation
+        if (blockIdx.x == 0 && threadIdx.x == 0 && dsign[0] == -1) record_status(HQ_ERR_ARG);
         // sign table: pattern p covers channels 128 p + c (c < 128) of a group
         // (for groups up to 128 channels, d[c mod G]); bf16 entries are two
         // words per element pair (bit 31 = sign of the even element, bit 31 =

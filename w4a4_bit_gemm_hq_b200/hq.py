@@ -185,9 +185,33 @@ class W4A4Linear:
         self.K, self.N, self.out_dtype = K, N, out_dtype
         self._ws = {}
 
+    @staticmethod
+    def check_inputs(K, group, r, H_signs=None, sal_idx=None):
+        """Host-side checks of the caller-supplied Hadamard signs and salient
+        channels (ValueError): H_signs is `group` entries in {+1, -1} with
+        H_signs[0] = +1 (the first row of H all ones); sal_idx is r strictly
+        ascending indices in [0, K)."""
+        if H_signs is not None:
+            d = H_signs.detach().to("cpu")
+            if d.dim() != 1 or d.numel() != group:
+                raise ValueError("H_signs must hold one sign per channel of a group (%d)" % group)
+            if not bool(((d == 1) | (d == -1)).all()):
+                raise ValueError("H_signs entries must be +1 or -1")
+            if int(d[0]) != 1:
+                raise ValueError("H_signs[0] must be +1 (the first row of H is all ones)")
+        if sal_idx is not None:
+            s = sal_idx.detach().to("cpu").to(torch.int64).reshape(-1)
+            if s.numel() != r:
+                raise ValueError("sal_idx holds %d indices, r = %d" % (s.numel(), r))
+            if r and (int(s.min()) < 0 or int(s.max()) >= K):
+                raise ValueError("sal_idx entries must lie in [0, K)")
+            if r > 1 and not bool((s[1:] > s[:-1]).all()):
+                raise ValueError("sal_idx must be strictly ascending")
+
     @classmethod
     def prepare(cls, W, group, gw, r, H_signs=None, X_calib=None, sal_idx=None, out_dtype=torch.bfloat16):
         N, K = W.shape
+        cls.check_inputs(K, group, r, H_signs, sal_idx)
         W_rot = hq_rotate(W, group, H_signs)
         Wq, sw, zw = w4_pack(W_rot, gw)
         if sal_idx is None and r > 0:
@@ -200,6 +224,13 @@ class W4A4Linear:
             sal_idx, Rq, sr = None, None, None
         del W_rot
         return cls(group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype)
+
+    def reset_workspaces(self):
+        """Zero the cached small-M workspaces.  Needed only after a call whose
+        device status reported HQ_ERR_TIMEOUT: a kernel that gave up may leave
+        arrival counters behind (every completed call leaves them at zero)."""
+        for ws in self._ws.values():
+            ws.zero_()
 
     def workspace(self, M, device):
         need = hq_linear_workspace_size(M, self.N, self.K, self.gw)
