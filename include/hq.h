@@ -193,7 +193,7 @@ hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* 
  * computed in fp32 and rounded once to yt.  One launch.
  *  Xq, sx   device, hq_rotate_quant outputs, [M][K/2] and [M]
  *  Wq, sw, zw, group   device, w4_pack outputs (Wq tile-major); group is 0 or a
- *           multiple of 128
+ *           multiple of 128 up to 2048 (HQ_ERR_UNSUPPORTED beyond)
  *  A, B     device, serq_prepare outputs Rq [N][ceil(r/2)] and sr [N] (NULL if r == 0)
  *  sal_idx  device, [r] int32 (NULL if r == 0).  An index outside [0, K) is
  *           never read through: it contributes 0 and the device status word

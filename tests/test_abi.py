@@ -84,6 +84,7 @@ def test_linear_argument_errors(L):
     assert _lin(L, K=192) == L.HQ_ERR_UNSUPPORTED          # K % 128
     assert _lin(L, N=100) == L.HQ_ERR_UNSUPPORTED          # N % 8
     assert _lin(L, g=64) == L.HQ_ERR_UNSUPPORTED           # group not a multiple of 128
+    assert _lin(L, K=4096, g=4096) == L.HQ_ERR_UNSUPPORTED  # group beyond 2048
     assert _lin(L, g=96) == L.HQ_ERR_ARG                   # K % group
     assert _lin(L, r=72) == L.HQ_ERR_UNSUPPORTED           # r > 64
     assert _lin(L, r=12) == L.HQ_ERR_UNSUPPORTED           # r % 8

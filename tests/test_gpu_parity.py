@@ -309,6 +309,9 @@ GEMM_CASES = [
     # 32-wide mma.sync K steps (the second one ragged for r = 40)
     (256, 512, 1024, 0, 64),
     (300, 264, 512, 0, 40),
+    # the largest weight group the large-M kernel takes (its accumulators are
+    # read back as floats: exact while |acc| < 2^22)
+    (160, 256, 4096, 2048, 8),
 ]
 
 
@@ -365,6 +368,30 @@ def test_small_m_linear_within_tolerance(M, N, K, gw, r, out):
                         workspace=ws)
     assert torch.equal(Y, Y2)          # same workspace, counters were reset: identical bytes
     assert int(ws.view(torch.int32)[: (N + 127) // 128].abs().sum()) == 0
+    no_device_error()
+
+
+@pytest.mark.parametrize("sign", [1, -1])
+def test_group_accumulators_extreme_codes(sign):
+    # every product at its extreme in the largest weight group the large-M
+    # kernel takes: activation codes -7 (or +7) against weight values 0 - 15;
+    # the group accumulator is +-7*15*2048 and the output matches the oracle
+    M, N, K, gw = 256, 264, 4096, 2048
+    Xq = np.full((M, K // 2), 0x99 if sign > 0 else 0x77, np.uint8)     # codes -7 / +7
+    sx = np.full((M,), 0.25, np.float32)
+    Wq = np.zeros((N, K // 2), np.uint8)                                 # unsigned code 0
+    zw = np.full((K // gw, N), 15.0, np.float16)
+    sw = np.full((K // gw, N), 0.5, np.float16)
+    acc_o, _ = O.accum(Xq, K, Wq, zw, gw)
+    assert np.all(acc_o == sign * 7 * 15 * gw)
+    t = dict(Xq=Xq, sx=sx, Wq=Wq, sw=sw, zw=zw, sal=np.zeros((0,), np.int32),
+             Rq=np.zeros((N, 0), np.uint8), sr=np.zeros((N,), np.float16))
+    g = _dev_inputs(t)
+    acc, _ = hq.hq_debug_accum(g["Xq"], g["Wq"], g["zw"], gw, None, None, N)
+    assert_same(host(acc).astype(np.int64), acc_o, "acc")
+    y64 = O.epilogue_f64(acc_o, None, sx, sw, None)
+    Y = hq.w4a4_linear(g["Xq"], g["sx"], g["Wq"], g["sw"], g["zw"], gw, None, None, None, torch.float32)
+    assert_y_close(y_host(Y), y64, 1e-3)
     no_device_error()
 
 

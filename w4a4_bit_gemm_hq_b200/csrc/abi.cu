@@ -42,7 +42,9 @@ static hq_status check_gemm(const uint8_t* Xq, int64_t M, int64_t K, const uint8
     if (r < 0 || r > K) return HQ_ERR_ARG;
     if (group < 0 || (group > 0 && K % group != 0)) return HQ_ERR_ARG;
     if (K % 128 != 0 || K > 65536 || N % 8 != 0) return HQ_ERR_UNSUPPORTED;
-    if (group % 128 != 0) return HQ_ERR_UNSUPPORTED;
+    // group weights: multiples of 128 up to 2048 inputs (the large-M kernel's
+    // group accumulators are read back as floats, exact for |acc| < 2^22)
+    if (group % 128 != 0 || group > 2048) return HQ_ERR_UNSUPPORTED;
     if (r > 64 || r % 8 != 0) return HQ_ERR_UNSUPPORTED;
     if (M > (1ll << 30) || N > (1ll << 30)) return HQ_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return HQ_OK;

@@ -437,7 +437,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 for (int kb = 0; ok && kb < KB; ++kb) {
                     const bool first = (kb % GPK) == 0;
                     if (first) {
-                        if (!mbar_wait_cluster(acce_bar(abuf), ((aphase >> abuf) & 1u) ^ 1u, p.limit_ns)) {
+                        // per-channel weights: the buffer's previous phase (free from the
+                        // start); group weights: its epilogues' preload of the next use
+                        const uint32_t par = ASYM ? ((aphase >> abuf) & 1u) : (((aphase >> abuf) & 1u) ^ 1u);
+                        if (!mbar_wait_cluster(acce_bar(abuf), par, p.limit_ns)) {
                             ok = false;
                             break;
                         }
@@ -451,7 +454,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                     const uint32_t dcol = tmem_base + static_cast<uint32_t>(abuf * BN);
 #pragma unroll
                     for (int kk = 0; kk < pf::BK / 32; ++kk)
-                        mma_i8_ss_pair(dcol, adesc + 2u * kk, bdesc + 2u * kk, IDESC, (first && kk == 0) ? 0u : 1u);
+                        mma_i8_ss_pair(dcol, adesc + 2u * kk, bdesc + 2u * kk, IDESC,
+                                       (!ASYM && first && kk == 0) ? 0u : 1u);   // group weights add onto the preload
                     tc_commit_pair_mc(empty_bar(stage), 0x3);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     if ((kb % GPK) == GPK - 1) {
@@ -540,13 +544,38 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
             }
         } else {
-            // group weights: one accumulator per (tile, group); per-thread fp32
-            // partial sums in the mma.sync fragment layout, 64 columns x the
-            // warp's 32 rows: ypart[chunk][row half][8-col group][4]
+            // group weights: one accumulator per (tile, group), drained into
+            // per-thread fp32 partial sums in the mma.sync fragment layout, 64
+            // columns x the warp's 32 rows: yp[chunk][row tile][8-col group][row half]
+            // holds the column pair (2 t4, 2 t4 + 1).
+            //
+            // Every buffer is preloaded with the bit pattern of 1.5 * 2^23 before
+            // a group's MMAs add onto it, so a drained int32 accumulator reads as
+            // the float 1.5 * 2^23 + acc, exactly (|acc| < 2^22): one packed
+            // subtract and one packed fma per column pair convert, scale and
+            // accumulate, with no integer -> float conversion instruction.
             const uint32_t* xs_w = reinterpret_cast<const uint32_t*>(smem + L::OFF_XS);
             const int g8 = lane >> 2, t4 = lane & 3;
             const int ksteps = (p.r + 31) / 32;
             constexpr int NC = BN / 2 / 32;   // 32-column chunks per warp
+            constexpr uint32_t MAGIC = 0x4B400000u;   // bits of 1.5 * 2^23
+            const float2 cmag = make_float2(12582912.0f, 12582912.0f);
+            auto preload = [&](int b) {
+                const uint32_t ta = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                    static_cast<uint32_t>(b * BN + hcol * (BN / 2));
+#pragma unroll
+                for (int c = 0; c < BN / 2 / 32; ++c) tmem_fill_32x32b_x32(ta + 32u * c, MAGIC);
+                tmem_wait_st();
+            };
+            auto release = [&](int b) {   // the buffer is preloaded: hand it to the MMA
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce_remote0 + 8u * static_cast<uint32_t>(b));
+            };
+            for (int b = 0; b < NACC; ++b) {
+                preload(b);
+                release(b);
+            }
             for (int tile = pair; tile < num_tiles; tile += npairs) {
                 const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM, n0 = (tile / MT) * BN;
                 const int mq0 = m0 + 32 * q;
@@ -565,8 +594,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                         if constexpr (OUT != OUT_DEBUG) sxr[mt][h] = m < p.M ? __ldg(p.sx + m) : 0.f;
                     }
                 named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);
-                // ---- SERQ term first: ypart = sr[n] * (X[m,S] . Rq[n,:])
-                float ypart[NC][2][4][4];
+                // ---- SERQ term first: yp = sr[n] * (X[m,S] . Rq[n,:])
+                float2 yp[NC][2][4][2];
                 {
                     uint32_t afr[2][2][4];
 #pragma unroll
@@ -606,17 +635,22 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                             for (int nt = 0; nt < 4; ++nt) {
                                 const int cl = scol + 8 * nt + 2 * t4;
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const int32_t cv = cc[nt][i] >> 4;   // Rq codes carry 16
+                                for (int h = 0; h < 2; ++h) {
+                                    // the Rq codes carry a factor 16, like yp until the end of the tile
+                                    const int32_t c0 = cc[nt][2 * h], c1 = cc[nt][2 * h + 1];
                                     if constexpr (OUT == OUT_DEBUG) {
-                                        const int m = mq0 + 16 * mt + g8 + 8 * (i >> 1);
-                                        const int n = n0 + cl + (i & 1);
-                                        if (p.r > 0 && m < p.M && n < p.N)
-                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n] = cv;
-                                        ypart[c][mt][nt][i] = 0.f;
+                                        const int m = mq0 + 16 * mt + g8 + 8 * h;
+                                        const int n = n0 + cl;
+                                        if (p.r > 0 && m < p.M && n < p.N) {
+                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n] = c0 >> 4;
+                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n + 1] = c1 >> 4;
+                                        }
+                                        yp[c][mt][nt][h] = make_float2(0.f, 0.f);
                                     } else {
-                                        ypart[c][mt][nt][i] =
-                                            (p.r > 0) ? __fmul_rn(sr_s[cl + (i & 1)], static_cast<float>(cv)) : 0.f;
+                                        yp[c][mt][nt][h] =
+                                            (p.r > 0) ? make_float2(__fmul_rn(sr_s[cl], static_cast<float>(c0)),
+                                                                    __fmul_rn(sr_s[cl + 1], static_cast<float>(c1)))
+                                                      : make_float2(0.f, 0.f);
                                     }
                                 }
                             }
@@ -654,6 +688,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
 #pragma unroll
                         for (int c = 0; c < NC; ++c) {
                             const int scol = hcol * (BN / 2) + 32 * c;
+                            // sw of the chunk's column pairs (yp carries the factor 16 of the
+                            // activation codes until the end of the tile)
+                            float2 swf[4];
+#pragma unroll
+                            for (int nt = 0; nt < 4; ++nt)
+                                swf[nt] = __half22float2(*reinterpret_cast<const __half2*>(&swc[c][nt]));
 #pragma unroll
                             for (int mt = 0; mt < 2; ++mt) {
                                 uint32_t v[16];
@@ -663,26 +703,29 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                                 tmem_wait_ld();
 #pragma unroll
                                 for (int nt = 0; nt < 4; ++nt) {
-                                    const float2 swf = __half22float2(*reinterpret_cast<const __half2*>(&swc[c][nt]));
 #pragma unroll
-                                    for (int i = 0; i < 4; ++i) {
-                                        const int32_t av = static_cast<int32_t>(v[4 * nt + i]) >> 4;
+                                    for (int h = 0; h < 2; ++h) {
+                                        const float2 f = make_float2(__uint_as_float(v[4 * nt + 2 * h]),
+                                                                     __uint_as_float(v[4 * nt + 2 * h + 1]));
                                         if constexpr (OUT == OUT_DEBUG) {
-                                            const int m = mq0 + 16 * mt + g8 + 8 * (i >> 1);
-                                            const int n = n0 + scol + 8 * nt + 2 * t4 + (i & 1);
-                                            if (m < p.M && n < p.N)
-                                                p.dbg_acc[(static_cast<int64_t>(m) * p.N + n) * NG + g] = av;
+                                            const int m = mq0 + 16 * mt + g8 + 8 * h;
+                                            const int n = n0 + scol + 8 * nt + 2 * t4;
+                                            if (m < p.M && n < p.N) {
+                                                const int64_t o = (static_cast<int64_t>(m) * p.N + n) * NG + g;
+                                                p.dbg_acc[o] = static_cast<int32_t>(v[4 * nt + 2 * h] - MAGIC) >> 4;
+                                                p.dbg_acc[o + NG] = static_cast<int32_t>(v[4 * nt + 2 * h + 1] - MAGIC) >> 4;
+                                            }
                                         } else {
-                                            ypart[c][mt][nt][i] = __fmaf_rn((i & 1) ? swf.y : swf.x,
-                                                                            static_cast<float>(av), ypart[c][mt][nt][i]);
+                                            // f - 1.5 * 2^23 = 16 acc exactly; yp += sw (16 acc)
+                                            yp[c][mt][nt][h] = __ffma2_rn(swf[nt], __fadd2_rn(f, make_float2(-cmag.x, -cmag.y)),
+                                                                          yp[c][mt][nt][h]);
                                         }
                                     }
                                 }
                             }
                         }
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(acce_remote0 + 8u * static_cast<uint32_t>(abuf));
+                        preload(abuf);
+                        release(abuf);
                     }
                     aphase ^= 1u << abuf;
                     abuf = (abuf + 1 == NACC) ? 0 : abuf + 1;
@@ -691,7 +734,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
 #pragma unroll
                         for (int nt = 0; nt < 4; ++nt) swc[c][nt] = swn[c][nt];
                 }
-                // ---- Y = sx[m] * ypart
+                // ---- Y = sx[m] * yp
                 if constexpr (OUT != OUT_DEBUG) {
                     if (ok) {
 #pragma unroll
@@ -706,9 +749,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                                     for (int h = 0; h < 2; ++h) {
                                         const int m = mq0 + 16 * mt + g8 + 8 * h;
                                         if (m >= p.M) continue;
+                                        // yp / 16 is exact: the same bits as accumulating sw * acc
                                         store_out2<OUT>(p.Y, static_cast<int64_t>(m) * p.N + n,
-                                                        __fmul_rn(sxr[mt][h], ypart[c][mt][nt][2 * h]),
-                                                        __fmul_rn(sxr[mt][h], ypart[c][mt][nt][2 * h + 1]));
+                                                        __fmul_rn(sxr[mt][h], __fmul_rn(yp[c][mt][nt][h].x, 0.0625f)),
+                                                        __fmul_rn(sxr[mt][h], __fmul_rn(yp[c][mt][nt][h].y, 0.0625f)));
                                     }
                                 }
                     }
