@@ -255,6 +255,44 @@ hq_status w4a4_linear_noalloc(const uint8_t* Xq, const float* sx, int64_t M, int
                               const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt, void* stream);
 
 /*
+ * W4A8 -- the layer with 8-bit activations for quantisation-sensitive layers.
+ * Source: "DynamicPTQ", Methodology 2 (the sensitive layers keep 8-bit
+ * activations while the rest of the model runs at 4 bit); "SERQ ...", section
+ * 4 (the same reconstruction evaluated at W4A8).  Weights, SERQ term and
+ * epilogue are those of the W4A4 calls.
+ *
+ * hq_rotate_quant8 -- hq_rotate_quant with 8-bit codes:
+ *   amax = max over the row of |u|,  q = clamp(rint(fl32(u * fl32(127/amax))), -127, 127)
+ *   (all 0 if amax == 0),  sx[m] = fl32(fl32(amax/127) * fl32(1/sqrt(group))).
+ *  Xq8     device, [M][K] int8 codes, one per byte, row-major (output)
+ * Other arguments, layouts and errors as hq_rotate_quant.
+ */
+hq_status hq_rotate_quant8(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                           int32_t group, const int8_t* H_signs, int8_t* Xq8, float* sx,
+                           void* stream);
+
+/*
+ * w4a8_linear -- w4a4_linear with the activation codes of hq_rotate_quant8:
+ *   acc_b[m][n] = sum_{k in group b} q8x[m][k] * (qw[n][k] - z[b][n]),
+ *   acc_c[m][n] = sum_{j<r} q8x[m][S_j] * qr[n][j],  Y as w4a4_linear.
+ *  Xq8     device, [M][K] int8 (16-byte aligned)
+ * Every other argument, requirement, workspace rule and error as w4a4_linear.
+ */
+hq_status w4a8_linear(const int8_t* Xq8, const float* sx, int64_t M, int64_t K,
+                      const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
+                      int32_t group, const uint8_t* A, const uint16_t* B,
+                      const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hq_debug_accum8 -- hq_debug_accum for w4a8_linear's kernels (test hook).
+ */
+hq_status hq_debug_accum8(const int8_t* Xq8, int64_t M, int64_t K, const uint8_t* Wq,
+                          const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
+                          const int32_t* sal_idx, int32_t r, int32_t* acc, int32_t* acc_c,
+                          int32_t decode, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * hq_debug_accum -- test hook: runs the GEMM kernel of w4a4_linear with the
  * epilogue replaced by a raw store of the exact integer accumulators.
  *  acc     device, int32 [M][N][G] with G = K/group (1 when group == 0)

@@ -163,3 +163,19 @@ def test_binding_validates_salient_indices_and_signs():
         hq.W4A4Linear.prepare(W, 128, 0, 0, torch.full((128,), 2, dtype=torch.int8))
     with pytest.raises(ValueError):    # one sign per channel of a group
         hq.W4A4Linear.prepare(W, 128, 0, 0, torch.ones(64, dtype=torch.int8))
+
+
+def test_w4a8_argument_errors(L):
+    # same checks as the W4A4 calls, on the host
+    assert L.lib.hq_rotate_quant8(P, 0, 4, 240, 240, 16, None, P, P, None) == L.HQ_ERR_ARG      # K % 32
+    assert L.lib.hq_rotate_quant8(P, 2, 4, 256, 256, 128, None, P, P, None) == L.HQ_ERR_UNSUPPORTED
+    assert L.lib.hq_rotate_quant8(ct.c_void_p(18), 0, 4, 256, 256, 128, None, P, P, None) == L.HQ_ERR_ALIGN
+    assert L.lib.hq_rotate_quant8(None, 0, 0, 256, 256, 128, None, None, None, None) == L.HQ_OK   # M == 0
+    lin8 = lambda **kw: L.lib.w4a8_linear(kw.get("Xq", P), P, kw.get("M", 16), kw.get("K", 256), P, P, P,
+                                          kw.get("N", 128), kw.get("g", 0), P, P, P, kw.get("r", 8), P, 1,
+                                          None, 0, None)
+    assert lin8(K=192) == L.HQ_ERR_UNSUPPORTED
+    assert lin8(r=12) == L.HQ_ERR_UNSUPPORTED
+    assert lin8(g=96) == L.HQ_ERR_ARG
+    assert lin8(Xq=ct.c_void_p(8)) == L.HQ_ERR_ALIGN
+    assert lin8(M=0) == L.HQ_OK

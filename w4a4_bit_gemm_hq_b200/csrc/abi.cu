@@ -133,6 +133,7 @@ extern "C" hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, 
     a.Xq = Xq; a.sx = sx; a.Wq = Wq; a.sw = sw; a.zw = zw; a.Rq = A; a.sr = B; a.sal = sal_idx;
     a.Y = Y;
     a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
+    a.act_bits = 4;
     return run_gemm(a, yt, small_supported(M, group), workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -150,5 +151,43 @@ extern "C" hq_status hq_debug_accum(const uint8_t* Xq, int64_t M, int64_t K, con
     a.Xq = Xq; a.Wq = Wq; a.zw = zw; a.Rq = A; a.sal = sal_idx;
     a.dbg_acc = acc; a.dbg_acc_c = acc_c;
     a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
+    a.act_bits = 4;
     return run_gemm(a, OUT_DEBUG, decode != 0, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------------------------ W4A8
+// The same GEMM with 8-bit activation codes (hq_rotate_quant8 outputs).
+extern "C" hq_status w4a8_linear(const int8_t* Xq8, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
+                                 const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
+                                 const uint16_t* B, const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+    const uint8_t* X8 = reinterpret_cast<const uint8_t*>(Xq8);
+    const hq_status s = check_linear(X8, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt);
+    if (s != HQ_OK) return s;
+    if (M == 0 || N == 0) return HQ_OK;
+    GemmArgs a{};
+    a.Xq = X8; a.sx = sx; a.Wq = Wq; a.sw = sw; a.zw = zw; a.Rq = A; a.sr = B; a.sal = sal_idx;
+    a.Y = Y;
+    a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
+    a.act_bits = 8;
+    return run_gemm(a, yt, small_supported(M, group), workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hq_status hq_debug_accum8(const int8_t* Xq8, int64_t M, int64_t K, const uint8_t* Wq, const uint16_t* zw,
+                                     int64_t N, int32_t group, const uint8_t* A, const int32_t* sal_idx, int32_t r,
+                                     int32_t* acc, int32_t* acc_c, int32_t decode, void* workspace, size_t ws_bytes,
+                                     void* stream) {
+    const uint8_t* X8 = reinterpret_cast<const uint8_t*>(Xq8);
+    hq_status s = check_gemm(X8, M, K, Wq, zw, N, group, A, sal_idx, r);
+    if (s != HQ_OK) return s;
+    if (M == 0 || N == 0) return HQ_OK;
+    if (!acc || (r > 0 && !acc_c)) return HQ_ERR_ARG;
+    if (decode && !small_supported(M, group)) return HQ_ERR_UNSUPPORTED;
+    GemmArgs a{};
+    a.Xq = X8; a.Wq = Wq; a.zw = zw; a.Rq = A; a.sal = sal_idx;
+    a.dbg_acc = acc; a.dbg_acc_c = acc_c;
+    a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
+    a.act_bits = 8;
+    return run_gemm(a, OUT_DEBUG, decode != 0, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+

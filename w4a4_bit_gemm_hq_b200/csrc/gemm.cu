@@ -78,7 +78,7 @@ constexpr uint32_t EPI_BAR = 1;       // named barrier of the epilogue warps
 // bytes each) and a ring of packed slots (PD deep) filled by the copy engine:
 // the 128 activation rows (64 bytes each), the BH weight rows in tile-major
 // order and, for group weights, their BH fp16 zero points of the block's group.
-template <int BN, bool ASYM>
+template <int BN, bool ASYM, bool A8 = false>
 struct PfSmem {
     static constexpr int BH = BN / 2;                                  // weight rows per CTA
     static constexpr int NACC = 512 / BN;                              // accumulator buffers
@@ -87,9 +87,11 @@ struct PfSmem {
     static constexpr int A_BYTES = pf::BM * pf::BK;
     static constexpr int B_BYTES = BH * pf::BK;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NCHUNK = (pf::BM + BH) * 4;                   // 16-byte packed chunks per stage
+    // 16-byte packed chunks per stage the producers expand (8-bit activations
+    // arrive in the int8 stage directly from the copy engine)
+    static constexpr int NCHUNK = ((A8 ? 0 : pf::BM) + BH) * 4;
     static constexpr int NCH = (NCHUNK + pf::NGROUP - 1) / pf::NGROUP;  // per producer thread and stage
-    static constexpr int PK_A = pf::BM * pf::PK_ROW;
+    static constexpr int PK_A = A8 ? 0 : pf::BM * pf::PK_ROW;
     static constexpr int PK_B = BH * pf::PK_ROW;
     static constexpr int PK_Z = ASYM ? BH * 2 : 0;
     static constexpr int PK_STAGE = ((PK_A + PK_B + PK_Z) + 127) / 128 * 128;
@@ -114,15 +116,15 @@ __device__ __forceinline__ uint32_t swz_chunk(int row, int chunk) { return stati
 // pointer) -> int8 operand tiles of the stage.  Chunk ci covers packed bytes
 // [16 ci, 16 ci + 16) of the slot: activation row ci / 4 for ci < 512, else
 // weight row (ci - 512) / 4, K bytes 16 (ci % 4) onwards.
-template <int BN, bool ASYM>
+template <int BN, bool ASYM, bool A8>
 __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, int pi) {
-    using L = PfSmem<BN, ASYM>;
+    using L = PfSmem<BN, ASYM, A8>;
 #pragma unroll
     for (int j = 0; j < L::NCH; ++j) {
         const int ci = pi + j * pf::NGROUP;
         if (ci >= L::NCHUNK) continue;
-        const bool isA = ci < pf::BM * 4;
-        const int cl = isA ? ci : ci - pf::BM * 4;
+        const bool isA = !A8 && ci < pf::BM * 4;
+        const int cl = isA ? ci : ci - (A8 ? 0 : pf::BM * 4);
         const int row = cl >> 2, c = cl & 3;
         const uint4 d = *reinterpret_cast<const uint4*>(pk + ci * 16);
         uint8_t* base = stage + (isA ? 0 : L::A_BYTES) + row * 128;
@@ -137,6 +139,16 @@ __device__ __forceinline__ void prod_unpack(const uint8_t* pk, uint8_t* stage, i
         } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e) unpack_s4x8_times16(w[e], o[2 * e], o[2 * e + 1]);
+        }
+        if constexpr (A8) {
+            // 8-bit activations keep their natural K order: interleave each
+            // (k0 k2 k4 k6, k1 k3 k5 k7) pair of words back to (k0..k3, k4..k7)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t lo = o[2 * e], hi = o[2 * e + 1];
+                o[2 * e] = __byte_perm(lo, hi, 0x5140);
+                o[2 * e + 1] = __byte_perm(lo, hi, 0x7362);
+            }
         }
         *reinterpret_cast<uint4*>(base + swz_chunk(row, 2 * c) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(base + swz_chunk(row, 2 * c + 1) * 16) = make_uint4(o[4], o[5], o[6], o[7]);
@@ -175,10 +187,11 @@ __device__ __forceinline__ void stage_column(const GemmArgs& p, int n, float* sw
 // unpack_s4x8_times16).  This thread writes the blocks i with i % 2 == half
 // (words 2i, 2i+1) of the first `nblk` blocks; blocks past r and rows past M
 // are zero.  All loads of the thread are in flight together.
+template <bool A8>
 __device__ __forceinline__ void gather_xs_smem(const GemmArgs& p, const int32_t* sal_s, int m, uint32_t* xs_w,
                                                int half, int nblk) {
     const bool mv = m < p.M;
-    const uint8_t* row = p.Xq + static_cast<int64_t>(mv ? m : 0) * (p.K / 2);
+    const uint8_t* row = p.Xq + static_cast<int64_t>(mv ? m : 0) * (A8 ? p.K : p.K / 2);
     uint32_t nib[4][8];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
@@ -189,7 +202,8 @@ __device__ __forceinline__ void gather_xs_smem(const GemmArgs& p, const int32_t*
             if (mv && 8 * i < p.r) {
                 const int k = sal_s[8 * i + t];
                 if (static_cast<unsigned>(k) < static_cast<unsigned>(p.K)) {
-                    nib[b][t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
+                    if constexpr (A8) nib[b][t] = __ldg(row + k);   // the 8-bit code itself
+                    else nib[b][t] = (static_cast<uint32_t>(__ldg(row + (k >> 1))) >> ((k & 1) * 4)) & 0xFu;
                 } else {
                     record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
                 }
@@ -203,7 +217,9 @@ __device__ __forceinline__ void gather_xs_smem(const GemmArgs& p, const int32_t*
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            const uint32_t code = (8 * i < p.r) ? static_cast<uint32_t>(static_cast<int>(nib[b][t] ^ 8u) - 8) & 0xFFu : 0u;
+            const uint32_t code = (8 * i >= p.r) ? 0u
+                                  : A8 ? (nib[b][t] & 0xFFu)
+                                       : static_cast<uint32_t>(static_cast<int>(nib[b][t] ^ 8u) - 8) & 0xFFu;
             if (t & 1) hi |= code << (8 * (t >> 1));
             else lo |= code << (8 * (t >> 1));
         }
@@ -232,7 +248,7 @@ __device__ __forceinline__ void store_out2(void* Y, int64_t off, float a, float 
 //  mq0    first output row of the warp;  n0c  first output column of the chunk
 //  scol   column of the chunk within the tile (index into the staged columns)
 //  afr    A fragments [row half][K step] of the warp's X[m,S] rows
-template <int OUT>
+template <int OUT, int AF>
 __device__ __forceinline__ void drain_sym_chunk(const GemmArgs& p, uint32_t tm, int mq0, int n0c, int scol,
                                                 const float* sw_s, const float* sr_s, const uint8_t* rq_s,
                                                 const uint32_t (&afr)[2][2][4], int ksteps, const float (&sxr)[2][2],
@@ -272,8 +288,9 @@ __device__ __forceinline__ void drain_sym_chunk(const GemmArgs& p, uint32_t tm, 
             for (int h = 0; h < 2; ++h) {
                 const int m = mq0 + 16 * mt + g + 8 * h;
                 if (m >= p.M) continue;
-                const int32_t a0 = static_cast<int32_t>(v[4 * nt + 2 * h]) >> 8;
-                const int32_t a1 = static_cast<int32_t>(v[4 * nt + 2 * h + 1]) >> 8;
+                // the weight codes carry 16, the activation codes AF
+                const int32_t a0 = static_cast<int32_t>(v[4 * nt + 2 * h]) >> (AF == 16 ? 8 : 4);
+                const int32_t a1 = static_cast<int32_t>(v[4 * nt + 2 * h + 1]) >> (AF == 16 ? 8 : 4);
                 const int32_t c0 = cc[nt][2 * h] >> 4, c1 = cc[nt][2 * h + 1] >> 4;   // Rq codes carry 16
                 const int64_t off = static_cast<int64_t>(m) * p.N + n;
                 if constexpr (OUT == OUT_DEBUG) {
@@ -297,9 +314,12 @@ __device__ __forceinline__ void drain_sym_chunk(const GemmArgs& p, uint32_t tm, 
 
 // OUT: HQ_F16 / HQ_BF16 / HQ_F32, or OUT_DEBUG for raw accumulators.
 // Launched as clusters of 2 CTAs (an even number of CTAs).
-template <int BN, bool ASYM, int OUT>
+template <int BN, bool ASYM, bool A8, int OUT>
 __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, const __grid_constant__ CUtensorMap tmX) {
-    using L = PfSmem<BN, ASYM>;
+    using L = PfSmem<BN, ASYM, A8>;
+    // factor of the activation codes in the int8 operand (4-bit codes are
+    // expanded as 16 q; 8-bit codes are used as they are)
+    constexpr int AF = A8 ? 1 : 16;
     constexpr int STAGES = L::STAGES;
     constexpr int PD = L::PD;
     constexpr int NACC = L::NACC;
@@ -376,13 +396,23 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 const int m0 = (tile % MT) * 2 * pf::BM + static_cast<int>(crank) * pf::BM;
                 const int nr = (tile / MT) * BN + static_cast<int>(crank) * BH;   // first weight row of this CTA
                 if (!mbar_wait(pkempty_bar(slot), ph ^ 1u, p.limit_ns)) break;
+                const int stg = item % STAGES;
+                if constexpr (A8) {
+                    // the 8-bit activation tile goes straight into the stage: wait
+                    // until the pair's MMAs have finished reading its previous use
+                    if (!mbar_wait_cluster(empty_bar(stg), (static_cast<uint32_t>(item / STAGES) & 1u) ^ 1u, p.limit_ns))
+                        break;
+                }
                 const uint32_t dst = pk0 + slot * L::PK_STAGE;
                 const bool has_b = nr < npad;
                 const int zrows = ASYM ? ((p.N - nr) < BH ? (p.N - nr) : BH) : 0;
                 const int zb = zrows > 0 ? zrows * 2 : 0;
                 mbar_arrive_expect_tx(pkfull_bar(slot),
-                                      static_cast<uint32_t>(L::PK_A + (has_b ? L::PK_B : 0) + zb));
-                tma_load_2d(dst, &tmX, kb * pf::PK_ROW, m0, pkfull_bar(slot));
+                                      static_cast<uint32_t>((A8 ? L::A_BYTES : L::PK_A) + (has_b ? L::PK_B : 0) + zb));
+                if constexpr (A8)   // 128 rows x 128 bytes, 128-byte swizzled: the MMA's K-major layout
+                    tma_load_2d(smem_u32(smem + stg * L::STAGE), &tmX, kb * pf::BK, m0, pkfull_bar(slot));
+                else
+                    tma_load_2d(dst, &tmX, kb * pf::PK_ROW, m0, pkfull_bar(slot));
                 if (has_b)
                     bulk_copy_g2s(dst + L::PK_A, p.Wq + wq_offset(nr, kb * 64, KB), L::PK_B, pkfull_bar(slot));
                 if constexpr (ASYM) {
@@ -416,7 +446,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
             bool ok = mbar_wait(pkfull_bar(slot), ph, p.limit_ns);
             ok = ok && mbar_wait_cluster(empty_bar(stage), phase ^ 1u, p.limit_ns);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
-            prod_unpack<BN, ASYM>(smem + L::OFF_PK + slot * L::PK_STAGE, smem + stage * L::STAGE, pi);
+            prod_unpack<BN, ASYM, A8>(smem + L::OFF_PK + slot * L::PK_STAGE, smem + stage * L::STAGE, pi);
             fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
             __syncwarp();
             if (lane == 0) {
@@ -499,7 +529,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);   // previous tile's readers are done
                 if (et < BN) stage_column<OUT>(p, n0 + et, sw_s + et, sr_s + et, rq_s + et * pf::RQ_LD);
                 if (p.r > 0)
-                    gather_xs_smem(p, sal_s, m0 + row,
+                    gather_xs_smem<A8>(p, sal_s, m0 + row,
                                    reinterpret_cast<uint32_t*>(smem + L::OFF_XS + row * pf::RQ_LD), hcol, 4 * ksteps);
                 float sxr[2][2];
 #pragma unroll
@@ -531,7 +561,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                     for (int c = 0; c < BN / 2 / 32; ++c) {
                         const int col = hcol * (BN / 2) + c * 32;
                         if (n0 + col >= p.N) break;
-                        drain_sym_chunk<OUT>(p,
+                        drain_sym_chunk<OUT, AF>(p,
                                              tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                                                  static_cast<uint32_t>(abuf * BN + col),
                                              mq0, n0 + col, col, sw_s, sr_s, rq_s, afr, ksteps, sxr, g8, t4);
@@ -582,7 +612,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                 named_bar_sync(pf::EPI_BAR, pf::EPI_THREADS);   // previous tile's readers are done
                 if (et < BN) stage_column<OUT>(p, n0 + et, sw_s + et, sr_s + et, rq_s + et * pf::RQ_LD);
                 if (p.r > 0)
-                    gather_xs_smem(p, sal_s, m0 + row,
+                    gather_xs_smem<A8>(p, sal_s, m0 + row,
                                    reinterpret_cast<uint32_t*>(smem + L::OFF_XS + row * pf::RQ_LD), hcol, 4 * ksteps);
                 float sxr[2][2];
 #pragma unroll
@@ -636,14 +666,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                                 const int cl = scol + 8 * nt + 2 * t4;
 #pragma unroll
                                 for (int h = 0; h < 2; ++h) {
-                                    // the Rq codes carry a factor 16, like yp until the end of the tile
-                                    const int32_t c0 = cc[nt][2 * h], c1 = cc[nt][2 * h + 1];
+                                    // the Rq codes carry a factor 16; yp carries AF (the factor of
+                                    // the activation codes) until the end of the tile
+                                    const int32_t c0 = AF == 16 ? cc[nt][2 * h] : cc[nt][2 * h] >> 4;
+                                    const int32_t c1 = AF == 16 ? cc[nt][2 * h + 1] : cc[nt][2 * h + 1] >> 4;
                                     if constexpr (OUT == OUT_DEBUG) {
                                         const int m = mq0 + 16 * mt + g8 + 8 * h;
                                         const int n = n0 + cl;
                                         if (p.r > 0 && m < p.M && n < p.N) {
-                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n] = c0 >> 4;
-                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n + 1] = c1 >> 4;
+                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n] = AF == 16 ? c0 >> 4 : c0;
+                                            p.dbg_acc_c[static_cast<int64_t>(m) * p.N + n + 1] = AF == 16 ? c1 >> 4 : c1;
                                         }
                                         yp[c][mt][nt][h] = make_float2(0.f, 0.f);
                                     } else {
@@ -712,11 +744,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                                             const int n = n0 + scol + 8 * nt + 2 * t4;
                                             if (m < p.M && n < p.N) {
                                                 const int64_t o = (static_cast<int64_t>(m) * p.N + n) * NG + g;
-                                                p.dbg_acc[o] = static_cast<int32_t>(v[4 * nt + 2 * h] - MAGIC) >> 4;
-                                                p.dbg_acc[o + NG] = static_cast<int32_t>(v[4 * nt + 2 * h + 1] - MAGIC) >> 4;
+                                                p.dbg_acc[o] = static_cast<int32_t>(v[4 * nt + 2 * h] - MAGIC) / AF;
+                                                p.dbg_acc[o + NG] = static_cast<int32_t>(v[4 * nt + 2 * h + 1] - MAGIC) / AF;
                                             }
                                         } else {
-                                            // f - 1.5 * 2^23 = 16 acc exactly; yp += sw (16 acc)
+                                            // f - 1.5 * 2^23 = AF acc exactly; yp += sw (AF acc)
                                             yp[c][mt][nt][h] = __ffma2_rn(swf[nt], __fadd2_rn(f, make_float2(-cmag.x, -cmag.y)),
                                                                           yp[c][mt][nt][h]);
                                         }
@@ -749,10 +781,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1) k_gemm_pf(const GemmArgs p, co
                                     for (int h = 0; h < 2; ++h) {
                                         const int m = mq0 + 16 * mt + g8 + 8 * h;
                                         if (m >= p.M) continue;
-                                        // yp / 16 is exact: the same bits as accumulating sw * acc
+                                        // yp / AF is exact: the same bits as accumulating sw * acc
+                                        constexpr float inv_af = 1.0f / AF;
                                         store_out2<OUT>(p.Y, static_cast<int64_t>(m) * p.N + n,
-                                                        __fmul_rn(sxr[mt][h], __fmul_rn(yp[c][mt][nt][h].x, 0.0625f)),
-                                                        __fmul_rn(sxr[mt][h], __fmul_rn(yp[c][mt][nt][h].y, 0.0625f)));
+                                                        __fmul_rn(sxr[mt][h], __fmul_rn(yp[c][mt][nt][h].x, inv_af)),
+                                                        __fmul_rn(sxr[mt][h], __fmul_rn(yp[c][mt][nt][h].y, inv_af)));
                                     }
                                 }
                     }
@@ -790,27 +823,32 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 
 // Tensor map of the packed activations Xq[M][K/2] (bytes): boxes of 64 bytes x
 // 128 rows, rows past M filled with zero.
-static hq_status xq_tensor_map(const GemmArgs& a, CUtensorMap* map) {
+static hq_status xq_tensor_map(const GemmArgs& a, CUtensorMap* map, bool a8) {
     const auto encode = encode_tiled();
     if (!encode) return HQ_ERR_CUDA;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 2), static_cast<cuuint64_t>(a.M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 2)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::PK_ROW), static_cast<cuuint32_t>(pf::BM)};
+    // 4-bit codes: boxes of 64 packed bytes x 128 rows into the packed ring;
+    // 8-bit codes: boxes of 128 bytes x 128 rows, 128-byte swizzled, straight
+    // into the MMA's operand stage.  Rows past M read as zero.
+    const cuuint64_t row = static_cast<cuuint64_t>(a8 ? a.K : a.K / 2);
+    const cuuint64_t dims[2] = {row, static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t strides[1] = {row};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(a8 ? pf::BK : pf::PK_ROW), static_cast<cuuint32_t>(pf::BM)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.Xq), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              a8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
 }
 
-template <int BN, bool ASYM, int OUT>
+template <int BN, bool ASYM, bool A8, int OUT>
 static hq_status launch_pf_t(const GemmArgs& a, cudaStream_t st, int nsm) {
-    auto kern = k_gemm_pf<BN, ASYM, OUT>;
-    const int smem = PfSmem<BN, ASYM>::ALLOC;
+    auto kern = k_gemm_pf<BN, ASYM, A8, OUT>;
+    const int smem = PfSmem<BN, ASYM, A8>::ALLOC;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
     CUtensorMap tmX;
-    const hq_status s = xq_tensor_map(a, &tmX);
+    const hq_status s = xq_tensor_map(a, &tmX, A8);
     if (s != HQ_OK) return s;
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
@@ -843,23 +881,28 @@ static hq_status launch_pf_t(const GemmArgs& a, cudaStream_t st, int nsm) {
     if (cudaLaunchKernelEx(&cfg, kern, a, tmX) != cudaSuccess) return HQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
-hq_status launch_gemm_prefill(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
+template <bool A8>
+static hq_status launch_pf_a(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
     if (a.gw == 0) {
         switch (out) {
-            case HQ_F16: return launch_pf_t<256, false, HQ_F16>(a, st, nsm);
-            case HQ_BF16: return launch_pf_t<256, false, HQ_BF16>(a, st, nsm);
-            case HQ_F32: return launch_pf_t<256, false, HQ_F32>(a, st, nsm);
-            case OUT_DEBUG: return launch_pf_t<256, false, OUT_DEBUG>(a, st, nsm);
+            case HQ_F16: return launch_pf_t<256, false, A8, HQ_F16>(a, st, nsm);
+            case HQ_BF16: return launch_pf_t<256, false, A8, HQ_BF16>(a, st, nsm);
+            case HQ_F32: return launch_pf_t<256, false, A8, HQ_F32>(a, st, nsm);
+            case OUT_DEBUG: return launch_pf_t<256, false, A8, OUT_DEBUG>(a, st, nsm);
         }
     } else {
         switch (out) {
-            case HQ_F16: return launch_pf_t<128, true, HQ_F16>(a, st, nsm);
-            case HQ_BF16: return launch_pf_t<128, true, HQ_BF16>(a, st, nsm);
-            case HQ_F32: return launch_pf_t<128, true, HQ_F32>(a, st, nsm);
-            case OUT_DEBUG: return launch_pf_t<128, true, OUT_DEBUG>(a, st, nsm);
+            case HQ_F16: return launch_pf_t<128, true, A8, HQ_F16>(a, st, nsm);
+            case HQ_BF16: return launch_pf_t<128, true, A8, HQ_BF16>(a, st, nsm);
+            case HQ_F32: return launch_pf_t<128, true, A8, HQ_F32>(a, st, nsm);
+            case OUT_DEBUG: return launch_pf_t<128, true, A8, OUT_DEBUG>(a, st, nsm);
         }
     }
     return HQ_ERR_UNSUPPORTED;
+}
+
+hq_status launch_gemm_prefill(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
+    return a.act_bits == 8 ? launch_pf_a<true>(a, out, st, nsm) : launch_pf_a<false>(a, out, st, nsm);
 }
 
 }  // namespace hq

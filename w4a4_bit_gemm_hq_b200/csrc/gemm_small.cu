@@ -142,9 +142,12 @@ __device__ __forceinline__ void ld_cols(uint32_t taddr, uint32_t (&v)[NT]) {
     }
 }
 
-template <int NT, bool ASYM, int OUT>
+// A8: 8-bit activation codes ([M][K] int8, used as they are) instead of packed
+// 4-bit codes (expanded as 16 q).
+template <int NT, bool ASYM, bool A8, int OUT>
 __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p, const SkPlan plan) {
     using L = SkSmem<NT>;
+    constexpr int XROW = A8 ? 128 : 64;   // activation bytes per token row and K-block
     constexpr int SB = L::SB;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, derived by pointer arithmetic on the __shared__
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
         // the unit's tokens into the set's token stage.
         const int pset = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
-        constexpr int TCH = (NT * 4 + 127) / 128;   // token chunks per thread per K-block
+        constexpr int TCH = (NT * (XROW / 16) + 127) / 128;   // token chunks per thread per K-block
         // write cursor (cp.async issue) over this set's K-blocks
         int wli = pset, wkbi = 0, wctr = 0;
         auto issue_next = [&]() {
@@ -251,10 +254,10 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
 #pragma unroll
                 for (int c = 0; c < TCH; ++c) {
                     const int tc = row + 128 * c;
-                    const int tr = tc >> 2, ch = tc & 3;
-                    if (kbi < nk && tc < NT * 4 && tr < p.M)
-                        tk[kbi][c] = __ldg(reinterpret_cast<const uint4*>(p.Xq + static_cast<int64_t>(tr) * (p.K / 2) +
-                                                                       (kb0 + kbi) * 64 + ch * 16));
+                    const int tr = tc / (XROW / 16), ch = tc % (XROW / 16);
+                    if (kbi < nk && tc < NT * (XROW / 16) && tr < p.M)
+                        tk[kbi][c] = __ldg(reinterpret_cast<const uint4*>(p.Xq + static_cast<int64_t>(tr) * (A8 ? p.K : p.K / 2) +
+                                                                       (kb0 + kbi) * XROW + ch * 16));
                 }
             }
         };
@@ -303,6 +306,13 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
                     for (int e = 0; e < 4; ++e) {
                         if constexpr (ASYM) unpack_u4x8_minus_z(w[e], z4, a[8 * c + 2 * e], a[8 * c + 2 * e + 1]);
                         else unpack_s4x8_times16(w[e], a[8 * c + 2 * e], a[8 * c + 2 * e + 1]);
+                        if constexpr (A8) {
+                            // 8-bit activations keep their natural K order: interleave the
+                            // (k0 k2 k4 k6, k1 k3 k5 k7) words back to (k0..k3, k4..k7)
+                            const uint32_t lo = a[8 * c + 2 * e], hi = a[8 * c + 2 * e + 1];
+                            a[8 * c + 2 * e] = __byte_perm(lo, hi, 0x5140);
+                            a[8 * c + 2 * e + 1] = __byte_perm(lo, hi, 0x7362);
+                        }
                     }
                 }
                 tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
@@ -311,16 +321,21 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
 #pragma unroll
                 for (int c = 0; c < TCH; ++c) {
                     const int tc = row + 128 * c;
-                    if (tc < NT * 4) {
-                        const int tr = tc >> 2, ch = tc & 3;
-                        uint32_t o[8];
-                        const uint32_t w[4] = {tk_cur[kbi][c].x, tk_cur[kbi][c].y, tk_cur[kbi][c].z, tk_cur[kbi][c].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) unpack_s4x8_times16(w[e], o[2 * e], o[2 * e + 1]);
+                    if (tc < NT * (XROW / 16)) {
+                        const int tr = tc / (XROW / 16), ch = tc % (XROW / 16);
                         uint8_t* trow = tstage + tr * 128;
-                        *reinterpret_cast<uint4*>(trow + (((2 * ch) ^ (tr & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                        *reinterpret_cast<uint4*>(trow + (((2 * ch + 1) ^ (tr & 7)) << 4)) =
-                            make_uint4(o[4], o[5], o[6], o[7]);
+                        if constexpr (A8) {
+                            // 16 codes as they are, into 16-byte chunk ch of the swizzled row
+                            *reinterpret_cast<uint4*>(trow + ((ch ^ (tr & 7)) << 4)) = tk_cur[kbi][c];
+                        } else {
+                            uint32_t o[8];
+                            const uint32_t w[4] = {tk_cur[kbi][c].x, tk_cur[kbi][c].y, tk_cur[kbi][c].z, tk_cur[kbi][c].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) unpack_s4x8_times16(w[e], o[2 * e], o[2 * e + 1]);
+                            *reinterpret_cast<uint4*>(trow + (((2 * ch) ^ (tr & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                            *reinterpret_cast<uint4*>(trow + (((2 * ch + 1) ^ (tr & 7)) << 4)) =
+                                make_uint4(o[4], o[5], o[6], o[7]);
+                        }
                     }
                 }
             }
@@ -415,7 +430,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
             const int m = idx / sk::XS_WORDS, w = idx % sk::XS_WORDS;
             uint32_t word = 0;
             if (m < p.M) {
-                const uint8_t* xrow = p.Xq + static_cast<int64_t>(m) * (p.K / 2);
+                const uint8_t* xrow = p.Xq + static_cast<int64_t>(m) * (A8 ? p.K : p.K / 2);
                 const int i = w >> 1, h = w & 1;   // word 2i+h holds positions 8i+2e+h, byte e
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -423,8 +438,12 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
                     if (j < p.r) {
                         const int k = sal_s[j];
                         if (static_cast<unsigned>(k) < static_cast<unsigned>(p.K)) {
-                            const int nib = (__ldg(xrow + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
-                            word |= (static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu) << (8 * e);
+                            if constexpr (A8) {
+                                word |= static_cast<uint32_t>(__ldg(xrow + k)) << (8 * e);
+                            } else {
+                                const int nib = (__ldg(xrow + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
+                                word |= (static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu) << (8 * e);
+                            }
                         } else {
                             record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
                         }
@@ -439,7 +458,9 @@ __global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p,
         uint32_t accph = 0;
         uint32_t* ws_cnt = static_cast<uint32_t*>(p.ws);
         float* ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(p.ws) + small_counter_bytes(plan.ntiles));
-        const int sh = ASYM ? 4 : 8;
+        // the accumulators carry the factor of the activation codes (16 for
+        // 4-bit codes, 1 for 8-bit) and 16 for symmetric weight codes
+        const int sh = (A8 ? 0 : 4) + (ASYM ? 0 : 4);
         const int G = ASYM ? p.K / p.gw : 1;
         int li = 0;
         while (li < nunits) {
@@ -612,9 +633,9 @@ size_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int gw, int nsm) {
     return small_counter_bytes(p.ntiles) + static_cast<size_t>(p.ntiles) * p.maxc * nt_for(M) * sk::BMW * sizeof(float);
 }
 
-template <int NT, bool ASYM, int OUT>
+template <int NT, bool ASYM, bool A8, int OUT>
 static hq_status launch_sk_t(const GemmArgs& a, const SkPlan& plan, cudaStream_t st) {
-    auto kern = k_gemm_small<NT, ASYM, OUT>;
+    auto kern = k_gemm_small<NT, ASYM, A8, OUT>;
     const int smem = SkSmem<NT>::ALLOC;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
@@ -636,21 +657,21 @@ static hq_status launch_sk_t(const GemmArgs& a, const SkPlan& plan, cudaStream_t
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
-template <int NT>
+template <int NT, bool A8>
 static hq_status launch_sk_nt(const GemmArgs& a, int out, const SkPlan& plan, cudaStream_t st) {
     if (a.gw == 0) {
         switch (out) {
-            case HQ_F16: return launch_sk_t<NT, false, HQ_F16>(a, plan, st);
-            case HQ_BF16: return launch_sk_t<NT, false, HQ_BF16>(a, plan, st);
-            case HQ_F32: return launch_sk_t<NT, false, HQ_F32>(a, plan, st);
-            case OUT_DEBUG: return launch_sk_t<NT, false, OUT_DEBUG>(a, plan, st);
+            case HQ_F16: return launch_sk_t<NT, false, A8, HQ_F16>(a, plan, st);
+            case HQ_BF16: return launch_sk_t<NT, false, A8, HQ_BF16>(a, plan, st);
+            case HQ_F32: return launch_sk_t<NT, false, A8, HQ_F32>(a, plan, st);
+            case OUT_DEBUG: return launch_sk_t<NT, false, A8, OUT_DEBUG>(a, plan, st);
         }
     } else {
         switch (out) {
-            case HQ_F16: return launch_sk_t<NT, true, HQ_F16>(a, plan, st);
-            case HQ_BF16: return launch_sk_t<NT, true, HQ_BF16>(a, plan, st);
-            case HQ_F32: return launch_sk_t<NT, true, HQ_F32>(a, plan, st);
-            case OUT_DEBUG: return launch_sk_t<NT, true, OUT_DEBUG>(a, plan, st);
+            case HQ_F16: return launch_sk_t<NT, true, A8, HQ_F16>(a, plan, st);
+            case HQ_BF16: return launch_sk_t<NT, true, A8, HQ_BF16>(a, plan, st);
+            case HQ_F32: return launch_sk_t<NT, true, A8, HQ_F32>(a, plan, st);
+            case OUT_DEBUG: return launch_sk_t<NT, true, A8, OUT_DEBUG>(a, plan, st);
         }
     }
     return HQ_ERR_UNSUPPORTED;
@@ -659,10 +680,11 @@ static hq_status launch_sk_nt(const GemmArgs& a, int out, const SkPlan& plan, cu
 hq_status launch_gemm_small(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
     if (!small_supported(a.M, a.gw)) return HQ_ERR_UNSUPPORTED;
     const SkPlan plan = sk_plan(a.M, a.N, a.K, a.gw, nsm);
+    const bool a8 = a.act_bits == 8;
     switch (nt_for(a.M)) {
-        case 16: return launch_sk_nt<16>(a, out, plan, st);
-        case 32: return launch_sk_nt<32>(a, out, plan, st);
-        default: return launch_sk_nt<64>(a, out, plan, st);
+        case 16: return a8 ? launch_sk_nt<16, true>(a, out, plan, st) : launch_sk_nt<16, false>(a, out, plan, st);
+        case 32: return a8 ? launch_sk_nt<32, true>(a, out, plan, st) : launch_sk_nt<32, false>(a, out, plan, st);
+        default: return a8 ? launch_sk_nt<64, true>(a, out, plan, st) : launch_sk_nt<64, false>(a, out, plan, st);
     }
 }
 

@@ -11,7 +11,7 @@ namespace hq {
 constexpr int OUT_DEBUG = 3;  // epilogue variant that stores raw integer accumulators
 
 struct GemmArgs {
-    const uint8_t* Xq;      // [M][K/2] packed activation codes
+    const uint8_t* Xq;      // [M][K/2] packed activation codes ([M][K] int8 when act_bits == 8)
     const float* sx;        // [M]
     const uint8_t* Wq;      // [N][K/2] packed weight codes
     const uint16_t* sw;     // fp16 bits, [N] or [K/gw][N]
@@ -24,6 +24,7 @@ struct GemmArgs {
     int32_t* dbg_acc_c;     // [M][N]    (debug epilogue)
     void* ws;               // scratch (small-M kernel)
     int M, N, K, gw, r;
+    int act_bits;           // 4: Xq packed int4 [M][K/2]; 8: Xq int8 codes [M][K] (W4A8)
     uint64_t limit_ns;      // bounded-wait limit
 };
 

@@ -26,7 +26,7 @@ namespace hq {
 
 constexpr int EPT = 32;  // channels per thread
 
-enum { MODE_QUANT = 0, MODE_ROTATE = 1, MODE_SQNORM = 2 };
+enum { MODE_QUANT = 0, MODE_ROTATE = 1, MODE_SQNORM = 2, MODE_QUANT8 = 3 };   // QUANT8: one 8-bit code per byte
 enum { XT_F16 = 0, XT_BF16 = 1, XT_F32 = 2 };
 
 __device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
@@ -263,9 +263,10 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
 #pragma unroll
                     for (int e = 0; e < 8; ++e) accsq[8 * ah + e] = __fmaf_rn(w[ah][e], w[ah][e], accsq[8 * ah + e]);
             }
-            if constexpr (MODE != MODE_QUANT) {
+            if constexpr (MODE != MODE_QUANT && MODE != MODE_QUANT8) {
                 __syncthreads();   // the next row rewrites the cross-warp buffer
             } else {
+                constexpr float LEVELS = MODE == MODE_QUANT8 ? 127.0f : 7.0f;
                 float amax = 0.f;
 #pragma unroll
                 for (int ah = 0; ah < 4; ++ah)
@@ -279,8 +280,22 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 amax = 0.f;
                 for (int wi = 0; wi < nw; ++wi) amax = fmaxf(amax, red[par][wi]);
                 uint32_t words[4] = {0u, 0u, 0u, 0u};
-                if (amax != 0.f) {
-                    const float inv = __fdiv_rn(7.0f, amax);
+                uint32_t bytes[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
+                if (amax != 0.f && MODE == MODE_QUANT8) {
+                    const float inv = __fdiv_rn(LEVELS, amax);
+                    const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+#pragma unroll
+                    for (int ah = 0; ah < 4; ++ah)
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            // the low byte of the sum's bits is the code in two's complement
+                            const float2 tq = make_float2(__fmul_rn(w[ah][e], inv), __fmul_rn(w[ah][e + 1], inv));
+                            const float2 r = f2add_rn(tq, magic);
+                            bytes[ah][e >> 2] |= ((__float_as_uint(r.x) & 0xFFu) | ((__float_as_uint(r.y) & 0xFFu) << 8))
+                                                 << (8 * (e & 2));
+                        }
+                } else if (amax != 0.f) {
+                    const float inv = __fdiv_rn(LEVELS, amax);
                     const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
 #pragma unroll
                     for (int ah = 0; ah < 4; ++ah) {
@@ -296,11 +311,18 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                         words[ah] = wd;
                     }
                 }
-                uint8_t* qrow = Xq + m * (K / 2);
+                if constexpr (MODE == MODE_QUANT8) {
+                    uint8_t* qrow = Xq + m * K;
 #pragma unroll
-                for (int ah = 0; ah < 4; ++ah)
-                    *reinterpret_cast<uint32_t*>(qrow + (grp0 + 1024 * ah) / 2) = words[ah];
-                if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+                    for (int ah = 0; ah < 4; ++ah)
+                        *reinterpret_cast<uint2*>(qrow + grp0 + 1024 * ah) = make_uint2(bytes[ah][0], bytes[ah][1]);
+                } else {
+                    uint8_t* qrow = Xq + m * (K / 2);
+#pragma unroll
+                    for (int ah = 0; ah < 4; ++ah)
+                        *reinterpret_cast<uint32_t*>(qrow + (grp0 + 1024 * ah) / 2) = words[ah];
+                }
+                if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, LEVELS), cg);
             }
         } else {
             // ---- shuffle stages: partner thread t ^ s holds channels +-32s
@@ -352,6 +374,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                     accsq[2 * i + 1] = __fmaf_rn(v[i].y, v[i].y, accsq[2 * i + 1]);
                 }
             } else {
+                constexpr float LEVELS = MODE == MODE_QUANT8 ? 127.0f : 7.0f;
                 // ---- per-token absmax over the whole row
                 float amax = 0.f;
     #pragma unroll
@@ -370,11 +393,28 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 }
                 // ---- scale, round half to even, pack
                 uint32_t words[EPT / 8];
+                uint32_t bytes[EPT / 4];
+    #pragma unroll
+                for (int j = 0; j < EPT / 4; ++j) bytes[j] = 0u;
                 if (amax == 0.f) {
     #pragma unroll
                     for (int j = 0; j < EPT / 8; ++j) words[j] = 0u;
+                } else if (MODE == MODE_QUANT8) {
+                    const float inv = __fdiv_rn(LEVELS, amax);
+                    const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    #pragma unroll
+                    for (int j = 0; j < EPT / 4; ++j) {
+                        // channels 4j .. 4j+3: the low byte of each sum's bits is its code
+                        const float2 t0 = make_float2(__fmul_rn(v[2 * j].x, inv), __fmul_rn(v[2 * j].y, inv));
+                        const float2 t1 = make_float2(__fmul_rn(v[2 * j + 1].x, inv), __fmul_rn(v[2 * j + 1].y, inv));
+                        const float2 r0 = f2add_rn(t0, magic), r1 = f2add_rn(t1, magic);
+                        bytes[j] = __byte_perm(__byte_perm(__float_as_uint(r0.x), __float_as_uint(r0.y), 0x0040),
+                                               __byte_perm(__float_as_uint(r1.x), __float_as_uint(r1.y), 0x0040), 0x5410);
+                    }
+    #pragma unroll
+                    for (int j = 0; j < EPT / 8; ++j) words[j] = 0u;
                 } else {
-                    const float inv = __fdiv_rn(7.0f, amax);
+                    const float inv = __fdiv_rn(LEVELS, amax);
                     const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
     #pragma unroll
                     for (int j = 0; j < EPT / 8; ++j) {
@@ -396,10 +436,16 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                     }
                 }
                 if (active) {
-                    uint4* dst = reinterpret_cast<uint4*>(Xq + m * (K / 2) + col0 / 2);
-                    *dst = make_uint4(words[0], words[1], words[2], words[3]);
+                    if constexpr (MODE == MODE_QUANT8) {
+                        uint4* dst = reinterpret_cast<uint4*>(Xq + m * K + col0);
+                        dst[0] = make_uint4(bytes[0], bytes[1], bytes[2], bytes[3]);
+                        dst[1] = make_uint4(bytes[4], bytes[5], bytes[6], bytes[7]);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(Xq + m * (K / 2) + col0 / 2);
+                        *dst = make_uint4(words[0], words[1], words[2], words[3]);
+                    }
                 }
-                if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+                if (t == 0) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, LEVELS), cg);
             }
         }
 #pragma unroll
@@ -469,7 +515,7 @@ static hq_status launch_rotate(int xt, int group, const void* X, int64_t M, int6
                                uint8_t* Xq, float* sx, float* out, cudaStream_t st) {
     if (xt == HQ_F16) return launch_g<XT_F16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
     if (xt == HQ_BF16) return launch_g<XT_BF16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
-    if constexpr (MODE != MODE_QUANT) {
+    if constexpr (MODE != MODE_QUANT && MODE != MODE_QUANT8) {
         if (xt == HQ_F32) return launch_g<XT_F32, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
     }
     return HQ_ERR_UNSUPPORTED;
@@ -479,7 +525,8 @@ static hq_status launch_rotate(int xt, int group, const void* X, int64_t M, int6
 // 128 channels (up to 16384); other shapes use k_rotate above.
 bool rotq_supported(int64_t M, int64_t K, int group);
 hq_status launch_rotate_quant_stream(int xt, int group, const void* X, int64_t M, int64_t K, int64_t ldx,
-                                     const int8_t* d, uint8_t* Xq, float* sx, cudaStream_t st, uint64_t limit_ns);
+                                     const int8_t* d, uint8_t* Xq, float* sx, cudaStream_t st, uint64_t limit_ns,
+                                     int bits);
 
 static bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -508,9 +555,26 @@ extern "C" hq_status hq_rotate_quant(const void* X, hq_dtype xt, int64_t M, int6
     if (!al16(X) || !al16(Xq) || (ld_x * 2) % 16 != 0) return HQ_ERR_ALIGN;
     if (rotq_supported(M, K, group))
         return launch_rotate_quant_stream(xt, group, X, M, K, ld_x, H_signs, Xq, sx, static_cast<cudaStream_t>(stream),
-                                          2000000000ull);
+                                          2000000000ull, 4);
     return launch_rotate<MODE_QUANT>(xt, group, X, M, K, ld_x, H_signs, Xq, sx, nullptr,
                                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hq_status hq_rotate_quant8(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x, int32_t group,
+                                      const int8_t* H_signs, int8_t* Xq8, float* sx, void* stream) {
+    hq_status s = check_rotate_args(xt, M, K, group);
+    if (s != HQ_OK) return s;
+    if (xt == HQ_F32) return HQ_ERR_UNSUPPORTED;
+    if (ld_x < K) return HQ_ERR_ARG;
+    if (M == 0) return HQ_OK;
+    if (!X || !Xq8 || !sx) return HQ_ERR_ARG;
+    if (!al16(X) || !al16(Xq8) || (ld_x * 2) % 16 != 0) return HQ_ERR_ALIGN;
+    uint8_t* q = reinterpret_cast<uint8_t*>(Xq8);
+    if (rotq_supported(M, K, group))
+        return launch_rotate_quant_stream(xt, group, X, M, K, ld_x, H_signs, q, sx, static_cast<cudaStream_t>(stream),
+                                          2000000000ull, 8);
+    return launch_rotate<MODE_QUANT8>(xt, group, X, M, K, ld_x, H_signs, q, sx, nullptr,
+                                      static_cast<cudaStream_t>(stream));
 }
 
 extern "C" hq_status hq_rotate(const void* X, hq_dtype xt, int64_t M, int64_t K, int32_t group,

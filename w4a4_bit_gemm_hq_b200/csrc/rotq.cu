@@ -127,8 +127,10 @@ __host__ __device__ inline RqLayout rq_layout(int K, int teams, int npat) {
     return L;
 }
 
-// G: Hadamard group; XT: 16-bit input type; SIGNED: d given (else d = 1).
-template <int G, int XT, bool SIGNED>
+// G: Hadamard group; XT: 16-bit input type; SIGNED: d given (else d = 1);
+// Q8: 8-bit codes in [-127, 127], one per byte (the W4A8 activations), else
+// 4-bit codes in [-7, 7], two per byte.
+template <int G, int XT, bool SIGNED, bool Q8>
 __global__ void __launch_bounds__(rq::THREADS, 1)
     k_rotq(const __grid_constant__ CUtensorMap tmX, const int8_t* __restrict__ dsign, int M, int K,
            uint8_t* __restrict__ Xq, float* __restrict__ sx, float cg, int team_warps, int teams,
@@ -204,7 +206,9 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
         prefetch_tmap(&tmX);
         for (; issued < rq::DEPTH && issued < nrows; ++issued) issue(issued);
     }
-    const float2 mg = make_float2(12582920.0f, 12582920.0f);   // 1.5 * 2^23 + 8
+    // 1.5 * 2^23 (+ 8 for 4-bit codes: 8 + q then sits in the low nibble)
+    const float2 mg = Q8 ? make_float2(12582912.0f, 12582912.0f) : make_float2(12582920.0f, 12582920.0f);
+    constexpr float LEVELS = Q8 ? 127.0f : 7.0f;
     int k = 0;
     for (; k < nrows; ++k) {
         const int m = r0 + team + teams * k;
@@ -375,8 +379,31 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
         if (abort_now) break;
 
         // ---- scale, round half to even, pack, store
-        const float inv = amax == 0.f ? 0.f : __fdiv_rn(7.0f, amax);   // amax == 0: every code is 0
-        if constexpr (T == 32) {
+        const float inv = amax == 0.f ? 0.f : __fdiv_rn(LEVELS, amax);   // amax == 0: every code is 0
+        if constexpr (Q8) {
+            // the low byte of fl32(fl32(u * inv) + 1.5 * 2^23) is q in two's complement
+            auto b4 = [&](float2 x0, float2 x1) {
+                const float2 r0 = rq_add2(make_float2(__fmul_rn(x0.x, inv), __fmul_rn(x0.y, inv)), mg);
+                const float2 r1 = rq_add2(make_float2(__fmul_rn(x1.x, inv), __fmul_rn(x1.y, inv)), mg);
+                return __byte_perm(__byte_perm(__float_as_uint(r0.x), __float_as_uint(r0.y), 0x0040),
+                                   __byte_perm(__float_as_uint(r1.x), __float_as_uint(r1.y), 0x0040), 0x5410);
+            };
+            if (act) {
+                if constexpr (T == 32) {
+                    // lane l: channels 128 a + 4 l .. + 3 of the warp's group, 4 bytes per a
+                    uint32_t* dst = reinterpret_cast<uint32_t*>(Xq + static_cast<int64_t>(m) * K + 4096 * wt) + lane;
+#pragma unroll
+                    for (int a = 0; a < 32; ++a) dst[32 * a] = b4(wq[0][a], wq[1][a]);
+                } else {
+                    // 128 bytes per thread, 16 at a time
+                    uint4* dst = reinterpret_cast<uint4*>(Xq + static_cast<int64_t>(m) * K + 128 * u);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_uint4(b4(v[8 * q], v[8 * q + 1]), b4(v[8 * q + 2], v[8 * q + 3]),
+                                            b4(v[8 * q + 4], v[8 * q + 5]), b4(v[8 * q + 6], v[8 * q + 7]));
+                }
+            }
+        } else if constexpr (T == 32) {
             // lane l: 2 bytes (channels 128 a + 4 l .. + 3) per a, 64 contiguous bytes per warp store
             if (act) {
                 uint16_t* dst = reinterpret_cast<uint16_t*>(Xq + static_cast<int64_t>(m) * (K / 2) + 2048 * wt) + lane;
@@ -417,7 +444,7 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
                 }
             }
         }
-        if (leader) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, 7.0f), cg);
+        if (leader) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, LEVELS), cg);
     }
     // no copy may still be landing when the CTA exits (immediate unless a
     // wait gave up): the rows issued but not consumed
@@ -472,40 +499,41 @@ bool rotq_supported(int64_t M, int64_t K, int group) {
     return rq_plan(M, K, group, 148, &p);
 }
 
-template <int G, int XT, bool SIGNED>
+template <int G, int XT, bool SIGNED, bool Q8>
 static hq_status launch_rotq_t(const CUtensorMap& tm, const RqPlan& p, const int8_t* d, int M, int K, uint8_t* Xq,
                                float* sx, float cg, uint64_t limit_ns, cudaStream_t st) {
-    auto kern = k_rotq<G, XT, SIGNED>;
+    auto kern = k_rotq<G, XT, SIGNED, Q8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) != cudaSuccess)
         return HQ_ERR_CUDA;
     kern<<<p.grid, rq::THREADS, p.smem, st>>>(tm, d, M, K, Xq, sx, cg, p.team_warps, p.teams, limit_ns);
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
-template <int XT, bool SIGNED>
+template <int XT, bool SIGNED, bool Q8>
 static hq_status launch_rotq_g(int group, const CUtensorMap& tm, const RqPlan& p, const int8_t* d, int M, int K,
                                uint8_t* Xq, float* sx, float cg, uint64_t limit_ns, cudaStream_t st) {
     switch (group) {
-        case 8: return launch_rotq_t<8, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 16: return launch_rotq_t<16, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 32: return launch_rotq_t<32, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 64: return launch_rotq_t<64, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 128: return launch_rotq_t<128, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 256: return launch_rotq_t<256, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 512: return launch_rotq_t<512, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 1024: return launch_rotq_t<1024, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 2048: return launch_rotq_t<2048, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
-        case 4096: return launch_rotq_t<4096, XT, SIGNED>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 8: return launch_rotq_t<8, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 16: return launch_rotq_t<16, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 32: return launch_rotq_t<32, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 64: return launch_rotq_t<64, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 128: return launch_rotq_t<128, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 256: return launch_rotq_t<256, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 512: return launch_rotq_t<512, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 1024: return launch_rotq_t<1024, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 2048: return launch_rotq_t<2048, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
+        case 4096: return launch_rotq_t<4096, XT, SIGNED, Q8>(tm, p, d, M, K, Xq, sx, cg, limit_ns, st);
         default: return HQ_ERR_UNSUPPORTED;
     }
 }
 
 // Caller has validated the arguments (16-bit type, power-of-two group in
 // [8, 4096] dividing K, 16-byte aligned X and Xq, ld_x * 2 a multiple of 16,
-// M > 0) and checked rotq_supported().
+// M > 0) and checked rotq_supported().  bits: 4 (packed nibbles, Xq [M][K/2])
+// or 8 (one code per byte, Xq [M][K]).
 hq_status launch_rotate_quant_stream(int xt, int group, const void* X, int64_t M, int64_t K, int64_t ldx,
                                      const int8_t* d, uint8_t* Xq, float* sx, cudaStream_t st,
-                                     uint64_t limit_ns) {
+                                     uint64_t limit_ns, int bits) {
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return HQ_ERR_CUDA;
@@ -528,12 +556,18 @@ hq_status launch_rotate_quant_stream(int xt, int group, const void* X, int64_t M
     if (r != CUDA_SUCCESS) return HQ_ERR_CUDA;
     const float cg = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(group)));
     const int Mi = static_cast<int>(M), Ki = static_cast<int>(K);
-    if (xt == HQ_BF16) {
-        return d ? launch_rotq_g<rq::XT_BF16, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
-                 : launch_rotq_g<rq::XT_BF16, false>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st);
+    if (bits == 8) {
+        if (xt == HQ_BF16)
+            return d ? launch_rotq_g<rq::XT_BF16, true, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
+                     : launch_rotq_g<rq::XT_BF16, false, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st);
+        return d ? launch_rotq_g<rq::XT_F16, true, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
+                 : launch_rotq_g<rq::XT_F16, false, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st);
     }
-    return d ? launch_rotq_g<rq::XT_F16, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
-             : launch_rotq_g<rq::XT_F16, false>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st);
+    if (xt == HQ_BF16)
+        return d ? launch_rotq_g<rq::XT_BF16, true, false>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
+                 : launch_rotq_g<rq::XT_BF16, false, false>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st);
+    return d ? launch_rotq_g<rq::XT_F16, true, false>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
+             : launch_rotq_g<rq::XT_F16, false, false>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st);
 }
 
 }  // namespace hq

@@ -20,6 +20,7 @@ __all__ = [
     "HQError", "hq_rotate_quant", "hq_rotate", "hq_channel_sqnorm", "hq_select_salient", "w4_pack",
     "serq_prepare", "w4a4_linear", "hq_linear_workspace_size", "hq_debug_accum", "hq_last_device_status",
     "hq_debug_wait_probe", "hq_packed_weight_bytes", "wq_tile", "wq_untile", "W4A4Linear",
+    "hq_rotate_quant8", "w4a8_linear", "hq_debug_accum8",
 ]
 
 
@@ -41,6 +42,19 @@ def hq_rotate_quant(X, group, H_signs=None, Xq=None, sx=None):
     check(lib.hq_rotate_quant(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), group, _signs_arg(H_signs),
                               ptr(Xq), ptr(sx), stream_handle()), "hq_rotate_quant")
     return Xq, sx
+
+
+def hq_rotate_quant8(X, group, H_signs=None, Xq8=None, sx=None):
+    """(Xq8 int8 [M, K], sx float32 [M]): the same rotation with per-token
+    symmetric 8-bit codes in [-127, 127] (the W4A8 activations)."""
+    M, K = X.shape
+    if Xq8 is None:
+        Xq8 = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if sx is None:
+        sx = torch.empty((M,), dtype=torch.float32, device=X.device)
+    check(lib.hq_rotate_quant8(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), group, _signs_arg(H_signs),
+                               ptr(Xq8), ptr(sx), stream_handle()), "hq_rotate_quant8")
+    return Xq8, sx
 
 
 def hq_rotate(X, group, H_signs=None, out=None):
@@ -144,6 +158,40 @@ def w4a4_linear(Xq, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat
     return Y
 
 
+def w4a8_linear(Xq8, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat16, Y=None, workspace=None):
+    """w4a4_linear on 8-bit activation codes Xq8 int8 [M, K]."""
+    M, K = Xq8.shape
+    N = sw.shape[-1]
+    r = 0 if sal_idx is None else int(sal_idx.numel())
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=Xq8.device)
+    need = hq_linear_workspace_size(M, N, K, group)
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=Xq8.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.w4a8_linear(ptr(Xq8), ptr(sx), M, K, ptr(Wq), ptr(sw), ptr(zw), N, group,
+                          ptr(A) if r else None, ptr(B) if r else None, ptr(sal_idx) if r else None, r,
+                          ptr(Y), dtype_code(Y.dtype), ptr(workspace), ws_bytes, stream_handle()), "w4a8_linear")
+    return Y
+
+
+def hq_debug_accum8(Xq8, Wq, zw, group, A, sal_idx, N, decode=False, workspace=None):
+    """Exact int32 accumulators of the W4A8 GEMM kernel: (acc [M, N, G], acc_c [M, N])."""
+    M, K = Xq8.shape
+    r = 0 if sal_idx is None else int(sal_idx.numel())
+    G = K // group if group else 1
+    acc = torch.zeros((M, N, G), dtype=torch.int32, device=Xq8.device)
+    acc_c = torch.zeros((M, N), dtype=torch.int32, device=Xq8.device)
+    need = hq_linear_workspace_size(M, N, K, group) if decode else 0
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=Xq8.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.hq_debug_accum8(ptr(Xq8), M, K, ptr(Wq), ptr(zw), N, group, ptr(A) if r else None,
+                              ptr(sal_idx) if r else None, r, ptr(acc), ptr(acc_c), 1 if decode else 0,
+                              ptr(workspace), ws_bytes, stream_handle()), "hq_debug_accum8")
+    return acc, acc_c
+
+
 def hq_debug_accum(Xq, Wq, zw, group, A, sal_idx, N, decode=False, workspace=None):
     """Exact int32 accumulators of the GEMM kernel: (acc [M, N, G], acc_c [M, N])."""
     M = Xq.shape[0]
@@ -171,7 +219,8 @@ def hq_debug_wait_probe(limit_ns):
 
 
 class W4A4Linear:
-    """A prepared W4A4 layer: rotation signs, packed weights, SERQ term, workspace.
+    """A prepared W4A4 (or, with act_bits=8, W4A8) layer: rotation signs, packed
+    weights, SERQ term, workspace.
 
     ``prepare`` runs the offline steps on the GPU: fold the rotation into W,
     pack to int4, pick the r salient input channels from calibration
@@ -179,10 +228,13 @@ class W4A4Linear:
     ``forward`` is the online path: one rotate/quant launch and one GEMM launch.
     """
 
-    def __init__(self, group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype):
+    def __init__(self, group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype, act_bits=4):
         self.group, self.gw, self.H_signs = group, gw, H_signs
         self.Wq, self.sw, self.zw, self.Rq, self.sr, self.sal_idx = Wq, sw, zw, Rq, sr, sal_idx
         self.K, self.N, self.out_dtype = K, N, out_dtype
+        if act_bits not in (4, 8):
+            raise ValueError("act_bits must be 4 (W4A4) or 8 (W4A8)")
+        self.act_bits = act_bits
         self._ws = {}
 
     @staticmethod
@@ -209,7 +261,8 @@ class W4A4Linear:
                 raise ValueError("sal_idx must be strictly ascending")
 
     @classmethod
-    def prepare(cls, W, group, gw, r, H_signs=None, X_calib=None, sal_idx=None, out_dtype=torch.bfloat16):
+    def prepare(cls, W, group, gw, r, H_signs=None, X_calib=None, sal_idx=None, out_dtype=torch.bfloat16,
+                act_bits=4):
         N, K = W.shape
         cls.check_inputs(K, group, r, H_signs, sal_idx)
         W_rot = hq_rotate(W, group, H_signs)
@@ -223,7 +276,7 @@ class W4A4Linear:
         else:
             sal_idx, Rq, sr = None, None, None
         del W_rot
-        return cls(group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype)
+        return cls(group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype, act_bits)
 
     def reset_workspaces(self):
         """Zero the cached small-M workspaces.  Needed only after a call whose
@@ -243,6 +296,10 @@ class W4A4Linear:
         return ws
 
     def forward(self, X, Y=None, Xq=None, sx=None):
+        if self.act_bits == 8:
+            Xq, sx = hq_rotate_quant8(X, self.group, self.H_signs, Xq, sx)
+            return w4a8_linear(Xq, sx, self.Wq, self.sw, self.zw, self.gw, self.Rq, self.sr, self.sal_idx,
+                               self.out_dtype, Y, self.workspace(X.shape[0], X.device))
         Xq, sx = hq_rotate_quant(X, self.group, self.H_signs, Xq, sx)
         return w4a4_linear(Xq, sx, self.Wq, self.sw, self.zw, self.gw, self.Rq, self.sr, self.sal_idx,
                            self.out_dtype, Y, self.workspace(X.shape[0], X.device))
