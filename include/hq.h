@@ -202,12 +202,11 @@ hq_status serq_prepare(const float* W_rot, int64_t N, int64_t K, const uint8_t* 
  *           with r % 8 == 0 (HQ_ERR_UNSUPPORTED otherwise)
  *  Y        device, [M][N] of type yt (HQ_F16, HQ_BF16 or HQ_F32) (output)
  *  workspace, ws_bytes   device scratch of at least
- *           hq_linear_workspace_size(M, N, K, group) bytes (may be NULL when
- *           that size is 0).  Zero it once before its first use; every call
- *           that completes leaves it zeroed again.  A call whose device status
- *           reports HQ_ERR_TIMEOUT may leave counters behind: zero the
- *           workspace again before its next use.  Calls that share a
- *           workspace must not overlap in time.
+ *           hq_linear_workspace_size(M, N, K, group) bytes.  The current
+ *           kernels need none: that size is 0 for every shape and workspace
+ *           may be NULL.  The parameters stay so that a kernel that needs
+ *           scratch can ask for it without a change of the ABI; a caller that
+ *           passes scratch must zero it before its first use.
  * Requirements: K % 128 == 0, 0 < K <= 65536, N % 8 == 0; Xq, Wq, sw, zw,
  * B, Y and workspace 16-byte aligned, A 4-byte aligned (HQ_ERR_ALIGN).
  * Errors: HQ_ERR_ARG, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA.
@@ -225,28 +224,16 @@ hq_status w4a4_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,
  * memory when they call it.  The pages have no counterpart: this is a service
  * of the library, not a step of the method.
  *
- * w4a4_linear asks its caller for a workspace whenever it uses the small-M
- * (decode, M <= 64) kernel, which needs scratch for the per-tile arrival
- * counters and partial sums of weight tiles split across SMs.  Runtimes that
- * plan all their device buffers once at start-up and forbid allocating later,
- * or whose memory pool is exhausted, cannot provide it.  This entry point takes
- * the same arguments minus the workspace and uses a fixed scratch array of
- * 8 MiB that lives in the library itself (every GPU that loads the library
- * holds it until the process exits); the call allocates nothing.
+ * Runtimes that plan all their device buffers once at start-up and forbid
+ * allocating later, or whose memory pool is exhausted, cannot hand a call
+ * scratch memory.  This entry point takes the arguments of w4a4_linear minus
+ * the workspace and never uses one: both GEMM kernels finish every output
+ * inside the CTA that computes it, so no shape needs scratch.
  *
- *  - The first call on a device looks up the array's device address (a set-up
- *    step done once per device, with that device current); make that first
- *    call before any stream capture.
- *  - All calls share the one array and it keeps the previous call's contents:
- *    each call first clears the arrival counters (an asynchronous memset on
- *    `stream`), so a timeout of an earlier call leaves nothing behind.  Calls
- *    that overlap on the GPU (different streams, or several host threads)
- *    race on the array and must not be issued.
  *  - Every argument check of w4a4_linear runs first; a rejected call enqueues
- *    nothing.  Shapes whose scratch would exceed 8 MiB (hq_linear_workspace_
- *    size(M, N, K, group) > 8 MiB) are rejected with HQ_ERR_UNSUPPORTED, also
- *    before anything is enqueued.  Large M (> 64) uses the large-M kernel,
- *    which needs no scratch.
+ *    nothing.  A shape for which hq_linear_workspace_size would be non-zero
+ *    (none with the current kernels) is rejected with HQ_ERR_UNSUPPORTED,
+ *    also before anything is enqueued.
  * Arguments, results and the other errors are those of w4a4_linear.
  */
 hq_status w4a4_linear_noalloc(const uint8_t* Xq, const float* sx, int64_t M, int64_t K,

@@ -821,24 +821,31 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
     return fn;
 }
 
-// Tensor map of the packed activations Xq[M][K/2] (bytes): boxes of 64 bytes x
-// 128 rows, rows past M filled with zero.
-static hq_status xq_tensor_map(const GemmArgs& a, CUtensorMap* map, bool a8) {
+// 2D tensor map over a row-major array of `outer` rows of `inner` elements,
+// `row_bytes` apart; boxes of box_in x box_out elements, out-of-range elements
+// read as zero.
+hq_status make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle swz) {
     const auto encode = encode_tiled();
     if (!encode) return HQ_ERR_CUDA;
-    // 4-bit codes: boxes of 64 packed bytes x 128 rows into the packed ring;
-    // 8-bit codes: boxes of 128 bytes x 128 rows, 128-byte swizzled, straight
-    // into the MMA's operand stage.  Rows past M read as zero.
-    const cuuint64_t row = static_cast<cuuint64_t>(a8 ? a.K : a.K / 2);
-    const cuuint64_t dims[2] = {row, static_cast<cuuint64_t>(a.M)};
-    const cuuint64_t strides[1] = {row};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(a8 ? pf::BK : pf::PK_ROW), static_cast<cuuint32_t>(pf::BM)};
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_in, box_out};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.Xq), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              a8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
+// Tensor map of the activation codes: 4-bit codes Xq[M][K/2] in boxes of 64
+// packed bytes x 128 rows (into the packed ring); 8-bit codes Xq[M][K] in
+// boxes of 128 bytes x 128 rows, 128-byte swizzled, straight into the MMA's
+// operand stage.  Rows past M read as zero.
+static hq_status xq_tensor_map(const GemmArgs& a, CUtensorMap* map, bool a8) {
+    const uint64_t row = static_cast<uint64_t>(a8 ? a.K : a.K / 2);
+    return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq, row, static_cast<uint64_t>(a.M), row,
+                        a8 ? pf::BK : pf::PK_ROW, pf::BM, a8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 template <int BN, bool ASYM, bool A8, int OUT>

@@ -8,31 +8,48 @@
 // from "OffQ: Taming Structured Outliers in LLM Quantization by Offsetting",
 // Methodology 3.
 //
-// Design:
-//  * operand roles swapped: the MMA's M side (128 TMEM lanes) is 128 weight
-//    rows, its N side is the NT (16, 32 or 64) padded tokens, so the tensor
-//    core does no wasted work on padding rows of a 128-row activation tile.
-//  * stream-K: the (weight-row tile, super-block of 4 K-blocks = 512 inputs)
-//    units are split into equal contiguous ranges, one per CTA, so every SM
-//    streams the same number of weight bytes whatever N is.  A tile split between CTAs is finished by the
-//    last CTA to arrive (an atomic counter per tile in the caller's workspace),
-//    which sums the partial results in a fixed order, so the output does not
-//    depend on arrival order; it resets the counter for the next call.
-//  * two sets of 4 producer warps take alternate K-blocks; each thread owns one
-//    weight row of the tile and streams its 64-byte pieces (contiguous 8 KB
-//    tile blocks in the tile-major weight layout) into a shared-memory ring with
-//    16-byte cp.async copies, 8 K-blocks ahead per set (128 KB in flight per
-//    SM: many independent requests, where one bulk-copy issuer per SM could
-//    not keep enough bytes in flight).  It expands each row to int8 in
-//    registers and writes it straight into tensor memory with tcgen05.st, where
-//    the MMA reads its A operand (no shared-memory round trip for the unpacked
-//    weights); the tokens are expanded into a 128-byte-swizzled shared tile.
-//  * one thread issues tcgen05.mma (A from TMEM) into a double-buffered int32
-//    accumulator with one region per weight group of the super-block; 4
-//    epilogue warps drain it, scale each group by sw[b][n] (one scalar per
-//    lane), and finish with sx[m] and the SERQ term.
-//  * every hand-over between roles (an mbarrier round trip, a few hundred
-//    cycles) covers a whole super-block, not a single 128-input K-block.
+// With at most 64 tokens the layer does at most 128 MACs per weight byte it
+// streams: it is bound by HBM, and the tensor core only has to keep up with
+// the weight stream.  What limits a kernel of this size is the latency of
+// every serial step (a single thread that issues copies or MMAs, hand-offs
+// through barriers), so this one has none: every warp streams, expands and
+// multiplies on its own, with warp-level int8 MMAs (m16n8k32) fed from
+// registers, and the warps meet once, at the end.
+//
+// Design (one CTA per SM, no workspace, no cross-CTA traffic):
+//  * row slices: CTA c owns the weight rows [c N / grid, (c + 1) N / grid), so
+//    every SM streams the same number of weight bytes (within one row) and
+//    finishes its own outputs: no split-K partial sums across CTAs.
+//  * the slice is cut into 16-row tiles; each warp takes one tile and a
+//    contiguous range of its K-blocks (128 inputs), the ranges of a tile
+//    splitting K evenly among the warps the tile gets.
+//  * weights: each thread owns one 16-byte quarter of two rows (g, g + 8) of
+//    every K-block, i.e. 32 codes of each row, and streams them with 16-byte
+//    cp.async copies into its own slots of a ring in shared memory, 8 K-blocks
+//    ahead (a warp's K-block is one contiguous kilobyte of the tile-major
+//    layout).  A thread reads back only what it copied: no barrier.
+//  * K order: the MMA's 32-input step pairs input columns 4t..4t+3 and
+//    16+4t..16+4t+3 of lane t; the kernel maps them to the low and high nibbles
+//    of one packed 32-bit word of 8 codes (inputs k0 k2 k4 k6 / k1 k3 k5 k7),
+//    the same for weights and tokens, so expanding a word to the A or B
+//    fragment is a mask and a shift, and the dot product is unchanged.
+//  * zero points: weights enter the MMA as their unsigned codes u (0..15); a
+//    second MMA with an all-ones A fragment gives each token's code sum S over
+//    the same inputs, and a group's accumulator is acc - z * S (per-channel
+//    weights: z = 8, the offset of the signed codes).
+//  * group accumulators start from the bits of 1.5 * 2^23, so at the end of a
+//    group the int32 result reads as an exact float offset by that constant:
+//    one packed add, then packed fmas for - z * S and the scale sw[b][n].
+//  * the group's zero points and scales ride in the same ring: six lanes copy
+//    the aligned 16-byte chunks that hold the warp's 16 rows, and the warp
+//    reads them after a __syncwarp.
+//  * tokens (the activation codes) are staged once per CTA in shared memory
+//    by bulk copies after the dependency wait (rows padded by 64 bytes, so
+//    the fragment loads hit distinct banks); when they do not fit, each
+//    thread loads its fragments through L1, prefetched 8 K-blocks ahead.
+//  * the warps of a tile add their partial sums in shared memory in a fixed
+//    order; the finish adds the SERQ term X[m,S] . Rq[n,:] (dp4a), multiplies
+//    by sx[m] and stores.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -43,76 +60,67 @@
 
 namespace hq {
 
-namespace sk {
-constexpr int BMW = 128;                 // weight rows per tile = MMA M
+namespace dk {
 constexpr int BK = 128;                  // inputs per K-block
-constexpr int PDEPTH = 8;                // K-blocks in flight per producer set
-constexpr int PSLOTS = 2 * PDEPTH;       // packed-weight ring slots (128 KB)
-constexpr int THREADS = 448;             // warps 0-7 stream + unpack (two sets), 8 TMEM owner, 9 MMA, 10-13 epilogue
-constexpr int ALLOC_WARP = 8;
-constexpr int MMA_WARP = 9;
-constexpr int EPI_WARP0 = 10;
-constexpr int PBYTES = BMW * 64;         // packed bytes of one weight tile block
-constexpr uint32_t TMEM_COLS = 512;
-constexpr int XS_WORDS = 16;             // r <= 64
-constexpr int UCAP = 16;                 // units whose group scales / zero points are staged in smem
-constexpr int MAXG = 4;                  // max weight groups per unit
-__host__ __device__ constexpr int sb_for(int nt) { return nt == 64 ? 2 : 4; }   // K-blocks per unit
-}  // namespace sk
+constexpr int DMAX = 8;                  // K-blocks in flight per warp (8, or 4 to make room for the tokens)
+constexpr int SLOT = 1152;               // one warp's K-block: 2 rows x 32 threads x 16 bytes, then
+                                         // 3 + 3 chunks of 8 zero points / scales
+constexpr int SMEM_MAX = 232448;         // opt-in dynamic shared memory per block
+constexpr int MAXROWS = 256;             // rows of one pass: 16 warps x 16
+constexpr int XS_WORDS = 16;             // salient codes per token as int8 words (r <= 64)
+constexpr uint32_t MAGIC = 0x4B400000u;  // bits of the float 1.5 * 2^23
+constexpr float MAGIC_F = 12582912.0f;
+}  // namespace dk
 
 template <int NT>
-struct SkSmem {
-    static constexpr int SB = sk::sb_for(NT);
-    static constexpr int OFF_RING = 0;
-    static constexpr int OFF_TOK = OFF_RING + sk::PSLOTS * sk::PBYTES;        // 2 stages x SB x NT x 128 B
-    static constexpr int TOK_BYTES = NT * 128;
-    static constexpr int OFF_XS = OFF_TOK + 2 * SB * TOK_BYTES;               // NT x 16 words
-    static constexpr int OFF_SAL = OFF_XS + NT * sk::XS_WORDS * 4;            // 64 int32
-    static constexpr int OFF_SS = OFF_SAL + 64 * 4;                           // UCAP x MAXG x 128 fp16 scales
-    static constexpr int OFF_ZS = OFF_SS + sk::UCAP * sk::MAXG * sk::BMW * 2; // same, zero points
-    static constexpr int OFF_BAR = OFF_ZS + sk::UCAP * sk::MAXG * sk::BMW * 2;
-    static constexpr int NBAR = 10;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;                       // tmem base, abort, last flag
-    static constexpr int BYTES = OFF_MISC + 16;
-    static constexpr int ALLOC = BYTES + 1024;
+struct DkCfg {
+    static constexpr int W = NT == 64 ? 8 : (NT == 32 ? 12 : 16);   // warps
+    static constexpr int THREADS = 32 * W;
+    static constexpr int NTT = NT / 8;                       // MMA n-tiles of 8 tokens
+    static constexpr int PART = W * 32 * NTT * 4 * 4;        // partial sums, aliased onto the ring
+    // after the ring: the token barrier, salient codes, the pass's SERQ rows Rq
+    // (r/2 bytes each), sr and sw (fp16 pairs from an even row), and sx
+    static constexpr int F_BAR = 0;
+    static constexpr int F_XS = 16;
+    static constexpr int F_RQ = F_XS + NT * dk::XS_WORDS * 4;
+    static constexpr int F_SR = F_RQ + dk::MAXROWS * 32;
+    static constexpr int F_SW = F_SR + (dk::MAXROWS + 8) * 2;
+    static constexpr int F_SX = F_SW + (dk::MAXROWS + 8) * 2;
+    static constexpr int FIX = (F_SX + NT * 4 + 15) / 16 * 16;
+    static constexpr int XITEMS = (NT * dk::XS_WORDS + THREADS - 1) / THREADS;
 };
 
-struct SkPlan {
-    int ntiles;   // weight-row tiles
-    int KB;       // K-blocks per row
-    int sb;       // K-blocks per unit (super-block)
-    int gs;       // K-blocks per weight group (1 for per-channel weights)
-    int upt;      // units per tile = ceil(KB / sb)
-    int units;    // ntiles * upt
-    int grid;     // CTAs
-    int maxc;     // max CTAs contributing to one tile
+struct DkPlan {
+    int grid;      // CTAs; CTA c owns weight rows [c N / grid, (c + 1) N / grid)
+    int D;         // K-blocks in flight per warp (8 or 4)
+    int ring;      // bytes of the rings (W x D slots)
+    int tstride;   // bytes per staged token row (row bytes + 64)
 };
-
-__host__ __device__ inline int sk_owner(int u, int units, int grid) {
-    return static_cast<int>((static_cast<long long>(u + 1) * grid - 1) / units);
-}
-__host__ __device__ inline int sk_begin(int c, int units, int grid) {
-    return static_cast<int>(static_cast<long long>(c) * units / grid);
-}
 
 static int nt_for(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-static SkPlan sk_plan(int64_t M, int64_t N, int64_t K, int gw, int nsm) {
-    SkPlan p{};
-    p.ntiles = static_cast<int>((N + sk::BMW - 1) / sk::BMW);
-    p.KB = static_cast<int>(K / sk::BK);
-    p.sb = sk::sb_for(nt_for(M));
-    p.gs = gw ? gw / sk::BK : 1;
-    p.upt = (p.KB + p.sb - 1) / p.sb;
-    p.units = p.ntiles * p.upt;
+// Launch plan; `staged` tells whether the tokens fit in shared memory.
+template <int NT>
+static DkPlan dk_plan(int64_t M, int64_t N, int64_t K, bool a8, int nsm, bool& staged) {
+    using C = DkCfg<NT>;
+    DkPlan p{};
     const int want = nsm > 0 ? nsm : 148;
-    p.grid = p.units < want ? p.units : want;
-    p.maxc = 1;
-    for (int t = 0; t < p.ntiles; ++t) {
-        const int a = sk_owner(t * p.upt, p.units, p.grid);
-        const int b = sk_owner((t + 1) * p.upt - 1, p.units, p.grid);
-        if (b - a + 1 > p.maxc) p.maxc = b - a + 1;
+    const int64_t tiles = (N + 15) / 16;   // at least one 16-row tile per CTA
+    p.grid = static_cast<int>(tiles < want ? tiles : want);
+    p.tstride = static_cast<int>(a8 ? K : K / 2) + 64;
+    const int64_t tok = static_cast<int64_t>(NT) * p.tstride;
+    staged = true;
+    for (int d : {dk::DMAX, 4}) {
+        const int64_t ring = static_cast<int64_t>(C::W) * d * dk::SLOT;
+        if (ring >= C::PART && ring + C::FIX + tok <= dk::SMEM_MAX) {
+            p.D = d;
+            p.ring = static_cast<int>(ring);
+            return p;
+        }
     }
+    staged = false;
+    p.D = dk::DMAX;
+    p.ring = C::W * dk::DMAX * dk::SLOT;
     return p;
 }
 
@@ -127,525 +135,476 @@ __device__ __forceinline__ void store_one(void* Y, int64_t i, float y) {
     }
 }
 
-// NT accumulator columns of one lane quarter -> registers (no wait).
-template <int NT>
-__device__ __forceinline__ void ld_cols(uint32_t taddr, uint32_t (&v)[NT]) {
-    if constexpr (NT == 16) {
-        tmem_ld_32x32b_x16(taddr, v);
-    } else if constexpr (NT == 32) {
-        tmem_ld_32x32b_x32(taddr, v);
-    } else {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-        tmem_ld_32x32b_x32(taddr, lo);
-        tmem_ld_32x32b_x32(taddr + 32, hi);
-    }
+// d = a * b + c (int8 x int8 -> int32, 16 x 8 x 32); c may alias d.
+__device__ __forceinline__ void mma_s8_c(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                         const uint32_t (&c)[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %11, %12, %13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(c[2]),
+          "r"(c[3]));
+}
+
+// B fragment words of 8 tokens codes k0..k7 held as two words (k0..k3,
+// k4..k7): (k0 k2 k4 k6) and (k1 k3 k5 k7), the order of unpack_s4x8_times16.
+__device__ __forceinline__ void tok_words8(uint32_t x0, uint32_t x1, uint32_t& lo, uint32_t& hi) {
+    lo = __byte_perm(x0, x1, 0x6420);
+    hi = __byte_perm(x0, x1, 0x7531);
 }
 
 // A8: 8-bit activation codes ([M][K] int8, used as they are) instead of packed
-// 4-bit codes (expanded as 16 q).
-template <int NT, bool ASYM, bool A8, int OUT>
-__global__ void __launch_bounds__(sk::THREADS, 1) k_gemm_small(const GemmArgs p, const SkPlan plan) {
-    using L = SkSmem<NT>;
-    constexpr int XROW = A8 ? 128 : 64;   // activation bytes per token row and K-block
-    constexpr int SB = L::SB;
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte aligned base, derived by pointer arithmetic on the __shared__
-    // array so that every access through it compiles to a shared-memory
-    // instruction (a pointer rebuilt from an integer is generic)
-    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t bar0 = smem_u32(smem + L::OFF_BAR);
-    auto fulla = [&](int s) { return bar0 + 8u * s; };          // A stage s written (producer set s)
-    auto emptya = [&](int s) { return bar0 + 8u * (2 + s); };   // A stage s consumed (MMA)
-    auto accf = [&](int b) { return bar0 + 8u * (4 + b); };
-    auto acce = [&](int b) { return bar0 + 8u * (6 + b); };
-    const uint32_t done_bar = bar0 + 8u * 8;
-    const uint32_t scl_bar = bar0 + 8u * 9;
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);   // [0] tmem, [1] abort, [2] last
-    volatile uint32_t* abort_flag = misc + 1;
-    uint32_t* xs_s = reinterpret_cast<uint32_t*>(smem + L::OFF_XS);
-    int32_t* sal_s = reinterpret_cast<int32_t*>(smem + L::OFF_SAL);
-    const uint16_t* ss = reinterpret_cast<const uint16_t*>(smem + L::OFF_SS);   // [unit][group][row]
-    const uint16_t* zs = reinterpret_cast<const uint16_t*>(smem + L::OFF_ZS);
+// 4-bit codes (expanded as 16 q).  TS: tokens staged in shared memory.
+template <int NT, bool ASYM, bool A8, int OUT, bool TS>
+__global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const GemmArgs p, const DkPlan plan) {
+    using C = DkCfg<NT>;
+    constexpr int NTT = C::NTT;
+    constexpr int W = C::W;
+    constexpr int TOKV = A8 ? 2 : 1;                   // uint4 per token fragment and K-block
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* fix = smem + plan.ring;
+    const uint32_t tbar = smem_u32(fix + C::F_BAR);
+    uint32_t* xs_s = reinterpret_cast<uint32_t*>(fix + C::F_XS);
+    const uint8_t* rq_s = fix + C::F_RQ;
+    const uint16_t* sr_s = reinterpret_cast<const uint16_t*>(fix + C::F_SR);
+    const uint16_t* sw_s = reinterpret_cast<const uint16_t*>(fix + C::F_SW);
+    float* sx_s = reinterpret_cast<float*>(fix + C::F_SX);
+    uint8_t* tok_s = fix + C::FIX;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int cta = blockIdx.x;
+    const int r0 = static_cast<int>(static_cast<long long>(cta) * p.N / plan.grid);
+    const int r1 = static_cast<int>(static_cast<long long>(cta + 1) * p.N / plan.grid);
+    const int RT = (r1 - r0 + 15) / 16;
+    const int KB = p.K / dk::BK;
+    const int gs = ASYM ? p.gw / dk::BK : KB;         // K-blocks per weight group
+    const int G = ASYM ? p.K / p.gw : 1;
+    const int64_t xrow = A8 ? p.K : p.K / 2;           // bytes per token row
+    const int D = plan.D;
+    // the accumulators carry the factor 16 of 4-bit activation codes
+    constexpr int sh = A8 ? 0 : 4;
+    constexpr float inv_act = A8 ? 1.0f : 0.0625f;
 
-    const int KB = plan.KB, upt = plan.upt, gs = plan.gs;
-    const int u0 = sk_begin(blockIdx.x, plan.units, plan.grid);
-    const int u1 = sk_begin(blockIdx.x + 1, plan.units, plan.grid);
-    const int nunits = u1 - u0;
-    const int nstaged = nunits < sk::UCAP ? nunits : sk::UCAP;
-    // unit geometry: tile, first K-block, K-blocks
-    auto unit_tile = [&](int u) { return u / upt; };
-    auto unit_kb0 = [&](int u) { return (u - (u / upt) * upt) * SB; };
-    auto unit_nk = [&](int u) { const int r = KB - unit_kb0(u); return r < SB ? r : SB; };
-
-    if (warp == sk::ALLOC_WARP) {
-        if (lane == 0) {
-            for (int s = 0; s < 2; ++s) {
-                mbar_init(fulla(s), 128);
-                mbar_init(emptya(s), 1);
-                mbar_init(accf(s), 1);
-                mbar_init(acce(s), 4);
-            }
-            mbar_init(done_bar, 1);
-            mbar_init(scl_bar, 128);
-            misc[1] = 0;
+    if constexpr (TS) {
+        if (tid == 0) {
+            mbar_init(tbar, 1);
             fence_mbar_init();
         }
-        __syncwarp();
-        tmem_alloc(smem_u32(misc), sk::TMEM_COLS);
-        tmem_relinquish();
+        // token rows past M read as zero
+        for (int i = tid; i < (NT - p.M) * (plan.tstride / 16); i += C::THREADS)
+            *reinterpret_cast<uint4*>(tok_s + (p.M + i / (plan.tstride / 16)) * plan.tstride + 16 * (i % (plan.tstride / 16))) =
+                make_uint4(0, 0, 0, 0);
+        __syncthreads();
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = misc[0];
-    const uint32_t acc_col0 = 2 * SB * 32;
 
-    auto waitx = [&](uint32_t bar, uint32_t parity) -> bool {
-        if (*abort_flag) return false;
-        if (!mbar_wait(bar, parity, p.limit_ns)) {
-            *abort_flag = 1;
-            return false;
+    // salient activation codes of every token, gathered into xs_s before the
+    // finish in the lo/hi word order of unpack_s4x8_times16: the indices now,
+    // the codes after the dependency wait, the shared-memory stores at the end
+    int salk[C::XITEMS][4];
+#pragma unroll
+    for (int it = 0; it < C::XITEMS; ++it) {
+        const int idx = tid + it * C::THREADS;
+        const int m = idx / dk::XS_WORDS, w = idx % dk::XS_WORDS;
+        const int i = w >> 1, hh = w & 1;   // word 2i+hh holds positions 8i+2e+hh, byte e
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = 8 * i + 2 * e + hh;
+            int k = -1;
+            if (idx < NT * dk::XS_WORDS && m < p.M && j < p.r) {
+                k = __ldg(p.sal + j);
+                if (static_cast<unsigned>(k) >= static_cast<unsigned>(p.K)) {
+                    record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
+                    k = -1;
+                }
+            }
+            salk[it][e] = k;
         }
-        return true;
+    }
+    uint32_t xsw[C::XITEMS];
+    bool waited = false, gathered = false;
+    auto deps = [&]() {
+        // the token codes are the preceding kernel's output
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if constexpr (TS) {
+            if (warp == 0) {
+                if (lane == 0) mbar_arrive_expect_tx(tbar, static_cast<uint32_t>(p.M * xrow));
+                __syncwarp();
+                for (int m = lane; m < p.M; m += 32)
+                    bulk_copy_g2s(smem_u32(tok_s + m * plan.tstride), p.Xq + m * xrow, static_cast<uint32_t>(xrow), tbar);
+            }
+        }
+        waited = true;
+    };
+    // (issued once the salient indices have arrived, so the loads do not stall)
+    auto gather = [&]() {
+        if (!waited) deps();
+#pragma unroll
+        for (int it = 0; it < C::XITEMS; ++it) {
+            const int m = (tid + it * C::THREADS) / dk::XS_WORDS;
+            uint32_t word = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = salk[it][e];
+                if (k >= 0) {
+                    const uint8_t* xr = p.Xq + static_cast<int64_t>(m) * xrow;
+                    if constexpr (A8) {
+                        word |= static_cast<uint32_t>(__ldg(xr + k)) << (8 * e);
+                    } else {
+                        const int nib = (__ldg(xr + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
+                        word |= (static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu) << (8 * e);
+                    }
+                }
+            }
+            xsw[it] = word;
+        }
+        if constexpr (OUT != OUT_DEBUG) {   // the debug entry passes no scales
+            for (int m = tid; m < NT; m += C::THREADS) sx_s[m] = m < p.M ? p.sx[m] : 0.f;
+        }
+        gathered = true;
     };
 
-    if (warp < 8) {
-        // ======================= producers: two sets of 4 warps take alternate units.
-        // Each thread owns one weight row of the tile: it streams the row's
-        // 64-byte pieces with cp.async, expands them to int8 and writes them into
-        // its lane of the set's tensor-memory A stage; it also expands a share of
-        // the unit's tokens into the set's token stage.
-        const int pset = warp >> 2;
-        const int row = (warp & 3) * 32 + lane;
-        constexpr int TCH = (NT * (XROW / 16) + 127) / 128;   // token chunks per thread per K-block
-        // write cursor (cp.async issue) over this set's K-blocks
-        int wli = pset, wkbi = 0, wctr = 0;
-        auto issue_next = [&]() {
-            if (wli < nunits) {
-                const int u = u0 + wli;
-                const int64_t blk = static_cast<int64_t>(unit_tile(u)) * KB + unit_kb0(u) + wkbi;
-                const int slot = pset * sk::PDEPTH + (wctr % sk::PDEPTH);
-                const uint8_t* src = p.Wq + blk * sk::PBYTES + row * 64;
-                const uint32_t dst = smem_u32(smem + L::OFF_RING + slot * sk::PBYTES + row * 64);
+    const uint32_t ring = smem_u32(smem + warp * D * dk::SLOT);
+    const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
+    const uint32_t zero4[4] = {0u, 0u, 0u, 0u};
+    const uint32_t mag4[4] = {dk::MAGIC, dk::MAGIC, dk::MAGIC, dk::MAGIC};
+    bool tok_ready = !TS;
+
+    const int npass = (RT + W - 1) / W;
+    for (int pass = 0; pass < npass; ++pass) {
+        const int t0 = pass * W;
+        const int ntp = (RT - t0) < W ? (RT - t0) : W;   // tiles of this pass
+        const int S = W / ntp;                           // warps per tile
+        const int tl = warp % ntp, sp = warp / ntp;
+        const bool active = sp < S;
+        const int base = r0 + 16 * (t0 + tl);            // the warp's first row
+        const int rowA = base + gq, rowB = rowA + 8;
+        const bool okA = rowA < r1, okB = rowB < r1;
+        const int c0 = base & ~7;                        // first of the 8-row chunks of zero points / scales
+        // the finish's operands of this pass's rows [pr0, pr1), in flight during the K loop:
+        // Rq rows (r/2 bytes each, a multiple of 4), and the fp16 pairs of sr and
+        // (per-channel) sw from the even row pb = pr0 & ~1
+        const int pr0 = r0 + 16 * t0, pr1 = (r0 + 16 * (t0 + ntp)) < r1 ? r0 + 16 * (t0 + ntp) : r1;
+        const int pb = pr0 & ~1;
+        {
+            const int nrq = (pr1 - pr0) * (p.r / 8);
+            for (int idx = tid; idx < nrq; idx += C::THREADS)
+                cp_async4(smem_u32(rq_s + 4 * idx), p.Rq + static_cast<int64_t>(pr0) * (p.r / 2) + 4 * idx);
+            if constexpr (OUT != OUT_DEBUG) {
+                const int npair = (pr1 - pb + 1) / 2;
+                for (int idx = tid; idx < npair; idx += C::THREADS) {
+                    if (p.r > 0) cp_async4(smem_u32(sr_s + 2 * idx), p.sr + pb + 2 * idx);
+                    if constexpr (!ASYM) cp_async4(smem_u32(sw_s + 2 * idx), p.sw + pb + 2 * idx);
+                }
+            }
+        }
+        const int kb0 = static_cast<int>(static_cast<long long>(sp) * KB / S);
+        int kb1 = active ? static_cast<int>(static_cast<long long>(sp + 1) * KB / S) : kb0;
+        // partial sums of this warp's K range, in the m16n8 accumulator layout:
+        // [nt][0,1] = row g, tokens 8 nt + 2 t + {0,1}; [nt][2,3] = row g + 8
+        float y[NTT][4];
+        int32_t yi[NTT][4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) cp_async16(dst + 16 * c, src + 16 * c);
-                if (++wkbi == unit_nk(u)) { wkbi = 0; wli += 2; }
+        for (int nt = 0; nt < NTT; ++nt)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                y[nt][v] = 0.f;
+                yi[nt][v] = 0;
+            }
+        // request cursor: next K-block, its ring slot, its sources (one weight tile
+        // after another: consecutive K-blocks of a row are 8 KB apart)
+        int ik = kb0, islot = 0, igk = kb0 % gs;
+        const uint8_t* srcA = p.Wq + (static_cast<int64_t>(rowA >> 7) * KB + kb0) * 8192 + (rowA & 127) * 64 + tq * 16;
+        const uint8_t* srcB = p.Wq + (static_cast<int64_t>(rowB >> 7) * KB + kb0) * 8192 + (rowB & 127) * 64 + tq * 16;
+        // zero points (lanes 0-2) and scales (3-5) of rows [c0, c0 + 24) of the
+        // group: 16-byte chunks of 8 rows (N % 8 == 0)
+        const int zj = lane < 3 ? lane : lane - 3;
+        const bool zlane = ASYM && lane < (OUT == OUT_DEBUG ? 3 : 6) && c0 + 8 * zj < p.N;
+        const uint16_t* zsrc = nullptr;
+        if constexpr (ASYM) zsrc = (lane < 3 || OUT == OUT_DEBUG ? p.zw : p.sw) + static_cast<int64_t>(kb0 / gs) * p.N + c0 + 8 * zj;
+        auto issue = [&]() {
+            if (ik < kb1) {
+                const uint32_t slot = ring + static_cast<uint32_t>(islot) * dk::SLOT;
+                if (okA) cp_async16(slot + lane * 16, srcA);
+                if (okB) cp_async16(slot + 512 + lane * 16, srcB);
+                if constexpr (ASYM) {
+                    if (zlane) cp_async16(slot + 1024 + 48 * (lane / 3) + 16 * zj, zsrc);
+                    if (++igk == gs) {
+                        igk = 0;
+                        zsrc += p.N;
+                    }
+                }
+                srcA += 8192;
+                srcB += 8192;
+                ++ik;
+                islot = islot + 1 == D ? 0 : islot + 1;
             }
             cp_async_commit();   // one group per K-block (possibly empty)
-            ++wctr;
         };
-        for (int d = 0; d < sk::PDEPTH; ++d) issue_next();
-        if (ASYM && nstaged > 0) __all_sync(0xFFFFFFFFu, waitx(scl_bar, 0));   // zero points staged
-        asm volatile("griddepcontrol.wait;" ::: "memory");   // tokens are the preceding kernel's output
-        // this thread's share of a unit's packed tokens, loaded one unit ahead
-        // (an L2 round trip is several hundred ns; it must not sit in the K loop)
-        auto load_unit_tokens = [&](int li, uint4 (&tk)[SB][TCH]) {
+        // token codes of K-block kb into L1 ahead of their loads (after the dependency wait only)
+        auto tok_prefetch = [&](int kb) {
+            if constexpr (!TS) {
+                if (kb < kb1) {
 #pragma unroll
-            for (int kbi = 0; kbi < SB; ++kbi)
-#pragma unroll
-                for (int c = 0; c < TCH; ++c) tk[kbi][c] = make_uint4(0, 0, 0, 0);
-            if (li >= nunits) return;
-            const int u = u0 + li;
-            const int kb0 = unit_kb0(u), nk = unit_nk(u);
-#pragma unroll
-            for (int kbi = 0; kbi < SB; ++kbi) {
-#pragma unroll
-                for (int c = 0; c < TCH; ++c) {
-                    const int tc = row + 128 * c;
-                    const int tr = tc / (XROW / 16), ch = tc % (XROW / 16);
-                    if (kbi < nk && tc < NT * (XROW / 16) && tr < p.M)
-                        tk[kbi][c] = __ldg(reinterpret_cast<const uint4*>(p.Xq + static_cast<int64_t>(tr) * (A8 ? p.K : p.K / 2) +
-                                                                       (kb0 + kbi) * XROW + ch * 16));
+                    for (int nt = 0; nt < NTT; ++nt) {
+                        const int m = 8 * nt + gq;
+                        if (m < p.M && tq == 0) prefetch_l1(p.Xq + static_cast<int64_t>(m) * xrow + kb * (A8 ? 128 : 64));
+                    }
                 }
             }
         };
-        uint4 tk_cur[SB][TCH], tk_nxt[SB][TCH];
-        load_unit_tokens(pset, tk_cur);
-        int rctr = 0;
-        bool ok = true;
-        for (int li = pset; ok && li < nunits; li += 2) {
-            const int u = u0 + li;
-            const int t = unit_tile(u), kb0 = unit_kb0(u), nk = unit_nk(u);
-            const int n = t * sk::BMW + row;
-            const uint32_t use = static_cast<uint32_t>(li >> 1);     // use count of this set's stage
-            load_unit_tokens(li + 2, tk_nxt);
-            if (!__all_sync(0xFFFFFFFFu, waitx(emptya(pset), (use & 1u) ^ 1u))) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kbi = 0; kbi < SB; ++kbi) {
-                if (kbi >= nk) break;
-                const int kb = kb0 + kbi;
-                uint32_t z4 = 0;
-                if constexpr (ASYM) {
-                    const int gi = kbi / gs;
-                    uint32_t z = 0;
-                    if (n < p.N) {
-                        if (li < sk::UCAP) {
-                            z = static_cast<uint32_t>(__half2float(__ushort_as_half(zs[(li * sk::MAXG + gi) * sk::BMW + row])));
-                        } else {
-                            const int g = (kb * sk::BK) / p.gw;
-                            z = static_cast<uint32_t>(__half2float(__ushort_as_half(p.zw[static_cast<int64_t>(g) * p.N + n])));
-                        }
-                    }
-                    z4 = z * 0x01010101u;
-                }
-                cp_async_wait_group<sk::PDEPTH - 1>();   // this thread's piece of the K-block has landed
-                const uint8_t* src = smem + L::OFF_RING + (pset * sk::PDEPTH + (rctr % sk::PDEPTH)) * sk::PBYTES + row * 64;
-                uint4 c4[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) c4[c] = *reinterpret_cast<const uint4*>(src + (c << 4));
-                ++rctr;
-                issue_next();                          // refill the slot just read
-                uint32_t a[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t w[4] = {c4[c].x, c4[c].y, c4[c].z, c4[c].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        if constexpr (ASYM) unpack_u4x8_minus_z(w[e], z4, a[8 * c + 2 * e], a[8 * c + 2 * e + 1]);
-                        else unpack_s4x8_times16(w[e], a[8 * c + 2 * e], a[8 * c + 2 * e + 1]);
-                        if constexpr (A8) {
-                            // 8-bit activations keep their natural K order: interleave the
-                            // (k0 k2 k4 k6, k1 k3 k5 k7) words back to (k0..k3, k4..k7)
-                            const uint32_t lo = a[8 * c + 2 * e], hi = a[8 * c + 2 * e + 1];
-                            a[8 * c + 2 * e] = __byte_perm(lo, hi, 0x5140);
-                            a[8 * c + 2 * e + 1] = __byte_perm(lo, hi, 0x7362);
-                        }
-                    }
-                }
-                tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
-                                       static_cast<uint32_t>((pset * SB + kbi) * 32), a);
-                uint8_t* tstage = smem + L::OFF_TOK + (pset * SB + kbi) * L::TOK_BYTES;
-#pragma unroll
-                for (int c = 0; c < TCH; ++c) {
-                    const int tc = row + 128 * c;
-                    if (tc < NT * (XROW / 16)) {
-                        const int tr = tc / (XROW / 16), ch = tc % (XROW / 16);
-                        uint8_t* trow = tstage + tr * 128;
-                        if constexpr (A8) {
-                            // 16 codes as they are, into 16-byte chunk ch of the swizzled row
-                            *reinterpret_cast<uint4*>(trow + ((ch ^ (tr & 7)) << 4)) = tk_cur[kbi][c];
-                        } else {
-                            uint32_t o[8];
-                            const uint32_t w[4] = {tk_cur[kbi][c].x, tk_cur[kbi][c].y, tk_cur[kbi][c].z, tk_cur[kbi][c].w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) unpack_s4x8_times16(w[e], o[2 * e], o[2 * e + 1]);
-                            *reinterpret_cast<uint4*>(trow + (((2 * ch) ^ (tr & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                            *reinterpret_cast<uint4*>(trow + (((2 * ch + 1) ^ (tr & 7)) << 4)) =
-                                make_uint4(o[4], o[5], o[6], o[7]);
-                        }
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(fulla(pset));
-#pragma unroll
-            for (int kbi = 0; kbi < SB; ++kbi)
-#pragma unroll
-                for (int c = 0; c < TCH; ++c) tk_cur[kbi][c] = tk_nxt[kbi][c];
-        }
-        cp_async_wait_all();   // nothing in flight when the CTA exits
-    } else if (warp == sk::MMA_WARP) {
-        // ======================= MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_i8(sk::BMW, NT);
-            int abuf = 0;
-            uint32_t accph = 0;
-            for (int li = 0; li < nunits; ++li) {
-                const int u = u0 + li;
-                const int t = unit_tile(u), nk = unit_nk(u);
-                const bool seg_first = (li == 0) || unit_tile(u - 1) != t;
-                const bool seg_last = (li + 1 == nunits) || unit_tile(u + 1) != t;
-                const bool grp_first = ASYM || seg_first;
-                const bool grp_last = ASYM || seg_last;
-                if (grp_first) {
-                    if (!waitx(acce(abuf), ((accph >> abuf) & 1u) ^ 1u)) break;
-                }
-                const int s = li & 1;
-                if (!waitx(fulla(s), static_cast<uint32_t>((li >> 1) & 1))) break;
-                tc_fence_after();
-                const uint32_t acc = tmem_base + acc_col0 + static_cast<uint32_t>(abuf * SB * NT);
-                for (int kbi = 0; kbi < nk; ++kbi) {
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + L::OFF_TOK + (s * SB + kbi) * L::TOK_BYTES));
-                    const uint32_t dcol = acc + (ASYM ? static_cast<uint32_t>((kbi / gs) * NT) : 0u);
-                    const bool fresh = ASYM ? (kbi % gs == 0) : (seg_first && kbi == 0);
-#pragma unroll
-                    for (int kk = 0; kk < sk::BK / 32; ++kk)
-                        mma_i8_ts(dcol, tmem_base + static_cast<uint32_t>((s * SB + kbi) * 32 + kk * 8), bdesc + 2u * kk,
-                                  IDESC, (fresh && kk == 0) ? 0u : 1u);
-                }
-                tc_commit(emptya(s));
-                if (grp_last) {
-                    tc_commit(accf(abuf));
-                    accph ^= 1u << abuf;
-                    abuf ^= 1;
-                }
-            }
-            tc_commit(done_bar);
-            mbar_wait(done_bar, 0, p.limit_ns);
-        }
-        __syncwarp();
-    } else if (warp >= sk::EPI_WARP0) {
-        // ======================= epilogue: drain, finish or hand over
-        const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int ethr = (warp - sk::EPI_WARP0) * 32 + lane;   // 0..127
-        if constexpr (ASYM) {
-            // weight-side group scales and zero points of the first UCAP units (they
-            // do not depend on the preceding kernel): 16-byte async copies of the
-            // 128-entry rows, all in flight together, one round trip
-            uint8_t* ssw = smem + L::OFF_SS;
-            uint8_t* zsw = smem + L::OFF_ZS;
-            const int arrays = (OUT == OUT_DEBUG) ? 1 : 2;
-            const int items = nstaged * sk::MAXG * arrays * 16;
-            const int G = p.K / p.gw;
-            for (int idx = ethr; idx < items; idx += 128) {
-                const int c = idx % 16, a = (idx / 16) % arrays, gi = (idx / (16 * arrays)) % sk::MAXG;
-                const int li = idx / (16 * arrays * sk::MAXG);
-                const int u = u0 + li;
-                const int g = unit_kb0(u) / gs + gi;
-                const int n0 = unit_tile(u) * sk::BMW + c * 8;
-                uint8_t* dst = (a == 0 ? zsw : ssw) + ((li * sk::MAXG + gi) * sk::BMW + c * 8) * 2;
-                if (n0 < p.N && gi * gs < unit_nk(u) && g < G) {
-                    const uint16_t* src = (a == 0 ? p.zw : p.sw) + static_cast<int64_t>(g) * p.N + n0;
-                    cp_async16(smem_u32(dst), src);
-                } else {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            cp_async_commit();
-            cp_async_wait_all();
-            mbar_arrive(scl_bar);
-        }
-        asm volatile("griddepcontrol.wait;" ::: "memory");   // sx, Xq and the outputs follow the preceding kernel
-        // gathered salient activation codes of every token (needed when a tile
-        // finishes): int8 words in the lo/hi order of unpack_s4x8_times16
-        for (int j = ethr; j < p.r; j += 128) sal_s[j] = p.sal[j];
-        named_bar_sync(1, 128);
-        for (int idx = ethr; idx < NT * sk::XS_WORDS; idx += 128) {
-            const int m = idx / sk::XS_WORDS, w = idx % sk::XS_WORDS;
-            uint32_t word = 0;
-            if (m < p.M) {
-                const uint8_t* xrow = p.Xq + static_cast<int64_t>(m) * (A8 ? p.K : p.K / 2);
-                const int i = w >> 1, h = w & 1;   // word 2i+h holds positions 8i+2e+h, byte e
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 8 * i + 2 * e + h;
-                    if (j < p.r) {
-                        const int k = sal_s[j];
-                        if (static_cast<unsigned>(k) < static_cast<unsigned>(p.K)) {
-                            if constexpr (A8) {
-                                word |= static_cast<uint32_t>(__ldg(xrow + k)) << (8 * e);
-                            } else {
-                                const int nib = (__ldg(xrow + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
-                                word |= (static_cast<uint32_t>((nib ^ 8) - 8) & 0xFFu) << (8 * e);
-                            }
-                        } else {
-                            record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
-                        }
-                    }
-                }
-            }
-            xs_s[idx] = word;
-        }
-        named_bar_sync(1, 128);
-        if (ASYM && nstaged > 0) waitx(scl_bar, 0);
-        int abuf = 0;
-        uint32_t accph = 0;
-        uint32_t* ws_cnt = static_cast<uint32_t*>(p.ws);
-        float* ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(p.ws) + small_counter_bytes(plan.ntiles));
-        // the accumulators carry the factor of the activation codes (16 for
-        // 4-bit codes, 1 for 8-bit) and 16 for symmetric weight codes
-        const int sh = (A8 ? 0 : 4) + (ASYM ? 0 : 4);
-        const int G = ASYM ? p.K / p.gw : 1;
-        int li = 0;
-        while (li < nunits) {
-            const int t = unit_tile(u0 + li);
-            int le = li + 1;
-            while (le < nunits && unit_tile(u0 + le) == t) ++le;
-            const int n = t * sk::BMW + row;
-            const bool nvalid = n < p.N;
-            // operands of the tile's finish, fetched early (their latency hides under the K loop)
-            uint32_t rqp[sk::XS_WORDS / 2];
-#pragma unroll
-            for (int i = 0; i < sk::XS_WORDS / 2; ++i) rqp[i] = 0;
-            float swn = 0.f, srn = 0.f;
-            if (nvalid) {
-                if (p.r > 0) {
-                    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.Rq + static_cast<int64_t>(n) * (p.r / 2));
-#pragma unroll
-                    for (int i = 0; i < sk::XS_WORDS / 2; ++i)
-                        if (i < p.r / 8) rqp[i] = __ldg(src + i);
-                }
-                if constexpr (OUT != OUT_DEBUG) {
-                    if constexpr (!ASYM) swn = __half2float(__ushort_as_half(p.sw[n]));
-                    if (p.r > 0) srn = __half2float(__ushort_as_half(p.sr[n]));
-                }
-            }
-            float y[NT];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) y[j] = 0.f;
-            const int drains = ASYM ? le - li : 1;
-            for (int di = 0; di < drains; ++di) {
-                waitx(accf(abuf), (accph >> abuf) & 1u);
-                tc_fence_after();
-                const uint32_t acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc_col0 +
-                                     static_cast<uint32_t>(abuf * SB * NT);
-                if constexpr (ASYM) {
-                    const int uli = li + di;
-                    const int uu = u0 + uli;
-                    const int ng = unit_nk(uu) / gs;
-                    for (int gi = 0; gi < ng; ++gi) {
-                        uint32_t v[NT];
-                        ld_cols<NT>(acc + static_cast<uint32_t>(gi * NT), v);
-                        tmem_wait_ld();
-                        const int g = unit_kb0(uu) / gs + gi;
-                        float s = 0.f;   // the debug entry passes no scales
-                        if constexpr (OUT != OUT_DEBUG) {
-                            if (uli < sk::UCAP)
-                                s = __half2float(__ushort_as_half(ss[(uli * sk::MAXG + gi) * sk::BMW + row]));
-                            else if (nvalid)
-                                s = __half2float(__ushort_as_half(p.sw[static_cast<int64_t>(g) * p.N + n]));
-                        }
-#pragma unroll
-                        for (int j = 0; j < NT; ++j) {
-                            const int a = static_cast<int32_t>(v[j]) >> sh;
-                            if constexpr (OUT == OUT_DEBUG) {
-                                if (nvalid && j < p.M) p.dbg_acc[(static_cast<int64_t>(j) * p.N + n) * G + g] = a;
-                            }
-                            y[j] = __fmaf_rn(s, static_cast<float>(a), y[j]);
-                        }
-                    }
-                } else {
-                    uint32_t v[NT];
-                    ld_cols<NT>(acc, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < NT; ++j) y[j] = static_cast<float>(static_cast<int32_t>(v[j]) >> sh);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acce(abuf));
-                accph ^= 1u << abuf;
-                abuf ^= 1;
-            }
-            const bool whole = (u0 + li == t * upt) && (u0 + le == (t + 1) * upt);
-            bool finish = whole;
-            if (!whole) {
-                // hand the partial result over: slot = position of this CTA among the tile's contributors
-                const int first = sk_owner(t * upt, plan.units, plan.grid);
-                const int last = sk_owner((t + 1) * upt - 1, plan.units, plan.grid);
-                const int slot = static_cast<int>(blockIdx.x) - first;
-                float* part = ws_part + (static_cast<int64_t>(t) * plan.maxc + slot) * NT * sk::BMW;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) part[j * sk::BMW + row] = y[j];
-                // one thread publishes the CTA's partial (the barrier orders every
-                // thread's stores before its fence) and counts the arrival; the
-                // last arriver's thread fences again before the CTA reads the
-                // other contributors' partials
-                named_bar_sync(1, 128);
-                if (ethr == 0) {
-                    __threadfence();
-                    const uint32_t old = atomicAdd(ws_cnt + t, 1u);
-                    const bool last_one = old == static_cast<uint32_t>(last - first);
-                    if (last_one) __threadfence();
-                    misc[2] = last_one ? 1u : 0u;
-                }
-                named_bar_sync(1, 128);
-                finish = misc[2] != 0;
-                if (finish) {
-#pragma unroll
-                    for (int j = 0; j < NT; ++j) y[j] = 0.f;
-                    // all contributors' partials, CB at a time in flight, summed in slot order
-                    constexpr int CB = NT <= 16 ? 4 : (NT <= 32 ? 2 : 1);
-                    const int nc = last - first + 1;
-                    for (int c0 = 0; c0 < nc; c0 += CB) {
-                        float pv[CB][NT];
-#pragma unroll
-                        for (int cc = 0; cc < CB; ++cc) {
-                            const float* pc = ws_part + (static_cast<int64_t>(t) * plan.maxc + c0 + cc) * NT * sk::BMW;
-#pragma unroll
-                            for (int j = 0; j < NT; ++j) pv[cc][j] = (c0 + cc < nc) ? __ldcg(pc + j * sk::BMW + row) : 0.f;
-                        }
-#pragma unroll
-                        for (int cc = 0; cc < CB; ++cc) {
-                            if (c0 + cc < nc) {
-#pragma unroll
-                                for (int j = 0; j < NT; ++j) y[j] = __fadd_rn(y[j], pv[cc][j]);
-                            }
-                        }
-                    }
-                    if (ethr == 0) ws_cnt[t] = 0u;   // ready for the next call
-                }
-                named_bar_sync(1, 128);           // misc[2] is rewritten by the next tile
-            }
-            if (finish && nvalid) {
-                // SERQ term: (X[m,S] . Rq[n,:]) with Rq[n] of this lane's row
-                uint32_t rq[sk::XS_WORDS];
-#pragma unroll
-                for (int i = 0; i < sk::XS_WORDS / 2; ++i) unpack_s4x8_times16(rqp[i], rq[2 * i], rq[2 * i + 1]);
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    if (j >= p.M) break;
-                    int cc = 0;
-                    if (p.r > 0) {
-#pragma unroll
-                        for (int i = 0; i < sk::XS_WORDS; ++i)
-                            cc = __dp4a(static_cast<int>(xs_s[j * sk::XS_WORDS + i]), static_cast<int>(rq[i]), cc);
-                        cc >>= 4;
-                    }
-                    if constexpr (OUT == OUT_DEBUG) {
-                        if constexpr (!ASYM) p.dbg_acc[static_cast<int64_t>(j) * p.N + n] = static_cast<int32_t>(y[j]);
-                        if (p.r > 0) p.dbg_acc_c[static_cast<int64_t>(j) * p.N + n] = cc;
-                    } else {
-                        const float base = ASYM ? y[j] : __fmul_rn(swn, y[j]);
-                        const float v = __fmul_rn(p.sx[j], __fmaf_rn(srn, static_cast<float>(cc), base));
-                        store_one<OUT>(p.Y, static_cast<int64_t>(j) * p.N + n, v);
-                    }
-                }
-            }
-            li = le;
-        }
-    }
 
-    __syncwarp();
-    tc_fence_before();
-    __syncthreads();
-    if (warp == sk::ALLOC_WARP) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, sk::TMEM_COLS);
+        if (active) {
+            for (int d = 0; d < D; ++d) issue();
+            if (!waited) deps();
+            for (int d = 0; d < D; ++d) tok_prefetch(kb0 + d);
+            if (!tok_ready) {
+                if (!mbar_wait(tbar, 0, p.limit_ns)) kb1 = kb0;   // timeout recorded: skip the K loop
+                tok_ready = true;
+            }
+            uint32_t acc[NTT][4], ssum[NTT][4];
+            bool fresh = true;
+            int cslot = 0, cgk = kb0 % gs, cg = kb0 / gs;   // consume cursor: ring slot, place in group, group
+            for (int kb = kb0; kb < kb1; ++kb) {
+                // this thread's copies of K-block kb have landed; the warp's too after the __syncwarp
+                if (D == 8) cp_async_wait_group<7>();
+                else cp_async_wait_group<3>();
+                if constexpr (ASYM) __syncwarp();
+                const uint8_t* slot = smem + (warp * D + cslot) * dk::SLOT;
+                cslot = cslot + 1 == D ? 0 : cslot + 1;
+                const uint4 wa = *reinterpret_cast<const uint4*>(slot + lane * 16);
+                const uint4 wb = *reinterpret_cast<const uint4*>(slot + 512 + lane * 16);
+                uint32_t za = 0, sa = 0;   // fp16 bits, low half = row g
+                if constexpr (ASYM) {
+                    const uint16_t* zc = reinterpret_cast<const uint16_t*>(slot + 1024);
+                    za = zc[rowA - c0] | (static_cast<uint32_t>(zc[rowB - c0]) << 16);
+                    if constexpr (OUT != OUT_DEBUG)
+                        sa = zc[24 + rowA - c0] | (static_cast<uint32_t>(zc[24 + rowB - c0]) << 16);
+                    __syncwarp();   // every lane has read the shared chunks before the slot is refilled
+                }
+                issue();
+                tok_prefetch(kb + D);
+                // token fragments: per n-tile, the 16 (32 for 8-bit codes) bytes of token
+                // 8 nt + g at this lane's quarter of the K-block
+                uint4 tn[NTT][TOKV];
+#pragma unroll
+                for (int nt = 0; nt < NTT; ++nt) {
+                    const int m = 8 * nt + gq;
+#pragma unroll
+                    for (int v = 0; v < TOKV; ++v) {
+                        const int64_t off = kb * (A8 ? 128 : 64) + tq * (A8 ? 32 : 16) + 16 * v;
+                        if constexpr (TS) {
+                            tn[nt][v] = *reinterpret_cast<const uint4*>(tok_s + m * plan.tstride + off);
+                        } else {
+                            tn[nt][v] = m < p.M ? __ldg(reinterpret_cast<const uint4*>(p.Xq + m * xrow + off))
+                                                : make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                // A fragments of the 4 steps: unsigned codes u (per-channel: signed code + 8)
+                uint32_t af[4][4];
+                const uint32_t wA[4] = {wa.x, wa.y, wa.z, wa.w}, wB[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint32_t fa = ASYM ? wA[s] : wA[s] ^ 0x88888888u;
+                    const uint32_t fb = ASYM ? wB[s] : wB[s] ^ 0x88888888u;
+                    af[s][0] = fa & 0x0F0F0F0Fu;
+                    af[s][1] = fb & 0x0F0F0F0Fu;
+                    af[s][2] = (fa >> 4) & 0x0F0F0F0Fu;
+                    af[s][3] = (fb >> 4) & 0x0F0F0F0Fu;
+                }
+#pragma unroll
+                for (int nt = 0; nt < NTT; ++nt) {
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        uint32_t b0, b1;
+                        if constexpr (A8) {
+                            const uint4 t0v = tn[nt][0], t1v = tn[nt][TOKV - 1];
+                            const uint32_t x[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+                            tok_words8(x[2 * s], x[2 * s + 1], b0, b1);
+                        } else {
+                            const uint32_t x[4] = {tn[nt][0].x, tn[nt][0].y, tn[nt][0].z, tn[nt][0].w};
+                            unpack_s4x8_times16(x[s], b0, b1);
+                        }
+                        if (fresh && s == 0) {
+                            mma_s8_c(acc[nt], af[s], b0, b1, ASYM ? mag4 : zero4);
+                            mma_s8_c(ssum[nt], ones, b0, b1, ASYM ? mag4 : zero4);
+                        } else {
+                            mma_s8_c(acc[nt], af[s], b0, b1, acc[nt]);
+                            mma_s8_c(ssum[nt], ones, b0, b1, ssum[nt]);
+                        }
+                    }
+                }
+                fresh = false;
+                if (!gathered) gather();
+                if constexpr (ASYM) {
+                    const bool gend = ++cgk == gs;
+                    if (gend) cgk = 0;
+                    if (gend || kb + 1 == kb1) {
+                        // end of a group (or of this warp's share of it): acc - z S, scaled
+                        const float zfa = __half2float(__ushort_as_half(static_cast<uint16_t>(za & 0xFFFFu)));
+                        const float zfb = __half2float(__ushort_as_half(static_cast<uint16_t>(za >> 16)));
+                        if constexpr (OUT == OUT_DEBUG) {
+                            const int zia = static_cast<int>(zfa), zib = static_cast<int>(zfb);
+                            const int g = cg;
+#pragma unroll
+                            for (int nt = 0; nt < NTT; ++nt) {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) {
+                                    const int m = 8 * nt + 2 * tq + (v & 1);
+                                    const int n = v < 2 ? rowA : rowB;
+                                    const int sv = static_cast<int>(ssum[nt][v & 1] - dk::MAGIC);
+                                    const int a = static_cast<int>(acc[nt][v] - dk::MAGIC) - (v < 2 ? zia : zib) * sv;
+                                    if ((v < 2 ? okA : okB) && m < p.M)
+                                        atomicAdd(p.dbg_acc + (static_cast<int64_t>(m) * p.N + n) * G + g, a >> sh);
+                                }
+                            }
+                        } else {
+                            const float sfa = __half2float(__ushort_as_half(static_cast<uint16_t>(sa & 0xFFFFu))) * inv_act;
+                            const float sfb = __half2float(__ushort_as_half(static_cast<uint16_t>(sa >> 16))) * inv_act;
+                            const float2 nmag = make_float2(-dk::MAGIC_F, -dk::MAGIC_F);
+                            const float2 nza = make_float2(-zfa, -zfa), nzb = make_float2(-zfb, -zfb);
+                            const float2 s2a = make_float2(sfa, sfa), s2b = make_float2(sfb, sfb);
+#pragma unroll
+                            for (int nt = 0; nt < NTT; ++nt) {
+                                const float2 sf = __fadd2_rn(make_float2(__uint_as_float(ssum[nt][0]), __uint_as_float(ssum[nt][1])), nmag);
+                                const float2 fa = __fadd2_rn(make_float2(__uint_as_float(acc[nt][0]), __uint_as_float(acc[nt][1])), nmag);
+                                const float2 fb = __fadd2_rn(make_float2(__uint_as_float(acc[nt][2]), __uint_as_float(acc[nt][3])), nmag);
+                                const float2 ta = __ffma2_rn(nza, sf, fa);   // exact: integers below 2^24
+                                const float2 tb = __ffma2_rn(nzb, sf, fb);
+                                float2 ya = make_float2(y[nt][0], y[nt][1]), yb = make_float2(y[nt][2], y[nt][3]);
+                                ya = __ffma2_rn(s2a, ta, ya);
+                                yb = __ffma2_rn(s2b, tb, yb);
+                                y[nt][0] = ya.x;
+                                y[nt][1] = ya.y;
+                                y[nt][2] = yb.x;
+                                y[nt][3] = yb.y;
+                            }
+                        }
+                        fresh = true;
+                        if (gend) ++cg;
+                    }
+                }
+            }
+            if constexpr (!ASYM) {
+                // per-channel: signed code = u - 8, exact integer partial sums
+                if (kb1 > kb0) {
+#pragma unroll
+                    for (int nt = 0; nt < NTT; ++nt)
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            yi[nt][v] = static_cast<int32_t>(acc[nt][v]) - 8 * static_cast<int32_t>(ssum[nt][v & 1]);
+                }
+            }
+        }
+        if (!gathered) gather();
+        // ---- the warps of a tile meet: partial sums through shared memory (over the rings)
+        cp_async_wait_all();
+        __syncthreads();
+        if (active) {
+            uint32_t* part = reinterpret_cast<uint32_t*>(smem) + (warp * 32 + lane) * (NTT * 4);
+#pragma unroll
+            for (int nt = 0; nt < NTT; ++nt)
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    part[nt * 4 + v] = ASYM ? __float_as_uint(y[nt][v]) : static_cast<uint32_t>(yi[nt][v]);
+        }
+        if (pass == 0) {
+#pragma unroll
+            for (int it = 0; it < C::XITEMS; ++it) {
+                const int idx = tid + it * C::THREADS;
+                if (idx < NT * dk::XS_WORDS) xs_s[idx] = xsw[it];
+            }
+        }
+        __syncthreads();
+        // ---- finish: one (row, 4 tokens) item per thread at a time, rows fastest
+        const int rows = ntp * 16;
+        const int items = rows * (NT / 4);
+        for (int it = tid; it < items; it += C::THREADS) {
+            const int rr = it % rows, q4 = it / rows;
+            const int tle = rr >> 4, rit = rr & 15;
+            const int n = r0 + 16 * (t0 + tle) + rit;
+            if (n >= r1 || 4 * q4 >= p.M) continue;
+            uint32_t rq[dk::XS_WORDS];
+#pragma unroll
+            for (int i = 0; i < dk::XS_WORDS; ++i) rq[i] = 0;
+            if (p.r > 0) {
+                const uint32_t* src = reinterpret_cast<const uint32_t*>(rq_s + (n - pr0) * (p.r / 2));
+#pragma unroll
+                for (int i = 0; i < dk::XS_WORDS / 2; ++i)
+                    if (i < p.r / 8) unpack_s4x8_times16(src[i], rq[2 * i], rq[2 * i + 1]);
+            }
+            float swn = 0.f, srn = 0.f;
+            if constexpr (OUT != OUT_DEBUG) {
+                if constexpr (!ASYM) swn = __half2float(__ushort_as_half(sw_s[n - pb]));
+                if (p.r > 0) srn = __half2float(__ushort_as_half(sr_s[n - pb]));
+            }
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+                const int m = 4 * q4 + mm;
+                if (m >= p.M) break;
+                // partial of (row rit, token m): lane (rit % 8) * 4 + (m % 8) / 2,
+                // value (m / 8) * 4 + (rit / 8) * 2 + m % 2 of each contributing warp
+                const int pl = (rit & 7) * 4 + ((m & 7) >> 1);
+                const int pv = (m >> 3) * 4 + (rit >> 3) * 2 + (m & 1);
+                float ys = 0.f;
+                int32_t yis = 0;
+                for (int s = 0; s < S; ++s) {
+                    const uint32_t v = reinterpret_cast<const uint32_t*>(smem)[((s * ntp + tle) * 32 + pl) * (NTT * 4) + pv];
+                    if constexpr (ASYM) ys = __fadd_rn(ys, __uint_as_float(v));
+                    else yis += static_cast<int32_t>(v);
+                }
+                int cc = 0;
+                if (p.r > 0) {
+                    const uint4* xw = reinterpret_cast<const uint4*>(xs_s + m * dk::XS_WORDS);
+#pragma unroll
+                    for (int i = 0; i < dk::XS_WORDS / 4; ++i) {
+                        const uint4 x4 = xw[i];
+                        cc = __dp4a(static_cast<int>(x4.x), static_cast<int>(rq[4 * i]), cc);
+                        cc = __dp4a(static_cast<int>(x4.y), static_cast<int>(rq[4 * i + 1]), cc);
+                        cc = __dp4a(static_cast<int>(x4.z), static_cast<int>(rq[4 * i + 2]), cc);
+                        cc = __dp4a(static_cast<int>(x4.w), static_cast<int>(rq[4 * i + 3]), cc);
+                    }
+                    cc >>= 4;
+                }
+                const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                if constexpr (OUT == OUT_DEBUG) {
+                    if constexpr (!ASYM) p.dbg_acc[o] = yis >> sh;
+                    if (p.r > 0) p.dbg_acc_c[o] = cc;
+                } else {
+                    const float base = ASYM ? ys : __fmul_rn(swn, static_cast<float>(yis >> sh));
+                    store_one<OUT>(p.Y, o, __fmul_rn(sx_s[m], __fmaf_rn(srn, static_cast<float>(cc), base)));
+                }
+            }
+        }
+        __syncthreads();   // the ring is reused by the next pass
+    }
+    if constexpr (TS) {
+        // no bulk copy may still be landing when the CTA exits (after a timeout)
+        if (tid == 0) mbar_wait(tbar, 0, p.limit_ns);
     }
 }
 
 // ------------------------------------------------------------------ host side
 bool small_supported(int64_t M, int gw) {
     if (M < 1 || M > 64) return false;
-    return gw == 0 || gw / sk::BK <= sk::sb_for(nt_for(M));
+    return gw == 0 || gw % dk::BK == 0;
 }
 
-size_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int gw, int nsm) {
-    if (!small_supported(M, gw) || N <= 0 || K < sk::BK) return 0;
-    const SkPlan p = sk_plan(M, N, K, gw, nsm);
-    return small_counter_bytes(p.ntiles) + static_cast<size_t>(p.ntiles) * p.maxc * nt_for(M) * sk::BMW * sizeof(float);
-}
+size_t small_workspace_bytes(int64_t, int64_t, int64_t, int, int) { return 0; }
 
-template <int NT, bool ASYM, bool A8, int OUT>
-static hq_status launch_sk_t(const GemmArgs& a, const SkPlan& plan, cudaStream_t st) {
-    auto kern = k_gemm_small<NT, ASYM, A8, OUT>;
-    const int smem = SkSmem<NT>::ALLOC;
+template <int NT, bool ASYM, bool A8, int OUT, bool TS>
+static hq_status launch_sk_ts(const GemmArgs& a, const DkPlan& plan, cudaStream_t st) {
+    auto kern = k_gemm_small<NT, ASYM, A8, OUT, TS>;
+    const int smem = plan.ring + DkCfg<NT>::FIX + (TS ? NT * plan.tstride : 0);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
     // Programmatic dependent launch: the kernel may start while the preceding
     // kernel of the stream (normally the activation rotate/quant) is still
-    // running; it streams weights, then waits (griddepcontrol.wait) before it
-    // reads activations or writes anything.
+    // running; it requests its first weight K-blocks, then waits
+    // (griddepcontrol.wait) before it reads activations or writes anything.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.grid);
-    cfg.blockDim = dim3(sk::THREADS);
+    cfg.blockDim = dim3(DkCfg<NT>::THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -657,21 +616,34 @@ static hq_status launch_sk_t(const GemmArgs& a, const SkPlan& plan, cudaStream_t
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
+template <int NT, bool ASYM, bool A8, int OUT>
+static hq_status launch_sk_t(const GemmArgs& a, cudaStream_t st, int nsm) {
+    bool staged = false;
+    const DkPlan plan = dk_plan<NT>(a.M, a.N, a.K, A8, nsm, staged);
+    // the debug entry adds the partial group sums of the warps with atomics
+    if (OUT == OUT_DEBUG && ASYM &&
+        cudaMemsetAsync(a.dbg_acc, 0, static_cast<size_t>(a.M) * a.N * (a.K / a.gw) * sizeof(int32_t), st) !=
+            cudaSuccess)
+        return HQ_ERR_CUDA;
+    return staged ? launch_sk_ts<NT, ASYM, A8, OUT, true>(a, plan, st)
+                  : launch_sk_ts<NT, ASYM, A8, OUT, false>(a, plan, st);
+}
+
 template <int NT, bool A8>
-static hq_status launch_sk_nt(const GemmArgs& a, int out, const SkPlan& plan, cudaStream_t st) {
+static hq_status launch_sk_nt(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
     if (a.gw == 0) {
         switch (out) {
-            case HQ_F16: return launch_sk_t<NT, false, A8, HQ_F16>(a, plan, st);
-            case HQ_BF16: return launch_sk_t<NT, false, A8, HQ_BF16>(a, plan, st);
-            case HQ_F32: return launch_sk_t<NT, false, A8, HQ_F32>(a, plan, st);
-            case OUT_DEBUG: return launch_sk_t<NT, false, A8, OUT_DEBUG>(a, plan, st);
+            case HQ_F16: return launch_sk_t<NT, false, A8, HQ_F16>(a, st, nsm);
+            case HQ_BF16: return launch_sk_t<NT, false, A8, HQ_BF16>(a, st, nsm);
+            case HQ_F32: return launch_sk_t<NT, false, A8, HQ_F32>(a, st, nsm);
+            case OUT_DEBUG: return launch_sk_t<NT, false, A8, OUT_DEBUG>(a, st, nsm);
         }
     } else {
         switch (out) {
-            case HQ_F16: return launch_sk_t<NT, true, A8, HQ_F16>(a, plan, st);
-            case HQ_BF16: return launch_sk_t<NT, true, A8, HQ_BF16>(a, plan, st);
-            case HQ_F32: return launch_sk_t<NT, true, A8, HQ_F32>(a, plan, st);
-            case OUT_DEBUG: return launch_sk_t<NT, true, A8, OUT_DEBUG>(a, plan, st);
+            case HQ_F16: return launch_sk_t<NT, true, A8, HQ_F16>(a, st, nsm);
+            case HQ_BF16: return launch_sk_t<NT, true, A8, HQ_BF16>(a, st, nsm);
+            case HQ_F32: return launch_sk_t<NT, true, A8, HQ_F32>(a, st, nsm);
+            case OUT_DEBUG: return launch_sk_t<NT, true, A8, OUT_DEBUG>(a, st, nsm);
         }
     }
     return HQ_ERR_UNSUPPORTED;
@@ -679,12 +651,11 @@ static hq_status launch_sk_nt(const GemmArgs& a, int out, const SkPlan& plan, cu
 
 hq_status launch_gemm_small(const GemmArgs& a, int out, cudaStream_t st, int nsm) {
     if (!small_supported(a.M, a.gw)) return HQ_ERR_UNSUPPORTED;
-    const SkPlan plan = sk_plan(a.M, a.N, a.K, a.gw, nsm);
     const bool a8 = a.act_bits == 8;
     switch (nt_for(a.M)) {
-        case 16: return a8 ? launch_sk_nt<16, true>(a, out, plan, st) : launch_sk_nt<16, false>(a, out, plan, st);
-        case 32: return a8 ? launch_sk_nt<32, true>(a, out, plan, st) : launch_sk_nt<32, false>(a, out, plan, st);
-        default: return a8 ? launch_sk_nt<64, true>(a, out, plan, st) : launch_sk_nt<64, false>(a, out, plan, st);
+        case 16: return a8 ? launch_sk_nt<16, true>(a, out, st, nsm) : launch_sk_nt<16, false>(a, out, st, nsm);
+        case 32: return a8 ? launch_sk_nt<32, true>(a, out, st, nsm) : launch_sk_nt<32, false>(a, out, st, nsm);
+        default: return a8 ? launch_sk_nt<64, true>(a, out, st, nsm) : launch_sk_nt<64, false>(a, out, st, nsm);
     }
 }
 

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/hq.h"
@@ -39,6 +40,8 @@ inline size_t small_counter_bytes_for_n(int64_t N) { return small_counter_bytes(
 hq_status check_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
                        const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,
                        const uint16_t* B, const int32_t* sal_idx, int32_t r, void* Y, hq_dtype yt);
+hq_status make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle swz);
 hq_status launch_gemm_prefill(const GemmArgs& a, int out, cudaStream_t st, int nsm);
 hq_status launch_gemm_small(const GemmArgs& a, int out, cudaStream_t st, int nsm);
 size_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int gw, int nsm);
