@@ -33,10 +33,12 @@
 //    of one packed 32-bit word of 8 codes (inputs k0 k2 k4 k6 / k1 k3 k5 k7),
 //    the same for weights and tokens, so expanding a word to the A or B
 //    fragment is a mask and a shift, and the dot product is unchanged.
-//  * zero points: weights enter the MMA as their unsigned codes u (0..15); a
-//    second MMA with an all-ones A fragment gives each token's code sum S over
-//    the same inputs, and a group's accumulator is acc - z * S (per-channel
-//    weights: z = 8, the offset of the signed codes).
+//  * zero points: weights enter the MMA as their unsigned codes u (0..15), and
+//    a group's accumulator is acc - z * S with S the token's code sum over the
+//    same inputs (per-channel weights: z = 8, the offset of the signed codes).
+//    With the tokens staged in shared memory, the CTA sums each token's codes
+//    per K-block once; otherwise a second MMA with an all-ones A fragment
+//    gives S.
 //  * group accumulators start from the bits of 1.5 * 2^23, so at the end of a
 //    group the int32 result reads as an exact float offset by that constant:
 //    one packed add, then packed fmas for - z * S and the scale sw[b][n].
@@ -95,9 +97,10 @@ struct DkPlan {
     int D;         // K-blocks in flight per warp (8 or 4)
     int ring;      // bytes of the rings (W x D slots)
     int tstride;   // bytes per staged token row (row bytes + 64)
+    int tbytes;    // bytes of the staged tokens and their sums (0 when not staged)
 };
 
-static int nt_for(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+static int nt_for(int64_t M) { return M <= 8 ? 8 : (M <= 16 ? 16 : (M <= 32 ? 32 : 64)); }
 
 // Launch plan; `staged` tells whether the tokens fit in shared memory.
 template <int NT>
@@ -108,17 +111,20 @@ static DkPlan dk_plan(int64_t M, int64_t N, int64_t K, bool a8, int nsm, bool& s
     const int64_t tiles = (N + 15) / 16;   // at least one 16-row tile per CTA
     p.grid = static_cast<int>(tiles < want ? tiles : want);
     p.tstride = static_cast<int>(a8 ? K : K / 2) + 64;
-    const int64_t tok = static_cast<int64_t>(NT) * p.tstride;
+    // staged token rows, then their code sums per K-block (int32 [K/128][NT])
+    const int64_t tok = static_cast<int64_t>(NT) * p.tstride + (K / dk::BK) * NT * 4;
     staged = true;
     for (int d : {dk::DMAX, 4}) {
         const int64_t ring = static_cast<int64_t>(C::W) * d * dk::SLOT;
         if (ring >= C::PART && ring + C::FIX + tok <= dk::SMEM_MAX) {
             p.D = d;
             p.ring = static_cast<int>(ring);
+            p.tbytes = static_cast<int>(tok);
             return p;
         }
     }
     staged = false;
+    p.tbytes = 0;
     p.D = dk::DMAX;
     p.ring = C::W * dk::DMAX * dk::SLOT;
     return p;
@@ -170,6 +176,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
     const uint16_t* sw_s = reinterpret_cast<const uint16_t*>(fix + C::F_SW);
     float* sx_s = reinterpret_cast<float*>(fix + C::F_SX);
     uint8_t* tok_s = fix + C::FIX;
+    int32_t* tsum_s = reinterpret_cast<int32_t*>(tok_s + NT * plan.tstride);   // [K/128][NT]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
     const int cta = blockIdx.x;
@@ -209,15 +216,8 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int j = 8 * i + 2 * e + hh;
-            int k = -1;
-            if (idx < NT * dk::XS_WORDS && m < p.M && j < p.r) {
-                k = __ldg(p.sal + j);
-                if (static_cast<unsigned>(k) >= static_cast<unsigned>(p.K)) {
-                    record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
-                    k = -1;
-                }
-            }
-            salk[it][e] = k;
+            // (checked when used: a test here would wait for the load)
+            salk[it][e] = (idx < NT * dk::XS_WORDS && m < p.M && j < p.r) ? __ldg(p.sal + j) : -1;
         }
     }
     uint32_t xsw[C::XITEMS];
@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int k = salk[it][e];
-                if (k >= 0) {
+                if (k >= p.K) record_status(HQ_ERR_ARG);   // a salient index outside [0, K): skipped
+                if (k >= 0 && k < p.K) {
                     const uint8_t* xr = p.Xq + static_cast<int64_t>(m) * xrow;
                     if constexpr (A8) {
                         word |= static_cast<uint32_t>(__ldg(xr + k)) << (8 * e);
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
     const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
     const uint32_t zero4[4] = {0u, 0u, 0u, 0u};
     const uint32_t mag4[4] = {dk::MAGIC, dk::MAGIC, dk::MAGIC, dk::MAGIC};
-    bool tok_ready = !TS;
+    bool tok_ready = !TS;   // (pass 0 of the active warps: tokens landed and summed)
 
     const int npass = (RT + W - 1) / W;
     for (int pass = 0; pass < npass; ++pass) {
@@ -354,14 +355,40 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
         };
 
         if (active) {
+            if (warp == 0 && !waited) deps();   // the tokens are on every warp's critical path
             for (int d = 0; d < D; ++d) issue();
             if (!waited) deps();
             for (int d = 0; d < D; ++d) tok_prefetch(kb0 + d);
             if (!tok_ready) {
                 if (!mbar_wait(tbar, 0, p.limit_ns)) kb1 = kb0;   // timeout recorded: skip the K loop
+                // each token's code sum per K-block (16 sum q for 4-bit codes),
+                // shared by the warps of this pass (a prefix of the CTA's warps)
+                const int nact = S * ntp * 32;
+                for (int idx = tid; idx < KB * NT; idx += nact) {
+                    const int kbs = idx / NT, m = idx - kbs * NT;
+                    const uint4* src = reinterpret_cast<const uint4*>(tok_s + m * plan.tstride + kbs * (A8 ? 128 : 64));
+                    int sum = 0;
+#pragma unroll
+                    for (int c = 0; c < (A8 ? 8 : 4); ++c) {
+                        const uint4 v = src[c];
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            if constexpr (A8) {
+                                sum = __dp4a(static_cast<int>(w[e]), 0x01010101, sum);
+                            } else {
+                                const uint32_t u = w[e] ^ 0x88888888u;   // q + 8 per nibble
+                                sum = __dp4a(static_cast<int>((u & 0x0F0F0F0Fu) + ((u >> 4) & 0x0F0F0F0Fu)), 0x01010101, sum);
+                            }
+                        }
+                    }
+                    tsum_s[idx] = A8 ? sum : 16 * (sum - 8 * dk::BK);
+                }
+                named_bar_sync(1, nact);
                 tok_ready = true;
             }
             uint32_t acc[NTT][4], ssum[NTT][4];
+            int32_t sacc[NTT][2];   // token sums of this warp's share of the current group (staged tokens)
             bool fresh = true;
             int cslot = 0, cgk = kb0 % gs, cg = kb0 / gs;   // consume cursor: ring slot, place in group, group
             for (int kb = kb0; kb < kb1; ++kb) {
@@ -427,11 +454,16 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                         }
                         if (fresh && s == 0) {
                             mma_s8_c(acc[nt], af[s], b0, b1, ASYM ? mag4 : zero4);
-                            mma_s8_c(ssum[nt], ones, b0, b1, ASYM ? mag4 : zero4);
+                            if constexpr (!TS) mma_s8_c(ssum[nt], ones, b0, b1, ASYM ? mag4 : zero4);
                         } else {
                             mma_s8_c(acc[nt], af[s], b0, b1, acc[nt]);
-                            mma_s8_c(ssum[nt], ones, b0, b1, ssum[nt]);
+                            if constexpr (!TS) mma_s8_c(ssum[nt], ones, b0, b1, ssum[nt]);
                         }
+                    }
+                    if constexpr (TS) {
+                        const int2 sv = *reinterpret_cast<const int2*>(tsum_s + kb * NT + 8 * nt + 2 * tq);
+                        sacc[nt][0] = (fresh ? 0 : sacc[nt][0]) + sv.x;
+                        sacc[nt][1] = (fresh ? 0 : sacc[nt][1]) + sv.y;
                     }
                 }
                 fresh = false;
@@ -452,7 +484,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                                 for (int v = 0; v < 4; ++v) {
                                     const int m = 8 * nt + 2 * tq + (v & 1);
                                     const int n = v < 2 ? rowA : rowB;
-                                    const int sv = static_cast<int>(ssum[nt][v & 1] - dk::MAGIC);
+                                    const int sv = TS ? sacc[nt][v & 1] : static_cast<int>(ssum[nt][v & 1] - dk::MAGIC);
                                     const int a = static_cast<int>(acc[nt][v] - dk::MAGIC) - (v < 2 ? zia : zib) * sv;
                                     if ((v < 2 ? okA : okB) && m < p.M)
                                         atomicAdd(p.dbg_acc + (static_cast<int64_t>(m) * p.N + n) * G + g, a >> sh);
@@ -466,7 +498,8 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                             const float2 s2a = make_float2(sfa, sfa), s2b = make_float2(sfb, sfb);
 #pragma unroll
                             for (int nt = 0; nt < NTT; ++nt) {
-                                const float2 sf = __fadd2_rn(make_float2(__uint_as_float(ssum[nt][0]), __uint_as_float(ssum[nt][1])), nmag);
+                                const float2 sf = TS ? make_float2(static_cast<float>(sacc[nt][0]), static_cast<float>(sacc[nt][1]))
+                                                     : __fadd2_rn(make_float2(__uint_as_float(ssum[nt][0]), __uint_as_float(ssum[nt][1])), nmag);
                                 const float2 fa = __fadd2_rn(make_float2(__uint_as_float(acc[nt][0]), __uint_as_float(acc[nt][1])), nmag);
                                 const float2 fb = __fadd2_rn(make_float2(__uint_as_float(acc[nt][2]), __uint_as_float(acc[nt][3])), nmag);
                                 const float2 ta = __ffma2_rn(nza, sf, fa);   // exact: integers below 2^24
@@ -492,7 +525,8 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                     for (int nt = 0; nt < NTT; ++nt)
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
-                            yi[nt][v] = static_cast<int32_t>(acc[nt][v]) - 8 * static_cast<int32_t>(ssum[nt][v & 1]);
+                            yi[nt][v] = static_cast<int32_t>(acc[nt][v]) -
+                                        8 * (TS ? sacc[nt][v & 1] : static_cast<int32_t>(ssum[nt][v & 1]));
                 }
             }
         }
@@ -501,12 +535,12 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
         cp_async_wait_all();
         __syncthreads();
         if (active) {
-            uint32_t* part = reinterpret_cast<uint32_t*>(smem) + (warp * 32 + lane) * (NTT * 4);
+            uint4* part = reinterpret_cast<uint4*>(smem) + (warp * 32 + lane) * NTT;
 #pragma unroll
             for (int nt = 0; nt < NTT; ++nt)
-#pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    part[nt * 4 + v] = ASYM ? __float_as_uint(y[nt][v]) : static_cast<uint32_t>(yi[nt][v]);
+                part[nt] = ASYM ? make_uint4(__float_as_uint(y[nt][0]), __float_as_uint(y[nt][1]), __float_as_uint(y[nt][2]),
+                                             __float_as_uint(y[nt][3]))
+                                : make_uint4(yi[nt][0], yi[nt][1], yi[nt][2], yi[nt][3]);
         }
         if (pass == 0) {
 #pragma unroll
@@ -516,63 +550,77 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
             }
         }
         __syncthreads();
-        // ---- finish: one (row, 4 tokens) item per thread at a time, rows fastest
-        const int rows = ntp * 16;
-        const int items = rows * (NT / 4);
-        for (int it = tid; it < items; it += C::THREADS) {
-            const int rr = it % rows, q4 = it / rows;
-            const int tle = rr >> 4, rit = rr & 15;
-            const int n = r0 + 16 * (t0 + tle) + rit;
-            if (n >= r1 || 4 * q4 >= p.M) continue;
-            uint32_t rq[dk::XS_WORDS];
+        // ---- finish: warp w < ntp completes tile w in its own fragment layout
+        if (warp < ntp) {
+            // partial sums of the tile's warps, added in warp order
 #pragma unroll
-            for (int i = 0; i < dk::XS_WORDS; ++i) rq[i] = 0;
-            if (p.r > 0) {
-                const uint32_t* src = reinterpret_cast<const uint32_t*>(rq_s + (n - pr0) * (p.r / 2));
+            for (int nt = 0; nt < NTT; ++nt) {
+                float ys[4] = {0.f, 0.f, 0.f, 0.f};
+                int32_t yis[4] = {0, 0, 0, 0};
+                for (int sidx = 0; sidx < S; ++sidx) {
+                    const uint4 v = reinterpret_cast<const uint4*>(smem)[((sidx * ntp + warp) * 32 + lane) * NTT + nt];
+                    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int i = 0; i < dk::XS_WORDS / 2; ++i)
-                    if (i < p.r / 8) unpack_s4x8_times16(src[i], rq[2 * i], rq[2 * i + 1]);
-            }
-            float swn = 0.f, srn = 0.f;
-            if constexpr (OUT != OUT_DEBUG) {
-                if constexpr (!ASYM) swn = __half2float(__ushort_as_half(sw_s[n - pb]));
-                if (p.r > 0) srn = __half2float(__ushort_as_half(sr_s[n - pb]));
-            }
-#pragma unroll
-            for (int mm = 0; mm < 4; ++mm) {
-                const int m = 4 * q4 + mm;
-                if (m >= p.M) break;
-                // partial of (row rit, token m): lane (rit % 8) * 4 + (m % 8) / 2,
-                // value (m / 8) * 4 + (rit / 8) * 2 + m % 2 of each contributing warp
-                const int pl = (rit & 7) * 4 + ((m & 7) >> 1);
-                const int pv = (m >> 3) * 4 + (rit >> 3) * 2 + (m & 1);
-                float ys = 0.f;
-                int32_t yis = 0;
-                for (int s = 0; s < S; ++s) {
-                    const uint32_t v = reinterpret_cast<const uint32_t*>(smem)[((s * ntp + tle) * 32 + pl) * (NTT * 4) + pv];
-                    if constexpr (ASYM) ys = __fadd_rn(ys, __uint_as_float(v));
-                    else yis += static_cast<int32_t>(v);
-                }
-                int cc = 0;
-                if (p.r > 0) {
-                    const uint4* xw = reinterpret_cast<const uint4*>(xs_s + m * dk::XS_WORDS);
-#pragma unroll
-                    for (int i = 0; i < dk::XS_WORDS / 4; ++i) {
-                        const uint4 x4 = xw[i];
-                        cc = __dp4a(static_cast<int>(x4.x), static_cast<int>(rq[4 * i]), cc);
-                        cc = __dp4a(static_cast<int>(x4.y), static_cast<int>(rq[4 * i + 1]), cc);
-                        cc = __dp4a(static_cast<int>(x4.z), static_cast<int>(rq[4 * i + 2]), cc);
-                        cc = __dp4a(static_cast<int>(x4.w), static_cast<int>(rq[4 * i + 3]), cc);
+                    for (int j = 0; j < 4; ++j) {
+                        if constexpr (ASYM) ys[j] = __fadd_rn(ys[j], __uint_as_float(vv[j]));
+                        else yis[j] += static_cast<int32_t>(vv[j]);
                     }
-                    cc >>= 4;
                 }
-                const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                if constexpr (OUT == OUT_DEBUG) {
-                    if constexpr (!ASYM) p.dbg_acc[o] = yis >> sh;
-                    if (p.r > 0) p.dbg_acc_c[o] = cc;
-                } else {
-                    const float base = ASYM ? ys : __fmul_rn(swn, static_cast<float>(yis >> sh));
-                    store_one<OUT>(p.Y, o, __fmul_rn(sx_s[m], __fmaf_rn(srn, static_cast<float>(cc), base)));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    y[nt][j] = ys[j];
+                    yi[nt][j] = yis[j];
+                }
+            }
+            // SERQ term X[m,S] . Rq[n,:] for rows g, g + 8 and the n-tiles' tokens:
+            // one or two 32-input MMA steps; lane t takes packed word 4 s + t of
+            // the Rq rows (A, 16 q) and the matching lo/hi words of X[m,S] (B)
+            const int rw = p.r / 8;   // packed Rq words per row
+            const int nA = r0 + 16 * (t0 + warp) + gq, nB = nA + 8;
+            uint32_t cc[NTT][4];
+#pragma unroll
+            for (int nt = 0; nt < NTT; ++nt) cc[nt][0] = cc[nt][1] = cc[nt][2] = cc[nt][3] = 0;
+            if (p.r > 0) {
+                const uint32_t* rqA = reinterpret_cast<const uint32_t*>(rq_s + (nA - pr0) * (p.r / 2));
+                const uint32_t* rqB = reinterpret_cast<const uint32_t*>(rq_s + (nB - pr0) * (p.r / 2));
+#pragma unroll
+                for (int st = 0; st < 2; ++st) {
+                    const int wi = 4 * st + tq;
+                    if (4 * st >= rw) break;
+                    const bool has = wi < rw;
+                    const uint32_t qa = has && nA < pr1 ? rqA[wi] : 0u;   // (two's complement nibbles)
+                    const uint32_t qb = has && nB < pr1 ? rqB[wi] : 0u;
+                    uint32_t a[4];
+                    unpack_s4x8_times16(qa, a[0], a[2]);
+                    unpack_s4x8_times16(qb, a[1], a[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NTT; ++nt) {
+                        const int m = 8 * nt + gq;
+                        const uint32_t b0 = has ? xs_s[m * dk::XS_WORDS + 2 * wi] : 0u;
+                        const uint32_t b1 = has ? xs_s[m * dk::XS_WORDS + 2 * wi + 1] : 0u;
+                        mma_s8_c(cc[nt], a, b0, b1, cc[nt]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NTT; ++nt) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int m = 8 * nt + 2 * tq + (j & 1);
+                    const int n = j < 2 ? nA : nB;
+                    if (n >= pr1 || m >= p.M) continue;
+                    const int c = static_cast<int32_t>(cc[nt][j]) >> 4;
+                    const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                    if constexpr (OUT == OUT_DEBUG) {
+                        if constexpr (!ASYM) p.dbg_acc[o] = yi[nt][j] >> sh;
+                        if (p.r > 0) p.dbg_acc_c[o] = c;
+                    } else {
+                        const float srn = p.r > 0 ? __half2float(__ushort_as_half(sr_s[n - pb])) : 0.f;
+                        const float base = ASYM ? y[nt][j]
+                                                : __fmul_rn(__half2float(__ushort_as_half(sw_s[n - pb])),
+                                                            static_cast<float>(yi[nt][j] >> sh));
+                        store_one<OUT>(p.Y, o, __fmul_rn(sx_s[m], __fmaf_rn(srn, static_cast<float>(c), base)));
+                    }
                 }
             }
         }
@@ -595,7 +643,7 @@ size_t small_workspace_bytes(int64_t, int64_t, int64_t, int, int) { return 0; }
 template <int NT, bool ASYM, bool A8, int OUT, bool TS>
 static hq_status launch_sk_ts(const GemmArgs& a, const DkPlan& plan, cudaStream_t st) {
     auto kern = k_gemm_small<NT, ASYM, A8, OUT, TS>;
-    const int smem = plan.ring + DkCfg<NT>::FIX + (TS ? NT * plan.tstride : 0);
+    const int smem = plan.ring + DkCfg<NT>::FIX + plan.tbytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
     // Programmatic dependent launch: the kernel may start while the preceding
@@ -653,6 +701,7 @@ hq_status launch_gemm_small(const GemmArgs& a, int out, cudaStream_t st, int nsm
     if (!small_supported(a.M, a.gw)) return HQ_ERR_UNSUPPORTED;
     const bool a8 = a.act_bits == 8;
     switch (nt_for(a.M)) {
+        case 8: return a8 ? launch_sk_nt<8, true>(a, out, st, nsm) : launch_sk_nt<8, false>(a, out, st, nsm);
         case 16: return a8 ? launch_sk_nt<16, true>(a, out, st, nsm) : launch_sk_nt<16, false>(a, out, st, nsm);
         case 32: return a8 ? launch_sk_nt<32, true>(a, out, st, nsm) : launch_sk_nt<32, false>(a, out, st, nsm);
         default: return a8 ? launch_sk_nt<64, true>(a, out, st, nsm) : launch_sk_nt<64, false>(a, out, st, nsm);
