@@ -64,11 +64,9 @@ namespace hq {
 
 namespace dk {
 constexpr int BK = 128;                  // inputs per K-block
-constexpr int DMAX = 8;                  // K-blocks in flight per warp (8, or 4 to make room for the tokens)
-constexpr int SLOT = 1152;               // one warp's K-block: 2 rows x 32 threads x 16 bytes, then
-                                         // 3 + 3 chunks of 8 zero points / scales
+constexpr int TSLOT = 1152;              // one tile's share of a warp's K-block: 2 rows x 32 threads x
+                                         // 16 bytes, then 3 + 3 chunks of 8 zero points / scales
 constexpr int SMEM_MAX = 232448;         // opt-in dynamic shared memory per block
-constexpr int MAXROWS = 256;             // rows of one pass: 16 warps x 16
 constexpr int XS_WORDS = 16;             // salient codes per token as int8 words (r <= 64)
 constexpr uint32_t MAGIC = 0x4B400000u;  // bits of the float 1.5 * 2^23
 constexpr float MAGIC_F = 12582912.0f;
@@ -77,24 +75,27 @@ constexpr float MAGIC_F = 12582912.0f;
 template <int NT>
 struct DkCfg {
     static constexpr int W = NT == 64 ? 8 : (NT == 32 ? 12 : 16);   // warps
+    static constexpr int TPW = 1;                            // 16-row tiles per warp (2 measured slower)
     static constexpr int THREADS = 32 * W;
     static constexpr int NTT = NT / 8;                       // MMA n-tiles of 8 tokens
-    static constexpr int PART = W * 32 * NTT * 4 * 4;        // partial sums, aliased onto the ring
-    // after the ring: the token barrier, salient codes, the pass's SERQ rows Rq
-    // (r/2 bytes each), sr and sw (fp16 pairs from an even row), and sx
+    static constexpr int SLOT = TPW * dk::TSLOT;             // bytes of one warp's K-block in its ring
+    static constexpr int PART = W * 32 * TPW * NTT * 16;     // partial sums, aliased onto the rings
+    static constexpr int MAXROWS = W * TPW * 16;             // rows of one pass
+    // after the rings: the token barrier, salient codes, the pass's SERQ rows
+    // Rq (r/2 bytes each), sr and sw (fp16 pairs from an even row), and sx
     static constexpr int F_BAR = 0;
     static constexpr int F_XS = 16;
     static constexpr int F_RQ = F_XS + NT * dk::XS_WORDS * 4;
-    static constexpr int F_SR = F_RQ + dk::MAXROWS * 32;
-    static constexpr int F_SW = F_SR + (dk::MAXROWS + 8) * 2;
-    static constexpr int F_SX = F_SW + (dk::MAXROWS + 8) * 2;
+    static constexpr int F_SR = F_RQ + MAXROWS * 32;
+    static constexpr int F_SW = F_SR + (MAXROWS + 8) * 2;
+    static constexpr int F_SX = F_SW + (MAXROWS + 8) * 2;
     static constexpr int FIX = (F_SX + NT * 4 + 15) / 16 * 16;
     static constexpr int XITEMS = (NT * dk::XS_WORDS + THREADS - 1) / THREADS;
 };
 
 struct DkPlan {
     int grid;      // CTAs; CTA c owns weight rows [c N / grid, (c + 1) N / grid)
-    int D;         // K-blocks in flight per warp (8 or 4)
+    int D;         // K-blocks in flight per warp (8, 4 or 2)
     int ring;      // bytes of the rings (W x D slots)
     int tstride;   // bytes per staged token row (row bytes + 64)
     int tbytes;    // bytes of the staged tokens and their sums (0 when not staged)
@@ -113,20 +114,22 @@ static DkPlan dk_plan(int64_t M, int64_t N, int64_t K, bool a8, int nsm, bool& s
     p.tstride = static_cast<int>(a8 ? K : K / 2) + 64;
     // staged token rows, then their code sums per K-block (int32 [K/128][NT])
     const int64_t tok = static_cast<int64_t>(NT) * p.tstride + (K / dk::BK) * NT * 4;
-    staged = true;
-    for (int d : {dk::DMAX, 4}) {
-        const int64_t ring = static_cast<int64_t>(C::W) * d * dk::SLOT;
-        if (ring >= C::PART && ring + C::FIX + tok <= dk::SMEM_MAX) {
-            p.D = d;
-            p.ring = static_cast<int>(ring);
-            p.tbytes = static_cast<int>(tok);
-            return p;
+    const int depths[3] = {8, 4, 2};
+    for (int st = 1; st >= 0; --st) {
+        for (int d : depths) {
+            if (st && d < 4 && C::TPW == 1) continue;
+            const int64_t ring = static_cast<int64_t>(C::W) * d * C::SLOT;
+            if (ring >= C::PART && ring + C::FIX + (st ? tok : 0) <= dk::SMEM_MAX) {
+                staged = st != 0;
+                p.D = d;
+                p.ring = static_cast<int>(ring);
+                p.tbytes = st ? static_cast<int>(tok) : 0;
+                return p;
+            }
         }
     }
     staged = false;
-    p.tbytes = 0;
-    p.D = dk::DMAX;
-    p.ring = C::W * dk::DMAX * dk::SLOT;
+    p.D = 0;   // nothing fits (not reached for the supported shapes)
     return p;
 }
 
@@ -159,6 +162,12 @@ __device__ __forceinline__ void tok_words8(uint32_t x0, uint32_t x1, uint32_t& l
     hi = __byte_perm(x0, x1, 0x7531);
 }
 
+__device__ __forceinline__ void cp_async_wait_depth(int D) {
+    if (D == 8) cp_async_wait_group<7>();
+    else if (D == 4) cp_async_wait_group<3>();
+    else cp_async_wait_group<1>();
+}
+
 // A8: 8-bit activation codes ([M][K] int8, used as they are) instead of packed
 // 4-bit codes (expanded as 16 q).  TS: tokens staged in shared memory.
 template <int NT, bool ASYM, bool A8, int OUT, bool TS>
@@ -166,6 +175,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
     using C = DkCfg<NT>;
     constexpr int NTT = C::NTT;
     constexpr int W = C::W;
+    constexpr int TPW = C::TPW;
     constexpr int TOKV = A8 ? 2 : 1;                   // uint4 per token fragment and K-block
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* fix = smem + plan.ring;
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
     const int cta = blockIdx.x;
     const int r0 = static_cast<int>(static_cast<long long>(cta) * p.N / plan.grid);
     const int r1 = static_cast<int>(static_cast<long long>(cta + 1) * p.N / plan.grid);
-    const int RT = (r1 - r0 + 15) / 16;
+    const int RG = (r1 - r0 + 16 * TPW - 1) / (16 * TPW);   // groups of TPW 16-row tiles
     const int KB = p.K / dk::BK;
     const int gs = ASYM ? p.gw / dk::BK : KB;         // K-blocks per weight group
     const int G = ASYM ? p.K / p.gw : 1;
@@ -264,27 +274,36 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
         gathered = true;
     };
 
-    const uint32_t ring = smem_u32(smem + warp * D * dk::SLOT);
+    const uint32_t ring = smem_u32(smem + warp * D * C::SLOT);
     const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
     const uint32_t zero4[4] = {0u, 0u, 0u, 0u};
     const uint32_t mag4[4] = {dk::MAGIC, dk::MAGIC, dk::MAGIC, dk::MAGIC};
     bool tok_ready = !TS;   // (pass 0 of the active warps: tokens landed and summed)
 
-    const int npass = (RT + W - 1) / W;
+    const int npass = (RG + W - 1) / W;
     for (int pass = 0; pass < npass; ++pass) {
-        const int t0 = pass * W;
-        const int ntp = (RT - t0) < W ? (RT - t0) : W;   // tiles of this pass
-        const int S = W / ntp;                           // warps per tile
+        const int t0 = pass * W;                         // first group of the pass
+        const int ntp = (RG - t0) < W ? (RG - t0) : W;   // groups of this pass
+        const int S = W / ntp;                           // warps per group
         const int tl = warp % ntp, sp = warp / ntp;
         const bool active = sp < S;
-        const int base = r0 + 16 * (t0 + tl);            // the warp's first row
-        const int rowA = base + gq, rowB = rowA + 8;
-        const bool okA = rowA < r1, okB = rowB < r1;
-        const int c0 = base & ~7;                        // first of the 8-row chunks of zero points / scales
+        const int gbase = r0 + 16 * TPW * (t0 + tl);     // the warp's first row
+        // rows g and g + 8 of each of the warp's tiles
+        int rowA[TPW], rowB[TPW], c0[TPW];
+        bool okA[TPW], okB[TPW];
+#pragma unroll
+        for (int j = 0; j < TPW; ++j) {
+            rowA[j] = gbase + 16 * j + gq;
+            rowB[j] = rowA[j] + 8;
+            okA[j] = rowA[j] < r1;
+            okB[j] = rowB[j] < r1;
+            c0[j] = (gbase + 16 * j) & ~7;               // first of the tile's 8-row chunks of zero points / scales
+        }
         // the finish's operands of this pass's rows [pr0, pr1), in flight during the K loop:
         // Rq rows (r/2 bytes each, a multiple of 4), and the fp16 pairs of sr and
         // (per-channel) sw from the even row pb = pr0 & ~1
-        const int pr0 = r0 + 16 * t0, pr1 = (r0 + 16 * (t0 + ntp)) < r1 ? r0 + 16 * (t0 + ntp) : r1;
+        const int pr0 = r0 + 16 * TPW * t0;
+        const int pr1 = (r0 + 16 * TPW * (t0 + ntp)) < r1 ? r0 + 16 * TPW * (t0 + ntp) : r1;
         const int pb = pr0 & ~1;
         {
             const int nrq = (pr1 - pr0) * (p.r / 8);
@@ -301,41 +320,55 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
         const int kb0 = static_cast<int>(static_cast<long long>(sp) * KB / S);
         int kb1 = active ? static_cast<int>(static_cast<long long>(sp + 1) * KB / S) : kb0;
         // partial sums of this warp's K range, in the m16n8 accumulator layout:
-        // [nt][0,1] = row g, tokens 8 nt + 2 t + {0,1}; [nt][2,3] = row g + 8
-        float y[NTT][4];
-        int32_t yi[NTT][4];
+        // [j][nt][0,1] = tile j row g, tokens 8 nt + 2 t + {0,1}; [j][nt][2,3] = row g + 8
+        float y[TPW][NTT][4];
+        int32_t yi[TPW][NTT][4];
 #pragma unroll
-        for (int nt = 0; nt < NTT; ++nt)
+        for (int j = 0; j < TPW; ++j)
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                y[nt][v] = 0.f;
-                yi[nt][v] = 0;
-            }
+            for (int nt = 0; nt < NTT; ++nt)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    y[j][nt][v] = 0.f;
+                    yi[j][nt][v] = 0;
+                }
         // request cursor: next K-block, its ring slot, its sources (one weight tile
         // after another: consecutive K-blocks of a row are 8 KB apart)
         int ik = kb0, islot = 0, igk = kb0 % gs;
-        const uint8_t* srcA = p.Wq + (static_cast<int64_t>(rowA >> 7) * KB + kb0) * 8192 + (rowA & 127) * 64 + tq * 16;
-        const uint8_t* srcB = p.Wq + (static_cast<int64_t>(rowB >> 7) * KB + kb0) * 8192 + (rowB & 127) * 64 + tq * 16;
-        // zero points (lanes 0-2) and scales (3-5) of rows [c0, c0 + 24) of the
-        // group: 16-byte chunks of 8 rows (N % 8 == 0)
-        const int zj = lane < 3 ? lane : lane - 3;
-        const bool zlane = ASYM && lane < (OUT == OUT_DEBUG ? 3 : 6) && c0 + 8 * zj < p.N;
+        const uint8_t* srcA[TPW];
+        const uint8_t* srcB[TPW];
+#pragma unroll
+        for (int j = 0; j < TPW; ++j) {
+            srcA[j] = p.Wq + (static_cast<int64_t>(rowA[j] >> 7) * KB + kb0) * 8192 + (rowA[j] & 127) * 64 + tq * 16;
+            srcB[j] = p.Wq + (static_cast<int64_t>(rowB[j] >> 7) * KB + kb0) * 8192 + (rowB[j] & 127) * 64 + tq * 16;
+        }
+        // zero points and scales of rows [c0, c0 + 24) of the group, per tile: lane
+        // 6 j + 0..2 copies zero-point chunk 0..2 of tile j, 6 j + 3..5 its scale
+        // chunks (16-byte chunks of 8 rows; N % 8 == 0)
+        const int zt = lane / 6, zl = lane % 6, zj = zl < 3 ? zl : zl - 3;
+        const int zc0 = zt < TPW ? c0[zt < TPW ? zt : 0] : 0;
+        const bool zlane = ASYM && zt < TPW && zl < (OUT == OUT_DEBUG ? 3 : 6) && zc0 + 8 * zj < p.N;
         const uint16_t* zsrc = nullptr;
-        if constexpr (ASYM) zsrc = (lane < 3 || OUT == OUT_DEBUG ? p.zw : p.sw) + static_cast<int64_t>(kb0 / gs) * p.N + c0 + 8 * zj;
+        if constexpr (ASYM)
+            zsrc = (zl < 3 || OUT == OUT_DEBUG ? p.zw : p.sw) + static_cast<int64_t>(kb0 / gs) * p.N + zc0 + 8 * zj;
+        const uint32_t zdst = static_cast<uint32_t>(1024 * TPW + 96 * zt + 48 * (zl / 3) + 16 * zj);
         auto issue = [&]() {
             if (ik < kb1) {
-                const uint32_t slot = ring + static_cast<uint32_t>(islot) * dk::SLOT;
-                if (okA) cp_async16(slot + lane * 16, srcA);
-                if (okB) cp_async16(slot + 512 + lane * 16, srcB);
+                const uint32_t slot = ring + static_cast<uint32_t>(islot) * C::SLOT;
+#pragma unroll
+                for (int j = 0; j < TPW; ++j) {
+                    if (okA[j]) cp_async16(slot + 1024 * j + lane * 16, srcA[j]);
+                    if (okB[j]) cp_async16(slot + 1024 * j + 512 + lane * 16, srcB[j]);
+                    srcA[j] += 8192;
+                    srcB[j] += 8192;
+                }
                 if constexpr (ASYM) {
-                    if (zlane) cp_async16(slot + 1024 + 48 * (lane / 3) + 16 * zj, zsrc);
+                    if (zlane) cp_async16(slot + zdst, zsrc);
                     if (++igk == gs) {
                         igk = 0;
                         zsrc += p.N;
                     }
                 }
-                srcA += 8192;
-                srcB += 8192;
                 ++ik;
                 islot = islot + 1 == D ? 0 : islot + 1;
             }
@@ -387,27 +420,31 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                 named_bar_sync(1, nact);
                 tok_ready = true;
             }
-            uint32_t acc[NTT][4], ssum[NTT][4];
+            uint32_t acc[TPW][NTT][4], ssum[NTT][4];
             int32_t sacc[NTT][2];   // token sums of this warp's share of the current group (staged tokens)
             bool fresh = true;
             int cslot = 0, cgk = kb0 % gs, cg = kb0 / gs;   // consume cursor: ring slot, place in group, group
             for (int kb = kb0; kb < kb1; ++kb) {
                 // this thread's copies of K-block kb have landed; the warp's too after the __syncwarp
-                if (D == 8) cp_async_wait_group<7>();
-                else cp_async_wait_group<3>();
+                cp_async_wait_depth(D);
                 if constexpr (ASYM) __syncwarp();
-                const uint8_t* slot = smem + (warp * D + cslot) * dk::SLOT;
+                const uint8_t* slot = smem + (warp * D + cslot) * C::SLOT;
                 cslot = cslot + 1 == D ? 0 : cslot + 1;
-                const uint4 wa = *reinterpret_cast<const uint4*>(slot + lane * 16);
-                const uint4 wb = *reinterpret_cast<const uint4*>(slot + 512 + lane * 16);
-                uint32_t za = 0, sa = 0;   // fp16 bits, low half = row g
-                if constexpr (ASYM) {
-                    const uint16_t* zc = reinterpret_cast<const uint16_t*>(slot + 1024);
-                    za = zc[rowA - c0] | (static_cast<uint32_t>(zc[rowB - c0]) << 16);
-                    if constexpr (OUT != OUT_DEBUG)
-                        sa = zc[24 + rowA - c0] | (static_cast<uint32_t>(zc[24 + rowB - c0]) << 16);
-                    __syncwarp();   // every lane has read the shared chunks before the slot is refilled
+                uint4 wa[TPW], wb[TPW];
+                uint32_t za[TPW], sa[TPW];   // fp16 bits, low half = row g
+#pragma unroll
+                for (int j = 0; j < TPW; ++j) {
+                    wa[j] = *reinterpret_cast<const uint4*>(slot + 1024 * j + lane * 16);
+                    wb[j] = *reinterpret_cast<const uint4*>(slot + 1024 * j + 512 + lane * 16);
+                    za[j] = sa[j] = 0;
+                    if constexpr (ASYM) {
+                        const uint16_t* zc = reinterpret_cast<const uint16_t*>(slot + 1024 * TPW + 96 * j);
+                        za[j] = zc[rowA[j] - c0[j]] | (static_cast<uint32_t>(zc[rowB[j] - c0[j]]) << 16);
+                        if constexpr (OUT != OUT_DEBUG)
+                            sa[j] = zc[24 + rowA[j] - c0[j]] | (static_cast<uint32_t>(zc[24 + rowB[j] - c0[j]]) << 16);
+                    }
                 }
+                if constexpr (ASYM) __syncwarp();   // every lane has read the shared chunks before the slot is refilled
                 issue();
                 tok_prefetch(kb + D);
                 // token fragments: per n-tile, the 16 (32 for 8-bit codes) bytes of token
@@ -427,22 +464,23 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                         }
                     }
                 }
-                // A fragments of the 4 steps: unsigned codes u (per-channel: signed code + 8)
-                uint32_t af[4][4];
-                const uint32_t wA[4] = {wa.x, wa.y, wa.z, wa.w}, wB[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
-                    const uint32_t fa = ASYM ? wA[s] : wA[s] ^ 0x88888888u;
-                    const uint32_t fb = ASYM ? wB[s] : wB[s] ^ 0x88888888u;
-                    af[s][0] = fa & 0x0F0F0F0Fu;
-                    af[s][1] = fb & 0x0F0F0F0Fu;
-                    af[s][2] = (fa >> 4) & 0x0F0F0F0Fu;
-                    af[s][3] = (fb >> 4) & 0x0F0F0F0Fu;
-                }
+                    // A fragments of step s: unsigned codes u (per-channel: signed code + 8)
+                    uint32_t af[TPW][4];
 #pragma unroll
-                for (int nt = 0; nt < NTT; ++nt) {
+                    for (int j = 0; j < TPW; ++j) {
+                        const uint32_t wA[4] = {wa[j].x, wa[j].y, wa[j].z, wa[j].w};
+                        const uint32_t wB[4] = {wb[j].x, wb[j].y, wb[j].z, wb[j].w};
+                        const uint32_t fa = ASYM ? wA[s] : wA[s] ^ 0x88888888u;
+                        const uint32_t fb = ASYM ? wB[s] : wB[s] ^ 0x88888888u;
+                        af[j][0] = fa & 0x0F0F0F0Fu;
+                        af[j][1] = fb & 0x0F0F0F0Fu;
+                        af[j][2] = (fa >> 4) & 0x0F0F0F0Fu;
+                        af[j][3] = (fb >> 4) & 0x0F0F0F0Fu;
+                    }
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
+                    for (int nt = 0; nt < NTT; ++nt) {
                         uint32_t b0, b1;
                         if constexpr (A8) {
                             const uint4 t0v = tn[nt][0], t1v = tn[nt][TOKV - 1];
@@ -453,14 +491,19 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                             unpack_s4x8_times16(x[s], b0, b1);
                         }
                         if (fresh && s == 0) {
-                            mma_s8_c(acc[nt], af[s], b0, b1, ASYM ? mag4 : zero4);
+#pragma unroll
+                            for (int j = 0; j < TPW; ++j) mma_s8_c(acc[j][nt], af[j], b0, b1, ASYM ? mag4 : zero4);
                             if constexpr (!TS) mma_s8_c(ssum[nt], ones, b0, b1, ASYM ? mag4 : zero4);
                         } else {
-                            mma_s8_c(acc[nt], af[s], b0, b1, acc[nt]);
+#pragma unroll
+                            for (int j = 0; j < TPW; ++j) mma_s8_c(acc[j][nt], af[j], b0, b1, acc[j][nt]);
                             if constexpr (!TS) mma_s8_c(ssum[nt], ones, b0, b1, ssum[nt]);
                         }
                     }
-                    if constexpr (TS) {
+                }
+                if constexpr (TS) {
+#pragma unroll
+                    for (int nt = 0; nt < NTT; ++nt) {
                         const int2 sv = *reinterpret_cast<const int2*>(tsum_s + kb * NT + 8 * nt + 2 * tq);
                         sacc[nt][0] = (fresh ? 0 : sacc[nt][0]) + sv.x;
                         sacc[nt][1] = (fresh ? 0 : sacc[nt][1]) + sv.y;
@@ -473,44 +516,46 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                     if (gend) cgk = 0;
                     if (gend || kb + 1 == kb1) {
                         // end of a group (or of this warp's share of it): acc - z S, scaled
-                        const float zfa = __half2float(__ushort_as_half(static_cast<uint16_t>(za & 0xFFFFu)));
-                        const float zfb = __half2float(__ushort_as_half(static_cast<uint16_t>(za >> 16)));
-                        if constexpr (OUT == OUT_DEBUG) {
-                            const int zia = static_cast<int>(zfa), zib = static_cast<int>(zfb);
-                            const int g = cg;
 #pragma unroll
-                            for (int nt = 0; nt < NTT; ++nt) {
+                        for (int j = 0; j < TPW; ++j) {
+                            const float zfa = __half2float(__ushort_as_half(static_cast<uint16_t>(za[j] & 0xFFFFu)));
+                            const float zfb = __half2float(__ushort_as_half(static_cast<uint16_t>(za[j] >> 16)));
+                            if constexpr (OUT == OUT_DEBUG) {
+                                const int zia = static_cast<int>(zfa), zib = static_cast<int>(zfb);
 #pragma unroll
-                                for (int v = 0; v < 4; ++v) {
-                                    const int m = 8 * nt + 2 * tq + (v & 1);
-                                    const int n = v < 2 ? rowA : rowB;
-                                    const int sv = TS ? sacc[nt][v & 1] : static_cast<int>(ssum[nt][v & 1] - dk::MAGIC);
-                                    const int a = static_cast<int>(acc[nt][v] - dk::MAGIC) - (v < 2 ? zia : zib) * sv;
-                                    if ((v < 2 ? okA : okB) && m < p.M)
-                                        atomicAdd(p.dbg_acc + (static_cast<int64_t>(m) * p.N + n) * G + g, a >> sh);
+                                for (int nt = 0; nt < NTT; ++nt) {
+#pragma unroll
+                                    for (int v = 0; v < 4; ++v) {
+                                        const int m = 8 * nt + 2 * tq + (v & 1);
+                                        const int n = v < 2 ? rowA[j] : rowB[j];
+                                        const int sv = TS ? sacc[nt][v & 1] : static_cast<int>(ssum[nt][v & 1] - dk::MAGIC);
+                                        const int a = static_cast<int>(acc[j][nt][v] - dk::MAGIC) - (v < 2 ? zia : zib) * sv;
+                                        if ((v < 2 ? okA[j] : okB[j]) && m < p.M)
+                                            atomicAdd(p.dbg_acc + (static_cast<int64_t>(m) * p.N + n) * G + cg, a >> sh);
+                                    }
                                 }
-                            }
-                        } else {
-                            const float sfa = __half2float(__ushort_as_half(static_cast<uint16_t>(sa & 0xFFFFu))) * inv_act;
-                            const float sfb = __half2float(__ushort_as_half(static_cast<uint16_t>(sa >> 16))) * inv_act;
-                            const float2 nmag = make_float2(-dk::MAGIC_F, -dk::MAGIC_F);
-                            const float2 nza = make_float2(-zfa, -zfa), nzb = make_float2(-zfb, -zfb);
-                            const float2 s2a = make_float2(sfa, sfa), s2b = make_float2(sfb, sfb);
+                            } else {
+                                const float sfa = __half2float(__ushort_as_half(static_cast<uint16_t>(sa[j] & 0xFFFFu))) * inv_act;
+                                const float sfb = __half2float(__ushort_as_half(static_cast<uint16_t>(sa[j] >> 16))) * inv_act;
+                                const float2 nmag = make_float2(-dk::MAGIC_F, -dk::MAGIC_F);
+                                const float2 nza = make_float2(-zfa, -zfa), nzb = make_float2(-zfb, -zfb);
+                                const float2 s2a = make_float2(sfa, sfa), s2b = make_float2(sfb, sfb);
 #pragma unroll
-                            for (int nt = 0; nt < NTT; ++nt) {
-                                const float2 sf = TS ? make_float2(static_cast<float>(sacc[nt][0]), static_cast<float>(sacc[nt][1]))
-                                                     : __fadd2_rn(make_float2(__uint_as_float(ssum[nt][0]), __uint_as_float(ssum[nt][1])), nmag);
-                                const float2 fa = __fadd2_rn(make_float2(__uint_as_float(acc[nt][0]), __uint_as_float(acc[nt][1])), nmag);
-                                const float2 fb = __fadd2_rn(make_float2(__uint_as_float(acc[nt][2]), __uint_as_float(acc[nt][3])), nmag);
-                                const float2 ta = __ffma2_rn(nza, sf, fa);   // exact: integers below 2^24
-                                const float2 tb = __ffma2_rn(nzb, sf, fb);
-                                float2 ya = make_float2(y[nt][0], y[nt][1]), yb = make_float2(y[nt][2], y[nt][3]);
-                                ya = __ffma2_rn(s2a, ta, ya);
-                                yb = __ffma2_rn(s2b, tb, yb);
-                                y[nt][0] = ya.x;
-                                y[nt][1] = ya.y;
-                                y[nt][2] = yb.x;
-                                y[nt][3] = yb.y;
+                                for (int nt = 0; nt < NTT; ++nt) {
+                                    const float2 sf = TS ? make_float2(static_cast<float>(sacc[nt][0]), static_cast<float>(sacc[nt][1]))
+                                                         : __fadd2_rn(make_float2(__uint_as_float(ssum[nt][0]), __uint_as_float(ssum[nt][1])), nmag);
+                                    const float2 fa = __fadd2_rn(make_float2(__uint_as_float(acc[j][nt][0]), __uint_as_float(acc[j][nt][1])), nmag);
+                                    const float2 fb = __fadd2_rn(make_float2(__uint_as_float(acc[j][nt][2]), __uint_as_float(acc[j][nt][3])), nmag);
+                                    const float2 ta = __ffma2_rn(nza, sf, fa);   // exact: integers below 2^24
+                                    const float2 tb = __ffma2_rn(nzb, sf, fb);
+                                    float2 ya = make_float2(y[j][nt][0], y[j][nt][1]), yb = make_float2(y[j][nt][2], y[j][nt][3]);
+                                    ya = __ffma2_rn(s2a, ta, ya);
+                                    yb = __ffma2_rn(s2b, tb, yb);
+                                    y[j][nt][0] = ya.x;
+                                    y[j][nt][1] = ya.y;
+                                    y[j][nt][2] = yb.x;
+                                    y[j][nt][3] = yb.y;
+                                }
                             }
                         }
                         fresh = true;
@@ -522,25 +567,30 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                 // per-channel: signed code = u - 8, exact integer partial sums
                 if (kb1 > kb0) {
 #pragma unroll
-                    for (int nt = 0; nt < NTT; ++nt)
+                    for (int j = 0; j < TPW; ++j)
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            yi[nt][v] = static_cast<int32_t>(acc[nt][v]) -
-                                        8 * (TS ? sacc[nt][v & 1] : static_cast<int32_t>(ssum[nt][v & 1]));
+                        for (int nt = 0; nt < NTT; ++nt)
+#pragma unroll
+                            for (int v = 0; v < 4; ++v)
+                                yi[j][nt][v] = static_cast<int32_t>(acc[j][nt][v]) -
+                                               8 * (TS ? sacc[nt][v & 1] : static_cast<int32_t>(ssum[nt][v & 1]));
                 }
             }
         }
         if (!gathered) gather();
-        // ---- the warps of a tile meet: partial sums through shared memory (over the rings)
+        // ---- the warps of a group meet: partial sums through shared memory (over the rings)
         cp_async_wait_all();
         __syncthreads();
         if (active) {
-            uint4* part = reinterpret_cast<uint4*>(smem) + (warp * 32 + lane) * NTT;
+            uint4* part = reinterpret_cast<uint4*>(smem) + (warp * 32 + lane) * (TPW * NTT);
 #pragma unroll
-            for (int nt = 0; nt < NTT; ++nt)
-                part[nt] = ASYM ? make_uint4(__float_as_uint(y[nt][0]), __float_as_uint(y[nt][1]), __float_as_uint(y[nt][2]),
-                                             __float_as_uint(y[nt][3]))
-                                : make_uint4(yi[nt][0], yi[nt][1], yi[nt][2], yi[nt][3]);
+            for (int j = 0; j < TPW; ++j)
+#pragma unroll
+                for (int nt = 0; nt < NTT; ++nt)
+                    part[j * NTT + nt] =
+                        ASYM ? make_uint4(__float_as_uint(y[j][nt][0]), __float_as_uint(y[j][nt][1]),
+                                          __float_as_uint(y[j][nt][2]), __float_as_uint(y[j][nt][3]))
+                             : make_uint4(yi[j][nt][0], yi[j][nt][1], yi[j][nt][2], yi[j][nt][3]);
         }
         if (pass == 0) {
 #pragma unroll
@@ -550,76 +600,79 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
             }
         }
         __syncthreads();
-        // ---- finish: warp w < ntp completes tile w in its own fragment layout
+        // ---- finish: warp w < ntp completes group w in its own fragment layout
         if (warp < ntp) {
-            // partial sums of the tile's warps, added in warp order
 #pragma unroll
-            for (int nt = 0; nt < NTT; ++nt) {
-                float ys[4] = {0.f, 0.f, 0.f, 0.f};
-                int32_t yis[4] = {0, 0, 0, 0};
-                for (int sidx = 0; sidx < S; ++sidx) {
-                    const uint4 v = reinterpret_cast<const uint4*>(smem)[((sidx * ntp + warp) * 32 + lane) * NTT + nt];
-                    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+            for (int j = 0; j < TPW; ++j) {
+                // partial sums of the group's warps, added in warp order
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if constexpr (ASYM) ys[j] = __fadd_rn(ys[j], __uint_as_float(vv[j]));
-                        else yis[j] += static_cast<int32_t>(vv[j]);
+                for (int nt = 0; nt < NTT; ++nt) {
+                    float ys[4] = {0.f, 0.f, 0.f, 0.f};
+                    int32_t yis[4] = {0, 0, 0, 0};
+                    for (int sidx = 0; sidx < S; ++sidx) {
+                        const uint4 v = reinterpret_cast<const uint4*>(smem)[((sidx * ntp + warp) * 32 + lane) * (TPW * NTT) + j * NTT + nt];
+                        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if constexpr (ASYM) ys[q] = __fadd_rn(ys[q], __uint_as_float(vv[q]));
+                            else yis[q] += static_cast<int32_t>(vv[q]);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        y[j][nt][q] = ys[q];
+                        yi[j][nt][q] = yis[q];
+                    }
+                }
+                // SERQ term X[m,S] . Rq[n,:] for rows g, g + 8 and the n-tiles' tokens:
+                // one or two 32-input MMA steps; lane t takes packed word 4 s + t of
+                // the Rq rows (A, 16 q) and the matching lo/hi words of X[m,S] (B)
+                const int rw = p.r / 8;   // packed Rq words per row
+                const int nA = r0 + 16 * (TPW * (t0 + warp) + j) + gq, nB = nA + 8;
+                uint32_t cc[NTT][4];
+#pragma unroll
+                for (int nt = 0; nt < NTT; ++nt) cc[nt][0] = cc[nt][1] = cc[nt][2] = cc[nt][3] = 0;
+                if (p.r > 0) {
+                    const uint32_t* rqA = reinterpret_cast<const uint32_t*>(rq_s + (nA - pr0) * (p.r / 2));
+                    const uint32_t* rqB = reinterpret_cast<const uint32_t*>(rq_s + (nB - pr0) * (p.r / 2));
+#pragma unroll
+                    for (int st = 0; st < 2; ++st) {
+                        const int wi = 4 * st + tq;
+                        if (4 * st >= rw) break;
+                        const bool has = wi < rw;
+                        const uint32_t qa = has && nA < pr1 ? rqA[wi] : 0u;   // (two's complement nibbles)
+                        const uint32_t qb = has && nB < pr1 ? rqB[wi] : 0u;
+                        uint32_t a[4];
+                        unpack_s4x8_times16(qa, a[0], a[2]);
+                        unpack_s4x8_times16(qb, a[1], a[3]);
+#pragma unroll
+                        for (int nt = 0; nt < NTT; ++nt) {
+                            const int m = 8 * nt + gq;
+                            const uint32_t b0 = has ? xs_s[m * dk::XS_WORDS + 2 * wi] : 0u;
+                            const uint32_t b1 = has ? xs_s[m * dk::XS_WORDS + 2 * wi + 1] : 0u;
+                            mma_s8_c(cc[nt], a, b0, b1, cc[nt]);
+                        }
                     }
                 }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    y[nt][j] = ys[j];
-                    yi[nt][j] = yis[j];
-                }
-            }
-            // SERQ term X[m,S] . Rq[n,:] for rows g, g + 8 and the n-tiles' tokens:
-            // one or two 32-input MMA steps; lane t takes packed word 4 s + t of
-            // the Rq rows (A, 16 q) and the matching lo/hi words of X[m,S] (B)
-            const int rw = p.r / 8;   // packed Rq words per row
-            const int nA = r0 + 16 * (t0 + warp) + gq, nB = nA + 8;
-            uint32_t cc[NTT][4];
+                for (int nt = 0; nt < NTT; ++nt) {
 #pragma unroll
-            for (int nt = 0; nt < NTT; ++nt) cc[nt][0] = cc[nt][1] = cc[nt][2] = cc[nt][3] = 0;
-            if (p.r > 0) {
-                const uint32_t* rqA = reinterpret_cast<const uint32_t*>(rq_s + (nA - pr0) * (p.r / 2));
-                const uint32_t* rqB = reinterpret_cast<const uint32_t*>(rq_s + (nB - pr0) * (p.r / 2));
-#pragma unroll
-                for (int st = 0; st < 2; ++st) {
-                    const int wi = 4 * st + tq;
-                    if (4 * st >= rw) break;
-                    const bool has = wi < rw;
-                    const uint32_t qa = has && nA < pr1 ? rqA[wi] : 0u;   // (two's complement nibbles)
-                    const uint32_t qb = has && nB < pr1 ? rqB[wi] : 0u;
-                    uint32_t a[4];
-                    unpack_s4x8_times16(qa, a[0], a[2]);
-                    unpack_s4x8_times16(qb, a[1], a[3]);
-#pragma unroll
-                    for (int nt = 0; nt < NTT; ++nt) {
-                        const int m = 8 * nt + gq;
-                        const uint32_t b0 = has ? xs_s[m * dk::XS_WORDS + 2 * wi] : 0u;
-                        const uint32_t b1 = has ? xs_s[m * dk::XS_WORDS + 2 * wi + 1] : 0u;
-                        mma_s8_c(cc[nt], a, b0, b1, cc[nt]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < NTT; ++nt) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int m = 8 * nt + 2 * tq + (j & 1);
-                    const int n = j < 2 ? nA : nB;
-                    if (n >= pr1 || m >= p.M) continue;
-                    const int c = static_cast<int32_t>(cc[nt][j]) >> 4;
-                    const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                    if constexpr (OUT == OUT_DEBUG) {
-                        if constexpr (!ASYM) p.dbg_acc[o] = yi[nt][j] >> sh;
-                        if (p.r > 0) p.dbg_acc_c[o] = c;
-                    } else {
-                        const float srn = p.r > 0 ? __half2float(__ushort_as_half(sr_s[n - pb])) : 0.f;
-                        const float base = ASYM ? y[nt][j]
-                                                : __fmul_rn(__half2float(__ushort_as_half(sw_s[n - pb])),
-                                                            static_cast<float>(yi[nt][j] >> sh));
-                        store_one<OUT>(p.Y, o, __fmul_rn(sx_s[m], __fmaf_rn(srn, static_cast<float>(c), base)));
+                    for (int q = 0; q < 4; ++q) {
+                        const int m = 8 * nt + 2 * tq + (q & 1);
+                        const int n = q < 2 ? nA : nB;
+                        if (n >= pr1 || m >= p.M) continue;
+                        const int c = static_cast<int32_t>(cc[nt][q]) >> 4;
+                        const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                        if constexpr (OUT == OUT_DEBUG) {
+                            if constexpr (!ASYM) p.dbg_acc[o] = yi[j][nt][q] >> sh;
+                            if (p.r > 0) p.dbg_acc_c[o] = c;
+                        } else {
+                            const float srn = p.r > 0 ? __half2float(__ushort_as_half(sr_s[n - pb])) : 0.f;
+                            const float base = ASYM ? y[j][nt][q]
+                                                    : __fmul_rn(__half2float(__ushort_as_half(sw_s[n - pb])),
+                                                                static_cast<float>(yi[j][nt][q] >> sh));
+                            store_one<OUT>(p.Y, o, __fmul_rn(sx_s[m], __fmaf_rn(srn, static_cast<float>(c), base)));
+                        }
                     }
                 }
             }
@@ -668,6 +721,7 @@ template <int NT, bool ASYM, bool A8, int OUT>
 static hq_status launch_sk_t(const GemmArgs& a, cudaStream_t st, int nsm) {
     bool staged = false;
     const DkPlan plan = dk_plan<NT>(a.M, a.N, a.K, A8, nsm, staged);
+    if (plan.D == 0) return HQ_ERR_UNSUPPORTED;
     // the debug entry adds the partial group sums of the warps with atomics
     if (OUT == OUT_DEBUG && ASYM &&
         cudaMemsetAsync(a.dbg_acc, 0, static_cast<size_t>(a.M) * a.N * (a.K / a.gw) * sizeof(int32_t), st) !=
