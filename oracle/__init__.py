@@ -60,6 +60,9 @@ _sig("hqo_serq_prepare", [_P, _I64, _I64, _P, _P, _P, _I32, _P, _I32, _P, _P, _P
 _sig("hqo_accum", [_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P], _ct.c_int)
 _sig("hqo_accum8", [_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P], _ct.c_int)
 _sig("hqo_epilogue_f64", [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P])
+_sig("hqo_rotate_quant_asym", [_P, _ct.c_int, _I64, _I64, _I32, _P, _P, _P, _P])
+_sig("hqo_accum_asym", [_P, _P, _I64, _I64, _I32, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P], _ct.c_int)
+_sig("hqo_epilogue_asym_f64", [_P, _P, _I64, _I64, _I64, _I32, _I32, _P, _P, _P, _P])
 _sig("hqo_linear_rows_f64", [_P, _P, _I64, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _P, _I64, _P])
 _sig("hqo_linear_fp64", [_P, _ct.c_int, _I64, _I64, _P, _ct.c_int, _I64, _P])
 _sig("hqo_salient_channels", [_P, _ct.c_int, _I64, _I64, _I32, _P, _I32, _P, _P])
@@ -261,6 +264,50 @@ def accum8(Xq8, K, Wq, zw, gw, Rq=None, sal=None):
                           _ptr(acc), _ptr(acc_c))
     assert ovf == 0, "accumulator exceeds int32"
     return acc, acc_c
+
+
+def rotate_quant_asym(X, xdtype, g, d=None):
+    """OffQ per-group asymmetric activations: (Xq [M, K/2] unsigned nibbles,
+    sx [M, K/g] float32, zx [M, K/g] int32)."""
+    X = _raw(X, xdtype)
+    M, K = X.shape
+    Xq = _np.empty((M, K // 2), _np.uint8)
+    sx = _np.empty((M, K // g), _np.float32)
+    zx = _np.empty((M, K // g), _np.int32)
+    _lib.hqo_rotate_quant_asym(_ptr(X), _DT[xdtype], M, K, g, _ptr(_signs(d, g)), _ptr(Xq), _ptr(sx), _ptr(zx))
+    return Xq, sx, zx
+
+
+def accum_asym(Xq, zx, K, g, Wq, zw, gw, Rq=None, sal=None):
+    """Integer accumulators per activation group with asymmetric activations:
+    acc [M, N, K/g] int64 and acc_c [M, N, K/g] int64."""
+    assert gw == 0 or gw % g == 0, "activation groups must nest in the weight groups"
+    Xq = _c(Xq, _np.uint8)
+    Wq = _c(Wq, _np.uint8)
+    M, N = Xq.shape[0], Wq.shape[0]
+    G = K // g
+    r = 0 if sal is None else len(sal)
+    acc = _np.empty((M, N, G), _np.int64)
+    acc_c = _np.zeros((M, N, G), _np.int64)
+    zp = None if zw is None else _c(zw, _np.float16)
+    salp = None if r == 0 else _c(sal, _np.int32)
+    Rqp = None if r == 0 else _c(Rq, _np.uint8)
+    ovf = _lib.hqo_accum_asym(_ptr(Xq), _ptr(_c(zx, _np.int32)), M, K, g, _ptr(Wq), _ptr(zp), N, gw, _ptr(Rqp),
+                              _ptr(salp), r, _ptr(acc), _ptr(acc_c))
+    assert ovf == 0, "accumulator exceeds int32"
+    return acc, acc_c
+
+
+def epilogue_asym_f64(acc, acc_c, g, gw, sx, sw, sr=None):
+    """y64 = sum_b sx[m, b] (sw[b', n] acc_b + sr[n] acc_c_b) in fp64."""
+    acc = _c(acc, _np.int64)
+    M, N, G = acc.shape
+    y = _np.empty((M, N), _np.float64)
+    srp = None if sr is None else _c(sr, _np.float16)
+    accc = None if sr is None else _c(acc_c, _np.int64)
+    _lib.hqo_epilogue_asym_f64(_ptr(acc), _ptr(accc), M, N, G, g, gw, _ptr(_c(sx, _np.float32)),
+                               _ptr(_c(sw, _np.float16)), _ptr(srp), _ptr(y))
+    return y
 
 
 def epilogue_f64(acc, acc_c, sx, sw, sr=None):

@@ -23,6 +23,9 @@
  *  [DynamicPTQ] "DynamicPTQ", Methodology 2 (8-bit activations on the
  *          quantisation-sensitive layers, weights and everything else in 4
  *          bit); SERQ section 4 evaluates the same layer at W4A8.
+ *  [OffQ-A] "OffQ ...", Methodology 2, last point (the constant offset the
+ *          rotation creates is absorbed by the zero point of an asymmetric
+ *          quantiser) and Methodology 3 (one scale and zero point per group).
  *
  * Readings where the pages are silent (each one is listed in the design
  * notes): H = diag(d) * Sylvester(g), d a +-1 vector with d[0] = +1; the
@@ -592,4 +595,114 @@ void hqo_f32_to_f16_array(const float* in, int64_t n, uint16_t* out)
 void hqo_f16_to_f32_array(const uint16_t* in, int64_t n, float* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = hqo_f16_to_f32(in[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* OffQ per-group asymmetric activations [OffQ-A].                           */
+/* ------------------------------------------------------------------------ */
+
+/* Per row m and Hadamard group b (g channels): u = the rotated group;
+ * lo = min u, hi = max u, dlt = fl32(hi - lo) (the group's own range: the
+ * offset is not forced into it); a constant group takes dlt = |lo| (15 when
+ * lo == 0), so it is reconstructed exactly.  s = fl32(dlt / 15),
+ * inv = fl32(15 / dlt), z = rint(fl32(-lo * inv)) (an integer, not clamped:
+ * an all-positive group has z < 0), q = clamp(rint(fl32(u * inv)) + z, 0, 15),
+ * unsigned nibbles.  sx[m][b] = fl32(s * fl32(1/sqrt(g))), zx[m][b] = z.
+ * Xq is [M][K/2] packed; sx, zx are [M][K/g]. */
+void hqo_rotate_quant_asym(const void* X, int dtype, int64_t M, int64_t K, int32_t g,
+                           const int8_t* d, uint8_t* Xq, float* sx, int32_t* zx)
+{
+    float cg = (float)(1.0 / sqrt((double)g));
+    int64_t G = K / g;
+    float* u = (float*)malloc((size_t)(M * K) * sizeof(float));
+    hqo_rotate_rows(X, dtype, M, K, g, d, u);
+    memset(Xq, 0, (size_t)(M * (K / 2)));
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        uint8_t* qrow = Xq + m * (K / 2);
+        for (int64_t b = 0; b < G; ++b) {
+            const float* gu = u + m * K + b * g;
+            float lo = gu[0], hi = gu[0];
+            for (int32_t k = 1; k < g; ++k) {
+                lo = fminf(lo, gu[k]);
+                hi = fmaxf(hi, gu[k]);
+            }
+            float dlt = hi - lo;
+            if (dlt == 0.0f) dlt = lo != 0.0f ? fabsf(lo) : 15.0f;
+            float s = dlt / 15.0f;
+            float inv = 15.0f / dlt;
+            float zf = rintf(-lo * inv);
+            int32_t z = (int32_t)zf;
+            sx[m * G + b] = s * cg;
+            zx[m * G + b] = z;
+            for (int32_t k = 0; k < g; ++k) {
+                float t = gu[k] * inv;
+                int q = (int)clampf(rintf(t) + zf, 0.0f, 15.0f);
+                put_nibble(qrow, b * g + k, q);
+            }
+        }
+    }
+    free(u);
+}
+
+/* The integer GEMM with per-group asymmetric activations (activation groups
+ * of g inputs, nested in the weight groups: gw == 0 or gw % g == 0):
+ *   acc[m][n][b]   = sum_{k in group b} (qx[m][k] - zx[m][b]) * wv[n][k]
+ *   acc_c[m][n][b] = sum_{j: S_j in group b} (qx[m][S_j] - zx[m][b]) * qr[n][j]
+ * wv = qw - z_w (group weights) or the signed code (per channel).  Plain
+ * loops in int64; returns 1 if any value does not fit in int32. */
+int hqo_accum_asym(const uint8_t* Xq, const int32_t* zx, int64_t M, int64_t K, int32_t g,
+                   const uint8_t* Wq, const uint16_t* zw, int64_t N, int32_t gw,
+                   const uint8_t* Rq, const int32_t* sal, int32_t r, int64_t* acc, int64_t* acc_c)
+{
+    int64_t G = K / g;
+    int64_t ldr = (r + 1) / 2;
+    int overflow = 0;
+    #pragma omp parallel for schedule(static) reduction(|:overflow)
+    for (int64_t m = 0; m < M; ++m) {
+        const uint8_t* xrow = Xq + m * (K / 2);
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* wrow = Wq + n * (K / 2);
+            for (int64_t b = 0; b < G; ++b) {
+                int64_t zb = zx[m * G + b];
+                int64_t s = 0;
+                for (int64_t k = b * g; k < (b + 1) * g; ++k) {
+                    int wv = gw ? get_nibble_u(wrow, k) - (int)hqo_f16_to_f32(zw[(k / gw) * N + n])
+                                : get_nibble_s(wrow, k);
+                    s += ((int64_t)get_nibble_u(xrow, k) - zb) * wv;
+                }
+                acc[(m * N + n) * G + b] = s;
+                if (s > INT32_MAX || s < INT32_MIN) overflow = 1;
+                if (acc_c) {
+                    int64_t c = 0;
+                    for (int32_t j = 0; j < r; ++j)
+                        if (sal[j] / g == b)
+                            c += ((int64_t)get_nibble_u(xrow, sal[j]) - zb) * get_nibble_s(Rq + n * ldr, j);
+                    acc_c[(m * N + n) * G + b] = c;
+                }
+            }
+        }
+    }
+    return overflow;
+}
+
+/* y64[m][n] = sum_b sx[m][b] * (sw[b'][n] * acc[m][n][b] + sr[n] * acc_c[m][n][b]),
+ * b' = the weight group holding activation group b (b' = 0 per channel),
+ * in fp64 from the exact integers.  sr / acc_c may be NULL. */
+void hqo_epilogue_asym_f64(const int64_t* acc, const int64_t* acc_c, int64_t M, int64_t N, int64_t G,
+                           int32_t g, int32_t gw, const float* sx, const uint16_t* sw, const uint16_t* sr,
+                           double* y)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double t = 0.0;
+            for (int64_t b = 0; b < G; ++b) {
+                int64_t bw = gw ? (b * g) / gw : 0;
+                double part = (double)hqo_f16_to_f32(sw[bw * N + n]) * (double)acc[(m * N + n) * G + b];
+                if (acc_c && sr) part += (double)hqo_f16_to_f32(sr[n]) * (double)acc_c[(m * N + n) * G + b];
+                t += (double)sx[m * G + b] * part;
+            }
+            y[m * N + n] = t;
+        }
 }

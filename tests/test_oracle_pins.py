@@ -537,3 +537,125 @@ def test_w4a8_layer_against_dequantised_matmul_and_closer_to_float(name):
     rel8 = np.linalg.norm(y8 - yf) / np.linalg.norm(yf)
     rel4 = np.linalg.norm(y4 - yf) / np.linalg.norm(yf)
     assert rel8 < rel4, (rel8, rel4)
+
+
+# ----------------------------------------------------------------- OffQ per-group asymmetric activations
+# OffQ, Methodology 2 (last point) and 3: the constant offset the all-ones row
+# of H creates is absorbed by the zero point of an asymmetric quantiser with one
+# scale and zero point per group.
+
+def _asym_setup(seed, M=6, K=512, g=128, outlier=True):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    if outlier:
+        x[0, 0] = 1000.0                           # one concentrated outlier in group 0's first channel
+        x[2, g + 0] = -400.0                       # a negative one in group 1
+    X = x.astype(np.float16)
+    d = synth.hadamard_signs(g, seed=seed)
+    return X, d
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_asym_activation_round_trip_and_endpoint_codes(seed):
+    g = 128
+    X, d = _asym_setup(seed)
+    Xq, sx, zx = O.rotate_quant_asym(X, "f16", g, d)
+    u = O.rotate_rows(X, "f16", g, d).astype(np.float64)
+    q = O.unpack_u4(Xq, X.shape[1]).astype(np.int64)
+    M, K = X.shape
+    for m in range(M):
+        for b in range(K // g):
+            ug = u[m, b * g:(b + 1) * g]
+            qg = q[m, b * g:(b + 1) * g]
+            s = (ug.max() - ug.min()) / 15.0      # the group's own range, in fp64
+            rec = s * (qg - zx[m, b])
+            # every element within half a step (plus the fp32 rounding of the reciprocal)
+            assert np.all(np.abs(rec - ug) <= 0.5 * s * (1 + 1e-5) + 1e-6 * np.abs(ug).max())
+            # the ends of the range take the extreme codes
+            assert qg.min() == 0 and qg.max() == 15
+            # the stored scale is that step times 1/sqrt(g)
+            assert abs(sx[m, b] - s / np.sqrt(g)) <= 1e-6 * s / np.sqrt(g)
+
+
+def test_asym_absorbs_the_rotated_offset():
+    # the outlier of row 0 becomes a constant offset of ~1000 over group 0; the
+    # per-token symmetric quantiser spends its range on it, the per-group
+    # asymmetric one moves it into the zero point
+    g = 128
+    X, d = _asym_setup(0)
+    u = O.rotate_rows(X, "f16", g, d).astype(np.float64)
+    assert np.all(u[0, :g] > 900)                  # the offset (OffQ, Methodology 2)
+    Xq, sx, zx = O.rotate_quant_asym(X, "f16", g, d)
+    qa = O.unpack_u4(Xq, X.shape[1]).astype(np.float64)
+    s_a = sx.astype(np.float64) * np.sqrt(g)
+    rec_a = s_a[0, 0] * (qa[0, :g] - zx[0, 0])
+    Xs, sxs = O.rotate_quant(X, "f16", g, d)
+    rec_s = O.unpack_s4(Xs, X.shape[1]).astype(np.float64)[0, :g] * sxs[0] * np.sqrt(g)
+    err_a = np.abs(rec_a - u[0, :g]).max()
+    err_s = np.abs(rec_s - u[0, :g]).max()
+    assert zx[0, 0] < -100                         # the offset sits in the zero point
+    assert err_a < err_s / 20
+
+
+def test_asym_constant_and_zero_groups():
+    g = 128
+    K = 2 * g
+    X = np.zeros((2, K), np.float16)
+    X[0, 0] = 3.0                                  # rotated group 0 of row 0: constant 3
+    X[1, g] = -5.0                                 # rotated group 1 of row 1: constant -5
+    d = synth.hadamard_signs(g, seed=4)
+    Xq, sx, zx = O.rotate_quant_asym(X, "f16", g, d)
+    q = O.unpack_u4(Xq, K).astype(np.int64)
+    s = sx.astype(np.float64) * np.sqrt(g)
+    rec = lambda m, b: s[m, b] * (q[m, b * g:(b + 1) * g] - zx[m, b])
+    assert np.allclose(rec(0, 0), 3.0, rtol=1e-6) and np.allclose(rec(1, 1), -5.0, rtol=1e-6)
+    # all-zero groups: code 0, zero point 0, reconstruction 0
+    for m, b in ((0, 1), (1, 0)):
+        assert zx[m, b] == 0 and np.all(q[m, b * g:(b + 1) * g] == 0) and np.all(rec(m, b) == 0)
+
+
+@pytest.mark.parametrize("gw", [0, 128, 256])
+def test_accum_asym_matches_numpy(gw):
+    rng = np.random.default_rng(11)
+    M, N, K, g = 4, 6, 512, 128
+    qx = rng.integers(0, 16, (M, K)).astype(np.int8)
+    Xq = O.pack_s4(qx)                             # nibble bits; read back unsigned
+    zx = rng.integers(-300, 16, (M, K // g)).astype(np.int32)
+    if gw:
+        Wq = O.pack_s4(rng.integers(0, 16, (N, K)).astype(np.int8))
+        z = rng.integers(0, 16, (K // gw, N)).astype(np.float16)
+        wv = O.unpack_u4(Wq, K).astype(np.int64) - np.repeat(z.astype(np.int64).T, gw, axis=1)
+    else:
+        qw = rng.integers(-8, 8, (N, K)).astype(np.int8)
+        Wq = O.pack_s4(qw)
+        z = None
+        wv = qw.astype(np.int64)
+    sal = np.array([3, 17, 130, 300, 511], np.int32)
+    qr = rng.integers(-8, 8, (N, 5)).astype(np.int8)
+    acc, acc_c = O.accum_asym(Xq, zx, K, g, Wq, z, gw, O.pack_s4(qr), sal)
+    xv = O.unpack_u4(Xq, K).astype(np.int64) - np.repeat(zx.astype(np.int64), g, axis=1)
+    for b in range(K // g):
+        sl = slice(b * g, (b + 1) * g)
+        assert np.array_equal(acc[:, :, b], xv[:, sl] @ wv[:, sl].T)
+        inb = sal // g == b
+        assert np.array_equal(acc_c[:, :, b], xv[:, sal[inb]] @ qr[:, inb].astype(np.int64).T)
+
+
+def test_epilogue_asym_against_dequantised_float_matmul():
+    g, gw = 128, 128
+    X, d = _asym_setup(5, M=8, K=256)
+    rng = np.random.default_rng(12)
+    Wrot = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    Wq, sw, zw = O.w4_pack(Wrot, "f32", gw)
+    sal = np.array([0, 7, 129, 200], np.int32)
+    Rq, sr = O.serq_prepare(Wrot, Wq, sw, zw, gw, sal)
+    Xq, sx, zx = O.rotate_quant_asym(X, "f16", g, d)
+    acc, acc_c = O.accum_asym(Xq, zx, 256, g, Wq, zw, gw, Rq, sal)
+    y = O.epilogue_asym_f64(acc, acc_c, g, gw, sx, sw, sr)
+    # independent formulation: dequantise both operands and multiply (numpy)
+    Xhat = (O.unpack_u4(Xq, 256).astype(np.float64) - np.repeat(zx, g, axis=1)) * np.repeat(
+        sx.astype(np.float64), g, axis=1)
+    What = O.w4_dequant(Wq, sw, zw, 256, gw).astype(np.float64)
+    Rhat = O.unpack_s4(Rq, len(sal)).astype(np.float64) * sr.astype(np.float64)[:, None]
+    ref = Xhat @ What.T + Xhat[:, sal] @ Rhat.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
