@@ -259,6 +259,53 @@ hq_status hq_rotate_quant8(const void* X, hq_dtype xt, int64_t M, int64_t K, int
                            void* stream);
 
 /*
+ * hq_rotate_quant_asym -- OffQ's per-group asymmetric activation quantiser.
+ * Source: "OffQ ...", Methodology 2, last point (the constant offset the
+ * all-ones first row of H creates over a group is absorbed by the zero point
+ * of an asymmetric quantiser) and Methodology 3 (one scale and zero point per
+ * group).  Per row m and Hadamard group b of `group` channels: u = the rotated
+ * group as in hq_rotate_quant; lo = min u, hi = max u, dlt = fl32(hi - lo)
+ * (|lo| for a constant group, 15 when that is 0); inv = fl32(15 / dlt);
+ * z = rint(fl32(-lo * inv)) (an integer, not clamped);
+ * q = clamp(rint(fl32(u * inv)) + z, 0, 15);
+ * sx[m][b] = fl32(fl32(dlt / 15) * fl32(1/sqrt(group))), zx[m][b] = z.
+ *  X, xt, ld_x, group, H_signs   as hq_rotate_quant (16-bit X); group in
+ *           [32, 1024] (HQ_ERR_UNSUPPORTED otherwise)
+ *  Xq       device, [M][K/2] unsigned codes, element 2j in the low nibble (output)
+ *  sx       device, [M][K/group] fp32 (output)
+ *  zx       device, [M][K/group] int32 (output)
+ * Errors: as hq_rotate_quant.
+ */
+hq_status hq_rotate_quant_asym(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                               int32_t group, const int8_t* H_signs, uint8_t* Xq, float* sx,
+                               int32_t* zx, void* stream);
+
+/*
+ * w4a4_linear_asym -- w4a4_linear with OffQ's per-group asymmetric activations
+ * (hq_rotate_quant_asym with group 128).  Source: "OffQ ...", Methodology 2
+ * and 3; "SERQ ...", section 2.2 for the residual path.
+ *   acc_b[m][n] = sum_{k in group b} (qx[m][k] - zx[m][b]) * (qw[n][k] - z[b'][n])
+ *   Y[m][n] = sum_b sx[m][b] (sw[b'][n] acc_b[m][n]) + sr[n] sum_j a[m][j] qr[n][j],
+ *   a[m][j] = sx[m][b_j] (qx[m][S_j] - zx[m][b_j]), b' = the weight group
+ *   holding group b (the per-channel scale sw[n] when group == 0), all in fp32.
+ *  Xq       device, [M][K/2] unsigned codes (hq_rotate_quant_asym, group 128)
+ *  sx, zx   device, [M][K/128] fp32 scales and int32 zero points
+ *  every other argument as w4a4_linear; group 0 or a multiple of 128.
+ * Implemented for M <= 64 (the small-M kernel): HQ_ERR_UNSUPPORTED above.  The
+ * call needs no workspace.  Errors: as w4a4_linear.
+ */
+hq_status w4a4_linear_asym(const uint8_t* Xq, const float* sx, const int32_t* zx, int64_t M, int64_t K,
+                           const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
+                           int32_t group, const uint8_t* A, const uint16_t* B, const int32_t* sal_idx,
+                           int32_t r, void* Y, hq_dtype yt, void* stream);
+
+/* hq_debug_accum_asym -- the exact integer accumulators acc_b of
+ * w4a4_linear_asym, acc [M][N][K/128] int32 (no SERQ term).  Test hook. */
+hq_status hq_debug_accum_asym(const uint8_t* Xq, const int32_t* zx, int64_t M, int64_t K,
+                              const uint8_t* Wq, const uint16_t* zw, int64_t N, int32_t group,
+                              int32_t* acc, void* stream);
+
+/*
  * w4a8_linear -- w4a4_linear with the activation codes of hq_rotate_quant8:
  *   acc_b[m][n] = sum_{k in group b} q8x[m][k] * (qw[n][k] - z[b][n]),
  *   acc_c[m][n] = sum_{j<r} q8x[m][S_j] * qr[n][j],  Y as w4a4_linear.

@@ -179,3 +179,30 @@ def test_w4a8_argument_errors(L):
     assert lin8(g=96) == L.HQ_ERR_ARG
     assert lin8(Xq=ct.c_void_p(8)) == L.HQ_ERR_ALIGN
     assert lin8(M=0) == L.HQ_OK
+
+
+def test_offq_argument_errors(L):
+    # the OffQ quantiser and GEMM check on the host, before any device work
+    rq = lambda **kw: L.lib.hq_rotate_quant_asym(kw.get("X", P), kw.get("xt", 0), kw.get("M", 4), 256,
+                                                 kw.get("ld", 256), kw.get("g", 128), None, P, P,
+                                                 kw.get("zx", P), None)
+    assert rq(g=16) == L.HQ_ERR_UNSUPPORTED              # groups of 32 .. 1024
+    assert rq(g=3) == L.HQ_ERR_ARG
+    assert rq(xt=2) == L.HQ_ERR_UNSUPPORTED              # fp32 input
+    assert rq(zx=None) == L.HQ_ERR_ARG
+    assert rq(X=ct.c_void_p(18)) == L.HQ_ERR_ALIGN
+    assert rq(ld=200) == L.HQ_ERR_ARG
+    assert rq(M=0, X=None, zx=None) == L.HQ_OK
+    lin = lambda **kw: L.lib.w4a4_linear_asym(kw.get("Xq", P), kw.get("sx", P), kw.get("zx", P), kw.get("M", 16),
+                                              kw.get("K", 256), P, P, P, 128, kw.get("g", 0), P, P, P,
+                                              kw.get("r", 8), P, 1, None)
+    assert lin(M=65) == L.HQ_ERR_UNSUPPORTED             # small-M kernel only
+    assert lin(K=4096, g=2048 + 128) == L.HQ_ERR_ARG     # K % group
+    assert lin(r=12) == L.HQ_ERR_UNSUPPORTED
+    assert lin(zx=None) == L.HQ_ERR_ARG
+    assert lin(zx=ct.c_void_p(18)) == L.HQ_ERR_ALIGN
+    assert lin(M=0) == L.HQ_OK
+    acc = lambda **kw: L.lib.hq_debug_accum_asym(P, kw.get("zx", P), kw.get("M", 4), 256, P, P, 128,
+                                                 kw.get("g", 0), P, None)
+    assert acc(M=100) == L.HQ_ERR_UNSUPPORTED
+    assert acc(zx=None) == L.HQ_ERR_ARG

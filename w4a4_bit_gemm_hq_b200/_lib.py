@@ -47,6 +47,9 @@ SIGNATURES = {
     "hq_debug_accum": ([_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32, _P, ct.c_size_t, _P],
                        _ST),
     "hq_rotate_quant8": ([_P, ct.c_int, _I64, _I64, _I64, _I32, _P, _P, _P, _P], _ST),
+    "hq_rotate_quant_asym": ([_P, ct.c_int, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P], _ST),
+    "w4a4_linear_asym": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _P, ct.c_int, _P], _ST),
+    "hq_debug_accum_asym": ([_P, _P, _I64, _I64, _P, _P, _I64, _I32, _P, _P], _ST),
     "w4a8_linear": ([_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _P, ct.c_int, _P,
                      ct.c_size_t, _P], _ST),
     "hq_debug_accum8": ([_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32, _P, ct.c_size_t, _P],

@@ -3,6 +3,7 @@
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
@@ -27,16 +28,20 @@ def build(force=False, verbose=False):
         return LIB
     bdir = os.path.join(HERE, "_build")
     os.makedirs(bdir, exist_ok=True)
-    objs = []
-    for src in SOURCES:
-        obj = os.path.join(bdir, src.replace(".cu", ".o"))
-        cmd = [NVCC, *FLAGS, "-rdc=true", "-c", os.path.join(CSRC, src), "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
+    objs = [os.path.join(bdir, src.replace(".cu", ".o")) for src in SOURCES]
+
+    def compile_one(i):
+        cmd = [NVCC, *FLAGS, "-rdc=true", "-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
+        return subprocess.run(cmd, capture_output=True, text=True)
+
+    # the sources compile independently: all at once
+    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+        results = list(ex.map(compile_one, range(len(SOURCES))))
+    for src, r in zip(SOURCES, results):
         if verbose or r.returncode:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode:
             raise RuntimeError("nvcc failed on " + src)
-        objs.append(obj)
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-rdc=true", *objs, "-o", tmp,
            "-lcudart"]

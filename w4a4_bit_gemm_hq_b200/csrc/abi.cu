@@ -191,3 +191,47 @@ extern "C" hq_status hq_debug_accum8(const int8_t* Xq8, int64_t M, int64_t K, co
     return run_gemm(a, OUT_DEBUG, decode != 0, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+
+// OffQ per-group asymmetric activations (hq_rotate_quant_asym's outputs):
+// the small-M kernel only; activation groups of 128 inputs (one K-block),
+// nested in the weight groups.
+static hq_status check_asym(const float* sx, const int32_t* zx, int64_t M, int32_t group) {
+    if (M > 64) return HQ_ERR_UNSUPPORTED;   // the large-M kernel has no OffQ mode
+    if (group != 0 && group % 128 != 0) return HQ_ERR_UNSUPPORTED;
+    if (M > 0 && (!zx || !sx)) return HQ_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(zx) & 3u) || (reinterpret_cast<uintptr_t>(sx) & 3u)) return HQ_ERR_ALIGN;
+    return HQ_OK;
+}
+
+extern "C" hq_status w4a4_linear_asym(const uint8_t* Xq, const float* sx, const int32_t* zx, int64_t M, int64_t K,
+                                      const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
+                                      int32_t group, const uint8_t* A, const uint16_t* B, const int32_t* sal_idx,
+                                      int32_t r, void* Y, hq_dtype yt, void* stream) {
+    hq_status s = check_linear(Xq, sx, M, K, Wq, sw, zw, N, group, A, B, sal_idx, r, Y, yt);
+    if (s != HQ_OK) return s;
+    s = check_asym(sx, zx, M, group);
+    if (s != HQ_OK) return s;
+    if (M == 0 || N == 0) return HQ_OK;
+    GemmArgs a{};
+    a.Xq = Xq; a.sx = sx; a.zx = zx; a.Wq = Wq; a.sw = sw; a.zw = zw; a.Rq = A; a.sr = B; a.sal = sal_idx;
+    a.Y = Y;
+    a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
+    a.act_bits = 4;
+    return run_gemm(a, yt, true, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hq_status hq_debug_accum_asym(const uint8_t* Xq, const int32_t* zx, int64_t M, int64_t K,
+                                         const uint8_t* Wq, const uint16_t* zw, int64_t N, int32_t group,
+                                         int32_t* acc, void* stream) {
+    hq_status s = check_gemm(Xq, M, K, Wq, zw, N, group, nullptr, nullptr, 0);
+    if (s != HQ_OK) return s;
+    if (M > 64 || (group != 0 && group % 128 != 0)) return HQ_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return HQ_OK;
+    if (!acc || !zx) return HQ_ERR_ARG;
+    GemmArgs a{};
+    a.Xq = Xq; a.zx = zx; a.Wq = Wq; a.zw = zw;
+    a.dbg_acc = acc;
+    a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = 0;
+    a.act_bits = 4;
+    return run_gemm(a, OUT_DEBUG, true, nullptr, 0, static_cast<cudaStream_t>(stream));
+}

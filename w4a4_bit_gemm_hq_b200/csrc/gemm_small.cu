@@ -50,8 +50,15 @@
 //    the fragment loads hit distinct banks); when they do not fit, each
 //    thread loads its fragments through L1, prefetched 8 K-blocks ahead.
 //  * the warps of a tile add their partial sums in shared memory in a fixed
-//    order; the finish adds the SERQ term X[m,S] . Rq[n,:] (dp4a), multiplies
-//    by sx[m] and stores.
+//    order; one warp per tile finishes: the SERQ term X[m,S] . Rq[n,:] on
+//    mma.sync, sx[m], the store.
+//  * OffQ activations (OQ): unsigned codes with a scale and an integer zero
+//    point per token and 128-input group, i.e. per K-block.  Per K-block the
+//    accumulator is acc = raw - zw Sx - zx (Su - 128 zw), raw the MMA of the
+//    unsigned codes, Sx the token's code sum, Su the weight row's code sum
+//    (dp4a in the lanes, two shuffles), and it is scaled by sx[m][b] sw[n]
+//    there; the SERQ term is an fp32 dot product of the dequantised salient
+//    activations with the Rq rows ("OffQ ...", Methodology 2-3).
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -89,7 +96,8 @@ struct DkCfg {
     static constexpr int F_SR = F_RQ + MAXROWS * 32;
     static constexpr int F_SW = F_SR + (MAXROWS + 8) * 2;
     static constexpr int F_SX = F_SW + (MAXROWS + 8) * 2;
-    static constexpr int FIX = (F_SX + NT * 4 + 15) / 16 * 16;
+    static constexpr int F_AS = (F_SX + NT * 4 + 15) / 16 * 16;       // OffQ: [NT][64] dequantised salient activations
+    static constexpr int FIX = F_AS + NT * 64 * 4;
     static constexpr int XITEMS = (NT * dk::XS_WORDS + THREADS - 1) / THREADS;
 };
 
@@ -105,7 +113,7 @@ static int nt_for(int64_t M) { return M <= 8 ? 8 : (M <= 16 ? 16 : (M <= 32 ? 32
 
 // Launch plan; `staged` tells whether the tokens fit in shared memory.
 template <int NT>
-static DkPlan dk_plan(int64_t M, int64_t N, int64_t K, bool a8, int nsm, bool& staged) {
+static DkPlan dk_plan(int64_t M, int64_t N, int64_t K, bool a8, int nsm, bool& staged, bool oq = false) {
     using C = DkCfg<NT>;
     DkPlan p{};
     const int want = nsm > 0 ? nsm : 148;
@@ -113,9 +121,10 @@ static DkPlan dk_plan(int64_t M, int64_t N, int64_t K, bool a8, int nsm, bool& s
     p.grid = static_cast<int>(tiles < want ? tiles : want);
     p.tstride = static_cast<int>(a8 ? K : K / 2) + 64;
     // staged token rows, then their code sums per K-block (int32 [K/128][NT])
-    const int64_t tok = static_cast<int64_t>(NT) * p.tstride + (K / dk::BK) * NT * 4;
+    // (OffQ activations: then their zero points and group scales, [K/128][NT] each)
+    const int64_t tok = static_cast<int64_t>(NT) * p.tstride + (K / dk::BK) * NT * (oq ? 12 : 4);
     const int depths[3] = {8, 4, 2};
-    for (int st = 1; st >= 0; --st) {
+    for (int st = 1; st >= (oq ? 1 : 0); --st) {
         for (int d : depths) {
             if (st && d < 4 && C::TPW == 1) continue;
             const int64_t ring = static_cast<int64_t>(C::W) * d * C::SLOT;
@@ -170,8 +179,9 @@ __device__ __forceinline__ void cp_async_wait_depth(int D) {
 
 // A8: 8-bit activation codes ([M][K] int8, used as they are) instead of packed
 // 4-bit codes (expanded as 16 q).  TS: tokens staged in shared memory.
-template <int NT, bool ASYM, bool A8, int OUT, bool TS>
+template <int NT, bool ASYM, bool A8, int OUT, bool TS, bool OQ = false>
 __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const GemmArgs p, const DkPlan plan) {
+    static_assert(!OQ || (TS && !A8), "OffQ activations: staged 4-bit tokens");
     using C = DkCfg<NT>;
     constexpr int NTT = C::NTT;
     constexpr int W = C::W;
@@ -187,6 +197,9 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
     float* sx_s = reinterpret_cast<float*>(fix + C::F_SX);
     uint8_t* tok_s = fix + C::FIX;
     int32_t* tsum_s = reinterpret_cast<int32_t*>(tok_s + NT * plan.tstride);   // [K/128][NT]
+    int32_t* zxg_s = tsum_s + (p.K / dk::BK) * NT;                            // OffQ: [K/128][NT] zero points
+    float* sxg_s = reinterpret_cast<float*>(zxg_s + (p.K / dk::BK) * NT);     // OffQ: [K/128][NT] group scales
+    float* as_s = reinterpret_cast<float*>(fix + C::F_AS);                    // OffQ: [NT][64]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
     const int cta = blockIdx.x;
@@ -198,9 +211,9 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
     const int G = ASYM ? p.K / p.gw : 1;
     const int64_t xrow = A8 ? p.K : p.K / 2;           // bytes per token row
     const int D = plan.D;
-    // the accumulators carry the factor 16 of 4-bit activation codes
-    constexpr int sh = A8 ? 0 : 4;
-    constexpr float inv_act = A8 ? 1.0f : 0.0625f;
+    // the accumulators carry the factor 16 of 4-bit signed activation codes
+    constexpr int sh = (A8 || OQ) ? 0 : 4;
+    constexpr float inv_act = (A8 || OQ) ? 1.0f : 0.0625f;
 
     if constexpr (TS) {
         if (tid == 0) {
@@ -268,7 +281,24 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
             }
             xsw[it] = word;
         }
-        if constexpr (OUT != OUT_DEBUG) {   // the debug entry passes no scales
+        if constexpr (OQ) {
+            // dequantised salient activations sx[m][b] (q - zx[m][b]), b = S_j / 128
+            const int KB_ = p.K / dk::BK;
+            for (int idx = tid; idx < NT * 64; idx += C::THREADS) {
+                const int m = idx >> 6, j = idx & 63;
+                float a = 0.f;
+                if (m < p.M && j < p.r) {
+                    const int k = __ldg(p.sal + j);
+                    if (static_cast<unsigned>(k) < static_cast<unsigned>(p.K)) {
+                        const int b = k / dk::BK;
+                        const int q = (__ldg(p.Xq + static_cast<int64_t>(m) * xrow + (k >> 1)) >> ((k & 1) * 4)) & 0xF;
+                        const float sg = OUT == OUT_DEBUG ? 0.f : __ldg(p.sx + static_cast<int64_t>(m) * KB_ + b);
+                        a = __fmul_rn(sg, static_cast<float>(q - __ldg(p.zx + static_cast<int64_t>(m) * KB_ + b)));
+                    }
+                }
+                as_s[idx] = a;
+            }
+        } else if constexpr (OUT != OUT_DEBUG) {   // the debug entry passes no scales
             for (int m = tid; m < NT; m += C::THREADS) sx_s[m] = m < p.M ? p.sx[m] : 0.f;
         }
         gathered = true;
@@ -410,12 +440,17 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                             if constexpr (A8) {
                                 sum = __dp4a(static_cast<int>(w[e]), 0x01010101, sum);
                             } else {
-                                const uint32_t u = w[e] ^ 0x88888888u;   // q + 8 per nibble
+                                const uint32_t u = OQ ? w[e] : w[e] ^ 0x88888888u;   // q (+ 8 for signed codes) per nibble
                                 sum = __dp4a(static_cast<int>((u & 0x0F0F0F0Fu) + ((u >> 4) & 0x0F0F0F0Fu)), 0x01010101, sum);
                             }
                         }
                     }
-                    tsum_s[idx] = A8 ? sum : 16 * (sum - 8 * dk::BK);
+                    tsum_s[idx] = (A8 || OQ) ? sum : 16 * (sum - 8 * dk::BK);
+                    if constexpr (OQ) {
+                        const bool mv = m < p.M;
+                        zxg_s[idx] = mv ? __ldg(p.zx + static_cast<int64_t>(m) * KB + kbs) : 0;
+                        sxg_s[idx] = (mv && OUT != OUT_DEBUG) ? __ldg(p.sx + static_cast<int64_t>(m) * KB + kbs) : 0.f;
+                    }
                 }
                 named_bar_sync(1, nact);
                 tok_ready = true;
@@ -464,6 +499,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                         }
                     }
                 }
+                int su[TPW][2] = {};   // OffQ: this lane's share of the rows' code sums
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     // A fragments of step s: unsigned codes u (per-channel: signed code + 8)
@@ -478,6 +514,10 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                         af[j][1] = fb & 0x0F0F0F0Fu;
                         af[j][2] = (fa >> 4) & 0x0F0F0F0Fu;
                         af[j][3] = (fb >> 4) & 0x0F0F0F0Fu;
+                        if constexpr (OQ) {
+                            su[j][0] = __dp4a(static_cast<int>(af[j][0] + af[j][2]), 0x01010101, su[j][0]);
+                            su[j][1] = __dp4a(static_cast<int>(af[j][1] + af[j][3]), 0x01010101, su[j][1]);
+                        }
                     }
 #pragma unroll
                     for (int nt = 0; nt < NTT; ++nt) {
@@ -486,13 +526,17 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                             const uint4 t0v = tn[nt][0], t1v = tn[nt][TOKV - 1];
                             const uint32_t x[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
                             tok_words8(x[2 * s], x[2 * s + 1], b0, b1);
+                        } else if constexpr (OQ) {
+                            const uint32_t x[4] = {tn[nt][0].x, tn[nt][0].y, tn[nt][0].z, tn[nt][0].w};
+                            b0 = x[s] & 0x0F0F0F0Fu;           // unsigned codes, (k0 k2 k4 k6)
+                            b1 = (x[s] >> 4) & 0x0F0F0F0Fu;    // (k1 k3 k5 k7)
                         } else {
                             const uint32_t x[4] = {tn[nt][0].x, tn[nt][0].y, tn[nt][0].z, tn[nt][0].w};
                             unpack_s4x8_times16(x[s], b0, b1);
                         }
                         if (fresh && s == 0) {
 #pragma unroll
-                            for (int j = 0; j < TPW; ++j) mma_s8_c(acc[j][nt], af[j], b0, b1, ASYM ? mag4 : zero4);
+                            for (int j = 0; j < TPW; ++j) mma_s8_c(acc[j][nt], af[j], b0, b1, (ASYM || OQ) ? mag4 : zero4);
                             if constexpr (!TS) mma_s8_c(ssum[nt], ones, b0, b1, ASYM ? mag4 : zero4);
                         } else {
 #pragma unroll
@@ -511,7 +555,49 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                 }
                 fresh = false;
                 if (!gathered) gather();
-                if constexpr (ASYM) {
+                if constexpr (OQ) {
+                    // one activation group per K-block: acc = raw - zw Sx - zx (Su - 128 zw),
+                    // scaled by sx[m][b] sw[n] (per-channel weights: sw at the end)
+#pragma unroll
+                    for (int j = 0; j < TPW; ++j) {
+                        int sua = su[j][0], sub = su[j][1];
+                        sua += __shfl_xor_sync(0xFFFFFFFFu, sua, 1);
+                        sua += __shfl_xor_sync(0xFFFFFFFFu, sua, 2);
+                        sub += __shfl_xor_sync(0xFFFFFFFFu, sub, 1);
+                        sub += __shfl_xor_sync(0xFFFFFFFFu, sub, 2);
+                        const int zia = ASYM ? static_cast<int>(__half2float(__ushort_as_half(static_cast<uint16_t>(za[j] & 0xFFFFu)))) : 8;
+                        const int zib = ASYM ? static_cast<int>(__half2float(__ushort_as_half(static_cast<uint16_t>(za[j] >> 16)))) : 8;
+                        const int sua2 = sua - dk::BK * zia, sub2 = sub - dk::BK * zib;
+                        float swa = 1.f, swb = 1.f;
+                        if constexpr (ASYM && OUT != OUT_DEBUG) {
+                            swa = __half2float(__ushort_as_half(static_cast<uint16_t>(sa[j] & 0xFFFFu)));
+                            swb = __half2float(__ushort_as_half(static_cast<uint16_t>(sa[j] >> 16)));
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NTT; ++nt) {
+                            const int ti = kb * NT + 8 * nt + 2 * tq;
+                            const int2 sxk = *reinterpret_cast<const int2*>(tsum_s + ti);
+                            const int2 zk = *reinterpret_cast<const int2*>(zxg_s + ti);
+                            const float2 gk = *reinterpret_cast<const float2*>(sxg_s + ti);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                const int tsx = (v & 1) ? sxk.y : sxk.x, tzx = (v & 1) ? zk.y : zk.x;
+                                const int a = static_cast<int>(acc[j][nt][v] - dk::MAGIC) - (v < 2 ? zia : zib) * tsx -
+                                              tzx * (v < 2 ? sua2 : sub2);
+                                if constexpr (OUT == OUT_DEBUG) {
+                                    const int m = 8 * nt + 2 * tq + (v & 1);
+                                    const int n = v < 2 ? rowA[j] : rowB[j];
+                                    if ((v < 2 ? okA[j] : okB[j]) && m < p.M)
+                                        atomicAdd(p.dbg_acc + (static_cast<int64_t>(m) * p.N + n) * KB + kb, a);
+                                } else {
+                                    const float coef = __fmul_rn((v & 1) ? gk.y : gk.x, v < 2 ? swa : swb);
+                                    y[j][nt][v] = __fmaf_rn(coef, static_cast<float>(a), y[j][nt][v]);
+                                }
+                            }
+                        }
+                    }
+                    fresh = true;
+                } else if constexpr (ASYM) {
                     const bool gend = ++cgk == gs;
                     if (gend) cgk = 0;
                     if (gend || kb + 1 == kb1) {
@@ -563,7 +649,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                     }
                 }
             }
-            if constexpr (!ASYM) {
+            if constexpr (!ASYM && !OQ) {
                 // per-channel: signed code = u - 8, exact integer partial sums
                 if (kb1 > kb0) {
 #pragma unroll
@@ -588,7 +674,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
 #pragma unroll
                 for (int nt = 0; nt < NTT; ++nt)
                     part[j * NTT + nt] =
-                        ASYM ? make_uint4(__float_as_uint(y[j][nt][0]), __float_as_uint(y[j][nt][1]),
+                        (ASYM || OQ) ? make_uint4(__float_as_uint(y[j][nt][0]), __float_as_uint(y[j][nt][1]),
                                           __float_as_uint(y[j][nt][2]), __float_as_uint(y[j][nt][3]))
                              : make_uint4(yi[j][nt][0], yi[j][nt][1], yi[j][nt][2], yi[j][nt][3]);
         }
@@ -614,7 +700,7 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                         const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            if constexpr (ASYM) ys[q] = __fadd_rn(ys[q], __uint_as_float(vv[q]));
+                            if constexpr (ASYM || OQ) ys[q] = __fadd_rn(ys[q], __uint_as_float(vv[q]));
                             else yis[q] += static_cast<int32_t>(vv[q]);
                         }
                     }
@@ -632,7 +718,28 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                 uint32_t cc[NTT][4];
 #pragma unroll
                 for (int nt = 0; nt < NTT; ++nt) cc[nt][0] = cc[nt][1] = cc[nt][2] = cc[nt][3] = 0;
-                if (p.r > 0) {
+                if constexpr (OQ) {
+                    // fp32 SERQ term: sum_j a[m][j] qr[n][j] with the dequantised salient activations
+                    if constexpr (OUT != OUT_DEBUG) {
+#pragma unroll
+                        for (int nt = 0; nt < NTT; ++nt) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int m = 8 * nt + 2 * tq + (q & 1);
+                                const int n = q < 2 ? nA : nB;
+                                float c = 0.f;
+                                if (n < pr1) {
+                                    const uint8_t* rq = rq_s + (n - pr0) * (p.r / 2);
+                                    for (int jj = 0; jj < p.r; ++jj) {
+                                        const int code = ((static_cast<int>(rq[jj >> 1]) >> ((jj & 1) * 4)) & 0xF) ^ 8;
+                                        c = __fmaf_rn(as_s[m * 64 + jj], static_cast<float>(code - 8), c);
+                                    }
+                                }
+                                cc[nt][q] = __float_as_uint(c);
+                            }
+                        }
+                    }
+                } else if (p.r > 0) {
                     const uint32_t* rqA = reinterpret_cast<const uint32_t*>(rq_s + (nA - pr0) * (p.r / 2));
                     const uint32_t* rqB = reinterpret_cast<const uint32_t*>(rq_s + (nB - pr0) * (p.r / 2));
 #pragma unroll
@@ -663,7 +770,14 @@ __global__ void __launch_bounds__(DkCfg<NT>::THREADS, 1) k_gemm_small(const Gemm
                         if (n >= pr1 || m >= p.M) continue;
                         const int c = static_cast<int32_t>(cc[nt][q]) >> 4;
                         const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                        if constexpr (OUT == OUT_DEBUG) {
+                        if constexpr (OQ) {
+                            if constexpr (OUT != OUT_DEBUG) {
+                                const float srn = p.r > 0 ? __half2float(__ushort_as_half(sr_s[n - pb])) : 0.f;
+                                const float base = ASYM ? y[j][nt][q]
+                                                        : __fmul_rn(__half2float(__ushort_as_half(sw_s[n - pb])), y[j][nt][q]);
+                                store_one<OUT>(p.Y, o, __fmaf_rn(srn, __uint_as_float(cc[nt][q]), base));
+                            }
+                        } else if constexpr (OUT == OUT_DEBUG) {
                             if constexpr (!ASYM) p.dbg_acc[o] = yi[j][nt][q] >> sh;
                             if (p.r > 0) p.dbg_acc_c[o] = c;
                         } else {
@@ -693,9 +807,9 @@ bool small_supported(int64_t M, int gw) {
 
 size_t small_workspace_bytes(int64_t, int64_t, int64_t, int, int) { return 0; }
 
-template <int NT, bool ASYM, bool A8, int OUT, bool TS>
+template <int NT, bool ASYM, bool A8, int OUT, bool TS, bool OQ = false>
 static hq_status launch_sk_ts(const GemmArgs& a, const DkPlan& plan, cudaStream_t st) {
-    auto kern = k_gemm_small<NT, ASYM, A8, OUT, TS>;
+    auto kern = k_gemm_small<NT, ASYM, A8, OUT, TS, OQ>;
     const int smem = plan.ring + DkCfg<NT>::FIX + plan.tbytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
@@ -719,14 +833,19 @@ static hq_status launch_sk_ts(const GemmArgs& a, const DkPlan& plan, cudaStream_
 
 template <int NT, bool ASYM, bool A8, int OUT>
 static hq_status launch_sk_t(const GemmArgs& a, cudaStream_t st, int nsm) {
+    const bool oq = a.zx != nullptr;   // OffQ activations
     bool staged = false;
-    const DkPlan plan = dk_plan<NT>(a.M, a.N, a.K, A8, nsm, staged);
+    const DkPlan plan = dk_plan<NT>(a.M, a.N, a.K, A8, nsm, staged, oq);
     if (plan.D == 0) return HQ_ERR_UNSUPPORTED;
     // the debug entry adds the partial group sums of the warps with atomics
-    if (OUT == OUT_DEBUG && ASYM &&
-        cudaMemsetAsync(a.dbg_acc, 0, static_cast<size_t>(a.M) * a.N * (a.K / a.gw) * sizeof(int32_t), st) !=
-            cudaSuccess)
+    const int64_t G = oq ? a.K / dk::BK : (ASYM ? a.K / a.gw : 0);
+    if (OUT == OUT_DEBUG && G > 0 &&
+        cudaMemsetAsync(a.dbg_acc, 0, static_cast<size_t>(a.M) * a.N * G * sizeof(int32_t), st) != cudaSuccess)
         return HQ_ERR_CUDA;
+    if (oq) {
+        if constexpr (A8) return HQ_ERR_UNSUPPORTED;
+        else return launch_sk_ts<NT, ASYM, false, OUT, true, true>(a, plan, st);
+    }
     return staged ? launch_sk_ts<NT, ASYM, A8, OUT, true>(a, plan, st)
                   : launch_sk_ts<NT, ASYM, A8, OUT, false>(a, plan, st);
 }

@@ -13,7 +13,8 @@ constexpr int OUT_DEBUG = 3;  // epilogue variant that stores raw integer accumu
 
 struct GemmArgs {
     const uint8_t* Xq;      // [M][K/2] packed activation codes ([M][K] int8 when act_bits == 8)
-    const float* sx;        // [M]
+    const float* sx;        // [M]; OffQ activations: [M][K/128], one scale per token and 128-input group
+    const int32_t* zx;      // OffQ activations: [M][K/128] integer zero points (else NULL)
     const uint8_t* Wq;      // [N][K/2] packed weight codes
     const uint16_t* sw;     // fp16 bits, [N] or [K/gw][N]
     const uint16_t* zw;     // fp16 bits, [K/gw][N] (gw > 0)
@@ -28,14 +29,6 @@ struct GemmArgs {
     int act_bits;           // 4: Xq packed int4 [M][K/2]; 8: Xq int8 codes [M][K] (W4A8)
     uint64_t limit_ns;      // bounded-wait limit
 };
-
-// Bytes at the start of the small-M kernel's workspace holding its per-tile
-// arrival counters (one uint32 per 128-row weight tile, padded to 16 bytes);
-// the partial sums follow.  Every call leaves the counters at zero.
-__host__ __device__ inline size_t small_counter_bytes(int64_t ntiles) {
-    return static_cast<size_t>((ntiles * 4 + 15) / 16 * 16);
-}
-inline size_t small_counter_bytes_for_n(int64_t N) { return small_counter_bytes((N + 127) / 128); }
 
 hq_status check_linear(const uint8_t* Xq, const float* sx, int64_t M, int64_t K, const uint8_t* Wq,
                        const uint16_t* sw, const uint16_t* zw, int64_t N, int32_t group, const uint8_t* A,

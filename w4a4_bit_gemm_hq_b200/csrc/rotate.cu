@@ -26,7 +26,9 @@ namespace hq {
 
 constexpr int EPT = 32;  // channels per thread
 
-enum { MODE_QUANT = 0, MODE_ROTATE = 1, MODE_SQNORM = 2, MODE_QUANT8 = 3 };   // QUANT8: one 8-bit code per byte
+// QUANT8: one 8-bit code per byte; QUANT_ASYM: OffQ's per-group asymmetric
+// 4-bit codes with a scale and an integer zero point per group
+enum { MODE_QUANT = 0, MODE_ROTATE = 1, MODE_SQNORM = 2, MODE_QUANT8 = 3, MODE_QUANT_ASYM = 4 };
 enum { XT_F16 = 0, XT_BF16 = 1, XT_F32 = 2 };
 
 __device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
@@ -69,7 +71,8 @@ __device__ __forceinline__ float2 f2add_rn(float2 a, float2 b) {
 template <int G, int XT, int MODE>
 __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int64_t M, int64_t K, int64_t ldx,
                                                  const int8_t* __restrict__ dsign, uint8_t* __restrict__ Xq,
-                                                 float* __restrict__ sx, float* __restrict__ out, float cg) {
+                                                 float* __restrict__ sx, float* __restrict__ out, float cg,
+                                                 int32_t* __restrict__ zx) {
     constexpr int TPG = (G > EPT) ? G / EPT : 1;     // threads per group
     constexpr int HREG = (G < EPT) ? G : EPT;        // in-register stages: h < HREG
     constexpr int TSHFL = (TPG < 32) ? TPG : 32;     // shuffle stages: s < TSHFL
@@ -357,7 +360,50 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
                 }
             }
 
-            if constexpr (MODE == MODE_ROTATE) {
+            if constexpr (MODE == MODE_QUANT_ASYM) {
+                // OffQ per-group asymmetric codes (groups of 32..1024 channels: the
+                // TPG threads of a group sit in one warp).  The group's own range
+                // [lo, hi] sets the step; the offset the all-ones row of H
+                // created goes into the integer zero point (not clamped); a
+                // constant group takes the step |lo| / 15 (1 when it is zero).
+                float lo = v[0].x, hi = v[0].x;
+    #pragma unroll
+                for (int i = 0; i < EPT / 2; ++i) {
+                    lo = fminf(lo, fminf(v[i].x, v[i].y));
+                    hi = fmaxf(hi, fmaxf(v[i].x, v[i].y));
+                }
+    #pragma unroll
+                for (int o = 1; o < TPG; o <<= 1) {
+                    lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+                    hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+                }
+                float dlt = __fsub_rn(hi, lo);
+                if (dlt == 0.f) dlt = lo != 0.f ? fabsf(lo) : 15.f;
+                const float inv = __fdiv_rn(15.f, dlt);
+                const float zf = rintf(__fmul_rn(-lo, inv));
+                uint32_t words[EPT / 8];
+    #pragma unroll
+                for (int j = 0; j < EPT / 8; ++j) {
+                    uint32_t w = 0;
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // q = clamp(rint(fl32(u * inv)) + z, 0, 15); the multiply is
+                        // rounded on its own (never merged into an fma)
+                        const float q0 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(v[4 * j + e].x, inv)), zf), 0.f), 15.f);
+                        const float q1 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(v[4 * j + e].y, inv)), zf), 0.f), 15.f);
+                        w |= (static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << 4)) << (8 * e);
+                    }
+                    words[j] = w;
+                }
+                if (active) {
+                    *reinterpret_cast<uint4*>(Xq + m * (K / 2) + col0 / 2) = make_uint4(words[0], words[1], words[2], words[3]);
+                    if (t % TPG == 0) {
+                        const int64_t gi = m * (K / G) + col0 / G;
+                        sx[gi] = __fmul_rn(__fdiv_rn(dlt, 15.f), cg);
+                        zx[gi] = static_cast<int32_t>(zf);
+                    }
+                }
+            } else if constexpr (MODE == MODE_ROTATE) {
                 if (active) {
                     float4* dst = reinterpret_cast<float4*>(out + m * K + col0);
                     const float2 c2 = make_float2(cg, cg);
@@ -472,7 +518,7 @@ __global__ void __launch_bounds__(512) k_rotate(const void* __restrict__ X, int6
 // ------------------------------------------------------------------ dispatch
 template <int XT, int MODE>
 static hq_status launch_g(int group, const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* d, uint8_t* Xq,
-                          float* sx, float* out, cudaStream_t st) {
+                          float* sx, float* out, cudaStream_t st, int32_t* zx = nullptr) {
     const int threads = static_cast<int>(((K / EPT) + 31) / 32 * 32);
     const float cg = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(group)));
     // G >= 2048: exchange area of EPT floats per thread; G == 4096 uses two
@@ -492,9 +538,20 @@ static hq_status launch_g(int group, const void* X, int64_t M, int64_t K, int64_
             return HQ_ERR_CUDA;
         int64_t grid = static_cast<int64_t>(per_sm) * nsm;
         if (grid > M) grid = M;
-        kern<<<static_cast<unsigned>(grid), threads, shm, st>>>(X, M, K, ldx, d, Xq, sx, out, cg);
+        kern<<<static_cast<unsigned>(grid), threads, shm, st>>>(X, M, K, ldx, d, Xq, sx, out, cg, zx);
         return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
     };
+    if constexpr (MODE == MODE_QUANT_ASYM) {   // groups inside one warp, at least one thread each
+        switch (group) {
+            case 32: return run(k_rotate<32, XT, MODE>);
+            case 64: return run(k_rotate<64, XT, MODE>);
+            case 128: return run(k_rotate<128, XT, MODE>);
+            case 256: return run(k_rotate<256, XT, MODE>);
+            case 512: return run(k_rotate<512, XT, MODE>);
+            case 1024: return run(k_rotate<1024, XT, MODE>);
+            default: return HQ_ERR_UNSUPPORTED;
+        }
+    }
     switch (group) {
         case 8: return run(k_rotate<8, XT, MODE>);
         case 16: return run(k_rotate<16, XT, MODE>);
@@ -512,10 +569,10 @@ static hq_status launch_g(int group, const void* X, int64_t M, int64_t K, int64_
 
 template <int MODE>
 static hq_status launch_rotate(int xt, int group, const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* d,
-                               uint8_t* Xq, float* sx, float* out, cudaStream_t st) {
-    if (xt == HQ_F16) return launch_g<XT_F16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
-    if (xt == HQ_BF16) return launch_g<XT_BF16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
-    if constexpr (MODE != MODE_QUANT && MODE != MODE_QUANT8) {
+                               uint8_t* Xq, float* sx, float* out, cudaStream_t st, int32_t* zx = nullptr) {
+    if (xt == HQ_F16) return launch_g<XT_F16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st, zx);
+    if (xt == HQ_BF16) return launch_g<XT_BF16, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st, zx);
+    if constexpr (MODE != MODE_QUANT && MODE != MODE_QUANT8 && MODE != MODE_QUANT_ASYM) {
         if (xt == HQ_F32) return launch_g<XT_F32, MODE>(group, X, M, K, ldx, d, Xq, sx, out, st);
     }
     return HQ_ERR_UNSUPPORTED;
@@ -575,6 +632,20 @@ extern "C" hq_status hq_rotate_quant8(const void* X, hq_dtype xt, int64_t M, int
                                           2000000000ull, 8);
     return launch_rotate<MODE_QUANT8>(xt, group, X, M, K, ld_x, H_signs, q, sx, nullptr,
                                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" hq_status hq_rotate_quant_asym(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                                          int32_t group, const int8_t* H_signs, uint8_t* Xq, float* sx, int32_t* zx,
+                                          void* stream) {
+    hq_status s = check_rotate_args(xt, M, K, group);
+    if (s != HQ_OK) return s;
+    if (xt == HQ_F32 || group < 32 || group > 1024) return HQ_ERR_UNSUPPORTED;
+    if (ld_x < K) return HQ_ERR_ARG;
+    if (M == 0) return HQ_OK;
+    if (!X || !Xq || !sx || !zx) return HQ_ERR_ARG;
+    if (!al16(X) || !al16(Xq) || (ld_x * 2) % 16 != 0) return HQ_ERR_ALIGN;
+    return launch_rotate<MODE_QUANT_ASYM>(xt, group, X, M, K, ld_x, H_signs, Xq, sx, nullptr,
+                                          static_cast<cudaStream_t>(stream), zx);
 }
 
 extern "C" hq_status hq_rotate(const void* X, hq_dtype xt, int64_t M, int64_t K, int32_t group,

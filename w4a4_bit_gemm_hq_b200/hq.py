@@ -20,7 +20,8 @@ __all__ = [
     "HQError", "hq_rotate_quant", "hq_rotate", "hq_channel_sqnorm", "hq_select_salient", "w4_pack",
     "serq_prepare", "w4a4_linear", "hq_linear_workspace_size", "hq_debug_accum", "hq_last_device_status",
     "hq_debug_wait_probe", "hq_packed_weight_bytes", "wq_tile", "wq_untile", "W4A4Linear",
-    "hq_rotate_quant8", "w4a8_linear", "hq_debug_accum8",
+    "hq_rotate_quant8", "w4a8_linear", "hq_debug_accum8", "hq_rotate_quant_asym", "w4a4_linear_asym",
+    "hq_debug_accum_asym",
 ]
 
 
@@ -42,6 +43,18 @@ def hq_rotate_quant(X, group, H_signs=None, Xq=None, sx=None):
     check(lib.hq_rotate_quant(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), group, _signs_arg(H_signs),
                               ptr(Xq), ptr(sx), stream_handle()), "hq_rotate_quant")
     return Xq, sx
+
+
+def hq_rotate_quant_asym(X, group, H_signs=None, Xq=None, sx=None, zx=None):
+    """OffQ per-group asymmetric codes: (Xq uint8 [M, K/2] unsigned nibbles,
+    sx float32 [M, K/group], zx int32 [M, K/group])."""
+    M, K = X.shape
+    Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device) if Xq is None else Xq
+    sx = torch.empty((M, K // group), dtype=torch.float32, device=X.device) if sx is None else sx
+    zx = torch.empty((M, K // group), dtype=torch.int32, device=X.device) if zx is None else zx
+    check(lib.hq_rotate_quant_asym(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), group, _signs_arg(H_signs),
+                                   ptr(Xq), ptr(sx), ptr(zx), stream_handle()), "hq_rotate_quant_asym")
+    return Xq, sx, zx
 
 
 def hq_rotate_quant8(X, group, H_signs=None, Xq8=None, sx=None):
@@ -173,6 +186,28 @@ def w4a8_linear(Xq8, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloa
                           ptr(A) if r else None, ptr(B) if r else None, ptr(sal_idx) if r else None, r,
                           ptr(Y), dtype_code(Y.dtype), ptr(workspace), ws_bytes, stream_handle()), "w4a8_linear")
     return Y
+
+
+def w4a4_linear_asym(Xq, sx, zx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat16, Y=None):
+    """Y [M, N] from OffQ per-group asymmetric codes (hq_rotate_quant_asym with
+    group 128; M <= 64)."""
+    M, K = Xq.shape[0], Xq.shape[1] * 2
+    N = sw.shape[-1]
+    r = 0 if sal_idx is None else sal_idx.numel()
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=Xq.device)
+    check(lib.w4a4_linear_asym(ptr(Xq), ptr(sx), ptr(zx), M, K, ptr(Wq), ptr(sw), ptr(zw), N, group, ptr(A), ptr(B),
+                               ptr(sal_idx), r, ptr(Y), dtype_code(Y.dtype), stream_handle()), "w4a4_linear_asym")
+    return Y
+
+
+def hq_debug_accum_asym(Xq, zx, Wq, zw, group, N):
+    """Integer accumulators [M, N, K/128] of w4a4_linear_asym (test hook)."""
+    M, K = Xq.shape[0], Xq.shape[1] * 2
+    acc = torch.empty((M, N, K // 128), dtype=torch.int32, device=Xq.device)
+    check(lib.hq_debug_accum_asym(ptr(Xq), ptr(zx), M, K, ptr(Wq), ptr(zw), N, group, ptr(acc), stream_handle()),
+          "hq_debug_accum_asym")
+    return acc
 
 
 def hq_debug_accum8(Xq8, Wq, zw, group, A, sal_idx, N, decode=False, workspace=None):
