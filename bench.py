@@ -48,6 +48,8 @@ SUITE = [("decode", 1), ("decode", 4), ("decode", 16), ("attn", 2048), ("down", 
 # shapes where K1 and the prefill GEMM have roofline targets (M >= 2048)
 TARGET_SHAPES = [("attn", 2048), ("down", 4096), ("large", 8192)]
 K1_TARGET, K2_TARGET = 0.70, 0.60
+# shapes also measured with W4A8 and OffQ activations
+VARIANT_SHAPES = [("decode", 16), ("down", 4096)]
 DEFAULT_STEPS = 500
 NOMINAL_INT8_PER_BF16 = 2.0   # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PF nominal)
 
@@ -400,6 +402,61 @@ class Shape:
             rec["k2_frac_int8"] = rec["k2_TOPs"] / R.int8_peak
         return rec
 
+    def variants(self, decode_like):
+        """The same layers with W4A8 activations (8-bit per-token codes) and,
+        for Hadamard groups of 128, OffQ activations (per-group scale and
+        zero point): K1, K2 and step times of each."""
+        R, wl, M, P = self.R, self.wl, self.M, self.P
+        torch, hq = R.torch, R.hq
+        out = []
+        Xq8 = [torch.empty((M, wl.K), dtype=torch.int8, device=R.dev) for _ in range(P)]
+        k1_8 = lambda i: hq.hq_rotate_quant8(self.X[i], wl.g, self.layers[i].H_signs, Xq8[i], self.sx[i])
+
+        def k2_8(i):
+            L = self.layers[i]
+            hq.w4a8_linear(Xq8[i], self.sx[i], L.Wq, L.sw, L.zw, L.gw, L.Rq, L.sr, L.sal_idx, self.xdt, self.Y[i],
+                           self.ws[i])
+        b1 = 2 * M * wl.K + M * wl.K + 4 * M
+        b2 = k2_bytes(M, wl.N, wl.K, wl.gw, self.r) + M * wl.K // 2
+        out.append(self._variant("w4a8", k1_8, k2_8, b1, b2, decode_like))
+        del Xq8
+        if wl.g == 128:
+            G = wl.K // 128
+            sxa = [torch.empty((M, G), dtype=torch.float32, device=R.dev) for _ in range(P)]
+            zxa = [torch.empty((M, G), dtype=torch.int32, device=R.dev) for _ in range(P)]
+            k1_a = lambda i: hq.hq_rotate_quant_asym(self.X[i], wl.g, self.layers[i].H_signs, self.Xq[i], sxa[i],
+                                                     zxa[i])
+
+            def k2_a(i):
+                L = self.layers[i]
+                hq.w4a4_linear_asym(self.Xq[i], sxa[i], zxa[i], L.Wq, L.sw, L.zw, L.gw, L.Rq, L.sr, L.sal_idx,
+                                    self.xdt, self.Y[i])
+            b1 = 2 * M * wl.K + M * wl.K // 2 + 8 * M * G
+            b2 = k2_bytes(M, wl.N, wl.K, wl.gw, self.r) + 8 * M * G - 4 * M
+            out.append(self._variant("offq", k1_a, k2_a, b1, b2, decode_like))
+            del sxa, zxa
+        return out
+
+    def _variant(self, name, k1, k2, b1, b2, decode_like):
+        R, wl, M, P = self.R, self.wl, self.M, self.P
+        for i in range(P):
+            k1(i)
+            k2(i)
+        R.torch.cuda.synchronize()
+        assert R.hq.hq_last_device_status() == 0
+        t1 = R.launch_ms(k1, P)
+        t2 = R.launch_ms(k2, P)
+        ts = R.launch_ms(lambda i: (k1(i), k2(i)), P)
+        ops = k2_ops(M, wl.N, wl.K)
+        rec = {"workload": wl.name, "M": M, "activations": name, "k1_us": t1 * 1e3, "k1_bytes": b1,
+               "k1_frac_hbm": b1 / (t1 * 1e-3) / 1e9 / R.peaks["hbm"], "k2_us": t2 * 1e3, "k2_bytes": b2,
+               "k2_TOPs": ops / (t2 * 1e-3) / 1e12, "step_us": ts * 1e3, "step_TOPS": ops / (ts * 1e-3) / 1e12}
+        if decode_like:
+            rec["k2_frac_hbm"] = b2 / (t2 * 1e-3) / 1e9 / R.peaks["hbm"]
+        else:
+            rec["k2_frac_int8"] = rec["k2_TOPs"] / R.int8_peak
+        return rec
+
     def free(self):
         for name in ("layers", "X", "Xq", "sx", "Y", "ws", "base"):
             setattr(self, name, None)
@@ -523,6 +580,7 @@ def main():
         e2e = {"value": job_tops(k2_ops(M, N, K), r * P, world, e_ms), "unit": "TOPS",
                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e_ms / (r * P)}
         del g_e2e, Xh, Yh
+    variants = [] if args.headline_only else S.variants(decode_like)
     S.free()
     del S
     torch.cuda.empty_cache()
@@ -542,6 +600,8 @@ def main():
             Sh = Shape(R, wl, M, base=base)
             base = Sh.base
             workloads.append(Sh.record(M <= 64))
+            if (name, M) in VARIANT_SHAPES:
+                variants += Sh.variants(M <= 64)
             Sh.free()
             del Sh
         base = None
@@ -602,6 +662,7 @@ def main():
         "targets": targets,
         "workloads": workloads,
         "serq_overhead": serq,
+        "activation_variants": variants,
         "peaks": {"hbm_GBs": R.peaks["hbm"], "bf16_TFs_burst": R.peaks["bf16"], "bf16_TFs_sustained": R.peaks["bf16_sus"],
                   "int8_TOPs_denominator": R.int8_peak, "source": R.peaks["src"],
                   "int8_cublaslt_8192_TOPs_live": int8_gemm_crosscheck(R)},

@@ -291,8 +291,9 @@ hq_status hq_rotate_quant_asym(const void* X, hq_dtype xt, int64_t M, int64_t K,
  *  Xq       device, [M][K/2] unsigned codes (hq_rotate_quant_asym, group 128)
  *  sx, zx   device, [M][K/128] fp32 scales and int32 zero points
  *  every other argument as w4a4_linear; group 0 or a multiple of 128.
- * Implemented for M <= 64 (the small-M kernel): HQ_ERR_UNSUPPORTED above.  The
- * call needs no workspace.  Errors: as w4a4_linear.
+ * Runs the small-M kernel once per slice of up to 64 token rows, in order on
+ * the stream (each slice streams the weights; past the first they come from L2
+ * when they fit there).  The call needs no workspace.  Errors: as w4a4_linear.
  */
 hq_status w4a4_linear_asym(const uint8_t* Xq, const float* sx, const int32_t* zx, int64_t M, int64_t K,
                            const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,

@@ -196,7 +196,7 @@ def test_offq_argument_errors(L):
     lin = lambda **kw: L.lib.w4a4_linear_asym(kw.get("Xq", P), kw.get("sx", P), kw.get("zx", P), kw.get("M", 16),
                                               kw.get("K", 256), P, P, P, 128, kw.get("g", 0), P, P, P,
                                               kw.get("r", 8), P, 1, None)
-    assert lin(M=65) == L.HQ_ERR_UNSUPPORTED             # small-M kernel only
+    assert lin(g=64) == L.HQ_ERR_UNSUPPORTED             # weight groups of 128 activation groups
     assert lin(K=4096, g=2048 + 128) == L.HQ_ERR_ARG     # K % group
     assert lin(r=12) == L.HQ_ERR_UNSUPPORTED
     assert lin(zx=None) == L.HQ_ERR_ARG
@@ -204,5 +204,5 @@ def test_offq_argument_errors(L):
     assert lin(M=0) == L.HQ_OK
     acc = lambda **kw: L.lib.hq_debug_accum_asym(P, kw.get("zx", P), kw.get("M", 4), 256, P, P, 128,
                                                  kw.get("g", 0), P, None)
-    assert acc(M=100) == L.HQ_ERR_UNSUPPORTED
+    assert acc(g=64) == L.HQ_ERR_UNSUPPORTED
     assert acc(zx=None) == L.HQ_ERR_ARG

@@ -90,6 +90,9 @@ OFFQ_CASES = [
     (33, 264, 512, 0, 24),
     (64, 1032, 1024, 256, 64),
     (8, 512, 4096, 2048, 32),
+    # more than 64 tokens: 64-row slices, the last one ragged
+    (65, 264, 512, 128, 8),
+    (200, 520, 1024, 0, 32),
 ]
 
 
@@ -117,11 +120,11 @@ def test_offq_linear_within_tolerance(M, N, K, gw, r, out):
     no_device_error()
 
 
-def test_offq_layer_decode_workload_from_raw_inputs():
-    # the decode layer (4096 -> 11008 shape class, N cut to 1024) end to end
-    # from raw activations and weights: OffQ quantiser, then the OffQ GEMM
-    wl = synth.WORKLOADS["decode"]
-    M, N = 16, 1024
+@pytest.mark.parametrize("name,M,N", [("decode", 16, 1024), ("down", 130, 256)])
+def test_offq_layer_end_to_end_from_raw_inputs(name, M, N):
+    # the layer from raw activations and weights (N cut down): OffQ quantiser,
+    # then the OffQ GEMM, through the layer class and through the two calls
+    wl = synth.WORKLOADS[name]
     X = synth.activations(wl, M=M)
     W = synth.weights(wl, N=N)
     d = synth.hadamard_signs(wl.g)
@@ -132,9 +135,14 @@ def test_offq_layer_decode_workload_from_raw_inputs():
     Xq_o, sx_o, zx_o = O.rotate_quant_asym(X, wl.xdtype, wl.g, d)
     acc_o, accc_o = O.accum_asym(Xq_o, zx_o, wl.K, wl.g, Wq_o, zw_o, wl.gw, Rq_o, sal)
     y64 = O.epilogue_asym_f64(acc_o, accc_o, wl.g, wl.gw, sx_o, sw_o, sr_o)
-    Xq, sx, zx = hq.hq_rotate_quant_asym(dev(X, wl.xdtype), wl.g, torch.from_numpy(d).cuda())
-    gi = _dev_inputs(dict(Xq=Xq_o, sx=sx_o, Wq=Wq_o, sw=sw_o, zw=zw_o, sal=sal, Rq=Rq_o, sr=sr_o))
-    Y = hq.w4a4_linear_asym(Xq, sx, zx, gi["Wq"], gi["sw"], gi["zw"], wl.gw, gi["Rq"], gi["sr"], gi["sal"],
-                            torch.float16)
+    out_dt = torch.float16 if wl.xdtype == "f16" else torch.bfloat16
+    layer = hq.W4A4Linear.prepare(dev(W, wl.wdtype), wl.g, wl.gw, wl.r, torch.from_numpy(d).cuda(),
+                                  sal_idx=torch.from_numpy(sal), out_dtype=out_dt, offq=True)
+    Y = layer(dev(X, wl.xdtype))
     assert_y_close(y_host(Y), y64, 1e-2)
+    Xq, sx, zx = hq.hq_rotate_quant_asym(dev(X, wl.xdtype), wl.g, torch.from_numpy(d).cuda())
+    assert_same(host(Xq), Xq_o, "codes")
+    gi = _dev_inputs(dict(Xq=Xq_o, sx=sx_o, Wq=Wq_o, sw=sw_o, zw=zw_o, sal=sal, Rq=Rq_o, sr=sr_o))
+    Y2 = hq.w4a4_linear_asym(Xq, sx, zx, gi["Wq"], gi["sw"], gi["zw"], wl.gw, gi["Rq"], gi["sr"], gi["sal"], out_dt)
+    assert torch.equal(Y, Y2)
     no_device_error()

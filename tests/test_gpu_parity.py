@@ -444,7 +444,8 @@ def test_layer_end_to_end_from_raw_inputs(name, M, N):
     no_device_error()
 
 
-@pytest.mark.parametrize("name,M", [("decode", 16), ("attn", 2048), ("down", 4096), ("large", 512)])
+@pytest.mark.parametrize("name,M", [("decode", 16), ("attn", 2048), ("down", 4096), ("large", 512),
+                                    ("large", 8192)])
 def test_full_size_sampled_rows(name, M):
     # the full-size layer in the configuration the benchmark times; the oracle
     # computes its own packed weights (full size) and a sample of output rows

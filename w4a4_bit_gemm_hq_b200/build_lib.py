@@ -29,15 +29,22 @@ def build(force=False, verbose=False):
     bdir = os.path.join(HERE, "_build")
     os.makedirs(bdir, exist_ok=True)
     objs = [os.path.join(bdir, src.replace(".cu", ".o")) for src in SOURCES]
+    # an object is rebuilt when it is older than its source or any header
+    headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
+    headers.append(os.path.join(HERE, "..", "include", "hq.h"))
+    t_hdr = max(os.path.getmtime(h) for h in headers)
+    todo = [i for i, src in enumerate(SOURCES)
+            if force or not os.path.exists(objs[i])
+            or os.path.getmtime(objs[i]) < max(t_hdr, os.path.getmtime(os.path.join(CSRC, src)))]
 
     def compile_one(i):
         cmd = [NVCC, *FLAGS, "-rdc=true", "-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
         return subprocess.run(cmd, capture_output=True, text=True)
 
     # the sources compile independently: all at once
-    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        results = list(ex.map(compile_one, range(len(SOURCES))))
-    for src, r in zip(SOURCES, results):
+    with ThreadPoolExecutor(max_workers=max(1, len(todo))) as ex:
+        results = list(ex.map(compile_one, todo))
+    for src, r in zip([SOURCES[i] for i in todo], results):
         if verbose or r.returncode:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode:

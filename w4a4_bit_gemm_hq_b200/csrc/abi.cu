@@ -193,15 +193,50 @@ extern "C" hq_status hq_debug_accum8(const int8_t* Xq8, int64_t M, int64_t K, co
 
 
 // OffQ per-group asymmetric activations (hq_rotate_quant_asym's outputs):
-// the small-M kernel only; activation groups of 128 inputs (one K-block),
-// nested in the weight groups.
-static hq_status check_asym(const float* sx, const int32_t* zx, int64_t M, int32_t group) {
-    if (M > 64) return HQ_ERR_UNSUPPORTED;   // the large-M kernel has no OffQ mode
+// the small-M kernel, one launch per slice of up to 64 token rows (a slice
+// reads the whole weight matrix, which stays in L2 across slices for weights
+// up to ~100 MB); activation groups of 128 inputs (one K-block), nested in the
+// weight groups.
+namespace {
+constexpr int64_t kAsymRows = 64;
+
+hq_status check_asym(const float* sx, const int32_t* zx, int64_t M, int32_t group) {
     if (group != 0 && group % 128 != 0) return HQ_ERR_UNSUPPORTED;
     if (M > 0 && (!zx || !sx)) return HQ_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(zx) & 3u) || (reinterpret_cast<uintptr_t>(sx) & 3u)) return HQ_ERR_ALIGN;
     return HQ_OK;
 }
+
+// launches the slices of rows [0, M) in order on one stream
+hq_status run_asym_slices(GemmArgs a, int64_t M, int out, size_t y_row_bytes, int64_t acc_row_elems,
+                          cudaStream_t st) {
+    const int64_t KB = a.K / 128;
+    const uint8_t* Xq = a.Xq;
+    const float* sx = a.sx;
+    const int32_t* zx = a.zx;
+    uint8_t* Y = static_cast<uint8_t*>(a.Y);
+    int32_t* acc = a.dbg_acc;
+    // the kernel stages a slice's codes in shared memory: long rows take
+    // thinner slices (an unsupported slice is rejected before any launch)
+    int64_t rows = kAsymRows;
+    for (int64_t m0 = 0; m0 < M;) {
+        a.M = static_cast<int>(M - m0 < rows ? M - m0 : rows);
+        a.Xq = Xq + m0 * (a.K / 2);
+        a.zx = zx + m0 * KB;
+        if (sx) a.sx = sx + m0 * KB;
+        if (Y) a.Y = Y + m0 * static_cast<int64_t>(y_row_bytes);
+        if (acc) a.dbg_acc = acc + m0 * acc_row_elems;
+        const hq_status s = run_gemm(a, out, true, nullptr, 0, st);
+        if (s == HQ_ERR_UNSUPPORTED && m0 == 0 && rows > 8) {
+            rows /= 2;
+            continue;
+        }
+        if (s != HQ_OK) return s;
+        m0 += rows;
+    }
+    return HQ_OK;
+}
+}  // namespace
 
 extern "C" hq_status w4a4_linear_asym(const uint8_t* Xq, const float* sx, const int32_t* zx, int64_t M, int64_t K,
                                       const uint8_t* Wq, const uint16_t* sw, const uint16_t* zw, int64_t N,
@@ -215,9 +250,10 @@ extern "C" hq_status w4a4_linear_asym(const uint8_t* Xq, const float* sx, const 
     GemmArgs a{};
     a.Xq = Xq; a.sx = sx; a.zx = zx; a.Wq = Wq; a.sw = sw; a.zw = zw; a.Rq = A; a.sr = B; a.sal = sal_idx;
     a.Y = Y;
-    a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
+    a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = r;
     a.act_bits = 4;
-    return run_gemm(a, yt, true, nullptr, 0, static_cast<cudaStream_t>(stream));
+    const size_t yrow = static_cast<size_t>(N) * (yt == HQ_F32 ? 4u : 2u);
+    return run_asym_slices(a, M, yt, yrow, 0, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" hq_status hq_debug_accum_asym(const uint8_t* Xq, const int32_t* zx, int64_t M, int64_t K,
@@ -225,13 +261,13 @@ extern "C" hq_status hq_debug_accum_asym(const uint8_t* Xq, const int32_t* zx, i
                                          int32_t* acc, void* stream) {
     hq_status s = check_gemm(Xq, M, K, Wq, zw, N, group, nullptr, nullptr, 0);
     if (s != HQ_OK) return s;
-    if (M > 64 || (group != 0 && group % 128 != 0)) return HQ_ERR_UNSUPPORTED;
+    if (group != 0 && group % 128 != 0) return HQ_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return HQ_OK;
     if (!acc || !zx) return HQ_ERR_ARG;
     GemmArgs a{};
     a.Xq = Xq; a.zx = zx; a.Wq = Wq; a.zw = zw;
     a.dbg_acc = acc;
-    a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = 0;
+    a.N = static_cast<int>(N); a.K = static_cast<int>(K); a.gw = group; a.r = 0;
     a.act_bits = 4;
-    return run_gemm(a, OUT_DEBUG, true, nullptr, 0, static_cast<cudaStream_t>(stream));
+    return run_asym_slices(a, M, OUT_DEBUG, 0, N * (K / 128), static_cast<cudaStream_t>(stream));
 }

@@ -190,7 +190,7 @@ def w4a8_linear(Xq8, sx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloa
 
 def w4a4_linear_asym(Xq, sx, zx, Wq, sw, zw, group, A, B, sal_idx, out_dtype=torch.bfloat16, Y=None):
     """Y [M, N] from OffQ per-group asymmetric codes (hq_rotate_quant_asym with
-    group 128; M <= 64)."""
+    group 128)."""
     M, K = Xq.shape[0], Xq.shape[1] * 2
     N = sw.shape[-1]
     r = 0 if sal_idx is None else sal_idx.numel()
@@ -254,8 +254,9 @@ def hq_debug_wait_probe(limit_ns):
 
 
 class W4A4Linear:
-    """A prepared W4A4 (or, with act_bits=8, W4A8) layer: rotation signs, packed
-    weights, SERQ term, workspace.
+    """A prepared W4A4 layer (W4A8 with act_bits=8; OffQ per-group asymmetric
+    4-bit activations with offq=True): rotation signs, packed weights, SERQ
+    term, workspace.
 
     ``prepare`` runs the offline steps on the GPU: fold the rotation into W,
     pack to int4, pick the r salient input channels from calibration
@@ -263,13 +264,16 @@ class W4A4Linear:
     ``forward`` is the online path: one rotate/quant launch and one GEMM launch.
     """
 
-    def __init__(self, group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype, act_bits=4):
+    def __init__(self, group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype, act_bits=4, offq=False):
         self.group, self.gw, self.H_signs = group, gw, H_signs
         self.Wq, self.sw, self.zw, self.Rq, self.sr, self.sal_idx = Wq, sw, zw, Rq, sr, sal_idx
         self.K, self.N, self.out_dtype = K, N, out_dtype
         if act_bits not in (4, 8):
             raise ValueError("act_bits must be 4 (W4A4) or 8 (W4A8)")
+        if offq and (act_bits != 4 or group != 128):
+            raise ValueError("OffQ activations are 4-bit with groups of 128 channels")
         self.act_bits = act_bits
+        self.offq = offq
         self._ws = {}
 
     @staticmethod
@@ -297,7 +301,7 @@ class W4A4Linear:
 
     @classmethod
     def prepare(cls, W, group, gw, r, H_signs=None, X_calib=None, sal_idx=None, out_dtype=torch.bfloat16,
-                act_bits=4):
+                act_bits=4, offq=False):
         N, K = W.shape
         cls.check_inputs(K, group, r, H_signs, sal_idx)
         W_rot = hq_rotate(W, group, H_signs)
@@ -311,12 +315,11 @@ class W4A4Linear:
         else:
             sal_idx, Rq, sr = None, None, None
         del W_rot
-        return cls(group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype, act_bits)
+        return cls(group, gw, H_signs, Wq, sw, zw, Rq, sr, sal_idx, K, N, out_dtype, act_bits, offq)
 
     def reset_workspaces(self):
-        """Zero the cached small-M workspaces.  Needed only after a call whose
-        device status reported HQ_ERR_TIMEOUT: a kernel that gave up may leave
-        arrival counters behind (every completed call leaves them at zero)."""
+        """Zero the cached workspaces (none is allocated while
+        hq_linear_workspace_size reports 0, as it does for every shape)."""
         for ws in self._ws.values():
             ws.zero_()
 
@@ -331,6 +334,10 @@ class W4A4Linear:
         return ws
 
     def forward(self, X, Y=None, Xq=None, sx=None):
+        if self.offq:
+            Xq, sx, zx = hq_rotate_quant_asym(X, self.group, self.H_signs, Xq, sx)
+            return w4a4_linear_asym(Xq, sx, zx, self.Wq, self.sw, self.zw, self.gw, self.Rq, self.sr,
+                                    self.sal_idx, self.out_dtype, Y)
         if self.act_bits == 8:
             Xq, sx = hq_rotate_quant8(X, self.group, self.H_signs, Xq, sx)
             return w4a8_linear(Xq, sx, self.Wq, self.sw, self.zw, self.gw, self.Rq, self.sr, self.sal_idx,
