@@ -47,6 +47,22 @@ def test_rotate_quant_asym_bit_exact(g, M, xdtype):
     no_device_error()
 
 
+@pytest.mark.parametrize("name,M", [("decode", 100), ("down", 200), ("down", 16)])
+@pytest.mark.parametrize("signed", [True, False])
+def test_rotate_quant_asym_workloads(name, M, signed):
+    # more than 64 rows of a group-128 layer run the streaming kernel (teams
+    # of one warp at K = 4096, of three at K = 11008); 16 rows the per-row one
+    wl = synth.WORKLOADS[name]
+    X = synth.activations(wl, M=M)
+    d = synth.hadamard_signs(wl.g) if signed else None
+    Xq_o, sx_o, zx_o = O.rotate_quant_asym(X, wl.xdtype, wl.g, d)
+    Xq, sx, zx = hq.hq_rotate_quant_asym(dev(X, wl.xdtype), wl.g, None if d is None else torch.from_numpy(d).cuda())
+    assert_same(host(Xq), Xq_o, "codes")
+    assert_same(host(sx), sx_o, "scales")
+    assert_same(host(zx), zx_o, "zero points")
+    no_device_error()
+
+
 def test_rotate_quant_asym_decode_workload_and_strided_rows():
     wl = synth.WORKLOADS["decode"]
     X = synth.activations(wl, M=16)

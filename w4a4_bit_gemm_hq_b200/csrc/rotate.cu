@@ -583,7 +583,7 @@ static hq_status launch_rotate(int xt, int group, const void* X, int64_t M, int6
 bool rotq_supported(int64_t M, int64_t K, int group);
 hq_status launch_rotate_quant_stream(int xt, int group, const void* X, int64_t M, int64_t K, int64_t ldx,
                                      const int8_t* d, uint8_t* Xq, float* sx, cudaStream_t st, uint64_t limit_ns,
-                                     int bits);
+                                     int bits, int32_t* zx = nullptr);
 
 static bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -644,6 +644,9 @@ extern "C" hq_status hq_rotate_quant_asym(const void* X, hq_dtype xt, int64_t M,
     if (M == 0) return HQ_OK;
     if (!X || !Xq || !sx || !zx) return HQ_ERR_ARG;
     if (!al16(X) || !al16(Xq) || (ld_x * 2) % 16 != 0) return HQ_ERR_ALIGN;
+    if (group == 128 && rotq_supported(M, K, group))
+        return launch_rotate_quant_stream(xt, group, X, M, K, ld_x, H_signs, Xq, sx, static_cast<cudaStream_t>(stream),
+                                          2000000000ull, 4, zx);
     return launch_rotate<MODE_QUANT_ASYM>(xt, group, X, M, K, ld_x, H_signs, Xq, sx, nullptr,
                                           static_cast<cudaStream_t>(stream), zx);
 }

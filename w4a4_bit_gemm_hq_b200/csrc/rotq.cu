@@ -38,6 +38,10 @@
 //    in the low nibble of the sum's bits (no borrow for q in [-7, 7]); two such
 //    nibbles form a byte with one integer multiply-add, four bytes a word with
 //    a byte permute, and xor 0x88 turns offset-8 nibbles into two's complement.
+//  * OffQ mode (ASYM, groups of 128): a thread's 128 channels are one group,
+//    so its scale and zero point come from its own registers (3-input
+//    min / max), and the codes follow the per-group sequence
+//    q = clamp(rint(fl32(u * inv)) + z, 0, 15) in fp32, as the per-row kernel.
 //  * every wait on a row slot is bounded; on timeout the status word records
 //    HQ_ERR_TIMEOUT, the team stops, and the leader waits (bounded) for its
 //    copies in flight before the CTA exits.
@@ -97,6 +101,18 @@ __device__ __forceinline__ float2 rq_fma2(float2 a, float2 b, float2 c) { return
 // first negate both lanes with separate instructions)
 __device__ __forceinline__ float2 rq_sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
 
+// min(a, b, c), max(a, b, c)
+__device__ __forceinline__ float rq_min3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float rq_max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // max(|a|, |b|, |c|)
 __device__ __forceinline__ float rq_max3abs(float a, float b, float c) {
     float r;
@@ -129,12 +145,14 @@ __host__ __device__ inline RqLayout rq_layout(int K, int teams, int npat) {
 
 // G: Hadamard group; XT: 16-bit input type; SIGNED: d given (else d = 1);
 // Q8: 8-bit codes in [-127, 127], one per byte (the W4A8 activations), else
-// 4-bit codes in [-7, 7], two per byte.
-template <int G, int XT, bool SIGNED, bool Q8>
+// 4-bit codes in [-7, 7], two per byte; ASYM: OffQ codes in [0, 15] with a
+// scale sx [M][K/128] and zero point zx [M][K/128] per group (G = 128).
+template <int G, int XT, bool SIGNED, bool Q8, bool ASYM = false>
 __global__ void __launch_bounds__(rq::THREADS, 1)
     k_rotq(const __grid_constant__ CUtensorMap tmX, const int8_t* __restrict__ dsign, int M, int K,
            uint8_t* __restrict__ Xq, float* __restrict__ sx, float cg, int team_warps, int teams,
-           uint64_t limit_ns) {
+           uint64_t limit_ns, int32_t* __restrict__ zx) {
+    static_assert(!ASYM || (G == rq::UNIT && !Q8), "OffQ codes: 4-bit, one group of 128 per thread");
     constexpr int T = G > rq::UNIT ? G / rq::UNIT : 1;   // threads per group
     constexpr int HREG = G < rq::UNIT ? G : rq::UNIT;   // in-register stages: h < HREG
     static_assert(T <= 32, "a group spans at most one warp");
@@ -351,7 +369,9 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
 
         // ---- row absmax
         float am[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (T == 32) {
+        if constexpr (ASYM) {
+            // per-group ranges below; the team still meets once per row
+        } else if constexpr (T == 32) {
 #pragma unroll
             for (int ph = 0; ph < 2; ++ph)
 #pragma unroll
@@ -380,7 +400,45 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
 
         // ---- scale, round half to even, pack, store
         const float inv = amax == 0.f ? 0.f : __fdiv_rn(LEVELS, amax);   // amax == 0: every code is 0
-        if constexpr (Q8) {
+        if constexpr (ASYM) {
+            if (act) {
+                float lo4[4], hi4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) lo4[i] = hi4[i] = v[i].x;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    lo4[j & 3] = rq_min3(lo4[j & 3], v[j].x, v[j].y);
+                    hi4[j & 3] = rq_max3(hi4[j & 3], v[j].x, v[j].y);
+                }
+                const float lo = fminf(fminf(lo4[0], lo4[1]), fminf(lo4[2], lo4[3]));
+                const float hi = fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3]));
+                float dlt = __fsub_rn(hi, lo);
+                if (dlt == 0.f) dlt = lo != 0.f ? fabsf(lo) : 15.f;   // a constant group
+                const float ginv = __fdiv_rn(15.f, dlt);
+                const float zf = rintf(__fmul_rn(-lo, ginv));        // not clamped
+                uint4* dst = reinterpret_cast<uint4*>(Xq + static_cast<int64_t>(m) * (K / 2) + 64 * u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t words[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t wd = 0;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = v[16 * q + 4 * w + e];
+                            const float q0 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(x.x, ginv)), zf), 0.f), 15.f);
+                            const float q1 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(x.y, ginv)), zf), 0.f), 15.f);
+                            wd |= (static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << 4)) << (8 * e);
+                        }
+                        words[w] = wd;
+                    }
+                    dst[q] = make_uint4(words[0], words[1], words[2], words[3]);
+                }
+                const int64_t gi = static_cast<int64_t>(m) * (K / rq::UNIT) + u;
+                sx[gi] = __fmul_rn(__fdiv_rn(dlt, 15.f), cg);
+                zx[gi] = static_cast<int32_t>(zf);
+            }
+        } else if constexpr (Q8) {
             // the low byte of fl32(fl32(u * inv) + 1.5 * 2^23) is q in two's complement
             auto b4 = [&](float2 x0, float2 x1) {
                 const float2 r0 = rq_add2(make_float2(__fmul_rn(x0.x, inv), __fmul_rn(x0.y, inv)), mg);
@@ -444,7 +502,7 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
                 }
             }
         }
-        if (leader) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, LEVELS), cg);
+        if (!ASYM && leader) sx[m] = (amax == 0.f) ? 0.f : __fmul_rn(__fdiv_rn(amax, LEVELS), cg);
     }
     // no copy may still be landing when the CTA exits (immediate unless a
     // wait gave up): the rows issued but not consumed
@@ -499,13 +557,13 @@ bool rotq_supported(int64_t M, int64_t K, int group) {
     return rq_plan(M, K, group, 148, &p);
 }
 
-template <int G, int XT, bool SIGNED, bool Q8>
+template <int G, int XT, bool SIGNED, bool Q8, bool ASYM = false>
 static hq_status launch_rotq_t(const CUtensorMap& tm, const RqPlan& p, const int8_t* d, int M, int K, uint8_t* Xq,
-                               float* sx, float cg, uint64_t limit_ns, cudaStream_t st) {
-    auto kern = k_rotq<G, XT, SIGNED, Q8>;
+                               float* sx, float cg, uint64_t limit_ns, cudaStream_t st, int32_t* zx = nullptr) {
+    auto kern = k_rotq<G, XT, SIGNED, Q8, ASYM>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) != cudaSuccess)
         return HQ_ERR_CUDA;
-    kern<<<p.grid, rq::THREADS, p.smem, st>>>(tm, d, M, K, Xq, sx, cg, p.team_warps, p.teams, limit_ns);
+    kern<<<p.grid, rq::THREADS, p.smem, st>>>(tm, d, M, K, Xq, sx, cg, p.team_warps, p.teams, limit_ns, zx);
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -530,10 +588,11 @@ static hq_status launch_rotq_g(int group, const CUtensorMap& tm, const RqPlan& p
 // Caller has validated the arguments (16-bit type, power-of-two group in
 // [8, 4096] dividing K, 16-byte aligned X and Xq, ld_x * 2 a multiple of 16,
 // M > 0) and checked rotq_supported().  bits: 4 (packed nibbles, Xq [M][K/2])
-// or 8 (one code per byte, Xq [M][K]).
+// or 8 (one code per byte, Xq [M][K]); zx non-null: OffQ codes (bits 4,
+// group 128), sx and zx [M][K/128].
 hq_status launch_rotate_quant_stream(int xt, int group, const void* X, int64_t M, int64_t K, int64_t ldx,
                                      const int8_t* d, uint8_t* Xq, float* sx, cudaStream_t st,
-                                     uint64_t limit_ns, int bits) {
+                                     uint64_t limit_ns, int bits, int32_t* zx) {
     int dev = 0, nsm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return HQ_ERR_CUDA;
@@ -556,6 +615,14 @@ hq_status launch_rotate_quant_stream(int xt, int group, const void* X, int64_t M
     if (r != CUDA_SUCCESS) return HQ_ERR_CUDA;
     const float cg = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(group)));
     const int Mi = static_cast<int>(M), Ki = static_cast<int>(K);
+    if (zx) {
+        if (bits != 4 || group != rq::UNIT) return HQ_ERR_UNSUPPORTED;
+        if (xt == HQ_BF16)
+            return d ? launch_rotq_t<128, rq::XT_BF16, true, false, true>(tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st, zx)
+                     : launch_rotq_t<128, rq::XT_BF16, false, false, true>(tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st, zx);
+        return d ? launch_rotq_t<128, rq::XT_F16, true, false, true>(tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st, zx)
+                 : launch_rotq_t<128, rq::XT_F16, false, false, true>(tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st, zx);
+    }
     if (bits == 8) {
         if (xt == HQ_BF16)
             return d ? launch_rotq_g<rq::XT_BF16, true, true>(group, tm, p, d, Mi, Ki, Xq, sx, cg, limit_ns, st)
