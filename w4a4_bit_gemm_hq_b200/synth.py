@@ -144,3 +144,31 @@ def to_float32(a, dtype):
     if dtype == "bf16":
         return bf16_bits_to_f32(a)
     return np.asarray(a, np.float32)
+
+
+_T_CAL, _T_DIR = 6, 7
+
+
+def calibration_activations(wl: Workload, S, L, seed=0, n_dir=4, massive=400.0):
+    """Calibration batch for the offline steps: S sequences of L tokens, X
+    [S*L, K] in wl.xdtype, drawn as the workload's activations (its own
+    distribution recipe, from a separate stream) plus, in every sequence, one
+    token at a seeded position that carries a shared outlier direction.
+
+    The direction ``u`` (float32 [K], returned unnormalised) has n_dir seeded
+    channels of magnitude 1 with seeded signs and a dense N(0, 0.02) part, so
+    it is neither a single channel nor axis-aligned; the token gets
+    a_s * u with a_s uniform in [0.5, 1] * massive (seeded, random sign).
+    Returns (X, u, pos) with pos [S] the planted token of each sequence."""
+    rng = _rng(seed, _T_CAL)
+    base = activations(wl, seed=seed + 1000, M=S * L)
+    x = to_float32(base, wl.xdtype).copy().reshape(S, L, wl.K)
+    dr = _rng(seed, _T_DIR)
+    u = (dr.standard_normal(wl.K) * 0.02).astype(np.float32)
+    ch = dr.choice(wl.K, size=n_dir, replace=False)
+    u[ch] = np.where(dr.random(n_dir) < 0.5, -1.0, 1.0).astype(np.float32)
+    pos = rng.integers(0, L, size=S)
+    amp = (rng.uniform(0.5, 1.0, size=S) * massive * np.where(rng.random(S) < 0.5, -1.0, 1.0)).astype(np.float32)
+    for s in range(S):
+        x[s, pos[s], :] += amp[s] * u
+    return _cast(x.reshape(S * L, wl.K), wl.xdtype), u, pos
