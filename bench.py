@@ -462,6 +462,55 @@ class Shape:
             setattr(self, name, None)
 
 
+def calibration_record(R, S=32, L=128, iters=100):
+    """Offline calibration of the down-projection layer (K = 11008) on a
+    synthetic calibration batch of S sequences x L tokens: each kernel timed
+    alone with CUDA events (median of 5 after one warm-up), with its
+    algorithmic bytes where it streams HBM.  Offline work: reported, not part
+    of the step."""
+    import numpy as np
+
+    torch, hq, synth = R.torch, R.hq, R.synth
+    wl = synth.WORKLOADS["down"]
+    Xh, _, _ = synth.calibration_activations(wl, S, L)
+    X = R.to_dev(Xh, wl.xdtype)
+    W = R.to_dev(synth.weights(wl), wl.wdtype)
+    M, K, N = S * L, wl.K, wl.N
+    st = {}
+
+    def timed(name, fn, nbytes=None):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            out = fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = float(np.median(ts))
+        rec = {"us": ms * 1e3}
+        if nbytes is not None:
+            rec["bytes"] = nbytes
+            rec["GB/s"] = nbytes / (ms * 1e-3) / 1e9
+            rec["frac_hbm"] = rec["GB/s"] / R.peaks["hbm"]
+        st[name] = rec
+        return out
+
+    tok, T = timed("extreme_tokens", lambda: hq.hq_calib_extreme_tokens(X, S, L), 2 * M * K + 4 * S * K)
+    v, lam = timed("top1_pca (%d iterations, one CTA, T in L2)" % iters, lambda: hq.hq_calib_top1_pca(T, iters))
+    Xr = timed("householder (activations)", lambda: hq.hq_calib_householder(X, v), 2 * M * K + 4 * M * K)
+    Wr = timed("householder (weights)", lambda: hq.hq_calib_householder(W, v), 2 * N * K + 4 * N * K)
+    amax = timed("channel_absmax", lambda: hq.hq_calib_channel_absmax(Xr), 4 * M * K)
+    perm = timed("sorted_perm (K^2 comparisons)", lambda: hq.hq_calib_sorted_perm(amax))
+    timed("permute_channels (weights)", lambda: hq.hq_permute_channels(Wr, perm), 8 * N * K)
+    assert hq.hq_last_device_status() == 0
+    total = sum(r["us"] for r in st.values())
+    return {"workload": "down: calibration batch %d sequences x %d tokens, K=%d, W %dx%d" % (S, L, K, N, K),
+            "kernels": st, "total_us": total, "lambda": float(lam.item())}
+
+
 def int8_gemm_crosscheck(R):
     """cuBLASLt int8 GEMM (torch._int_mm) at 8192^3, best of 10: a cross-check
     of the int8 denominator, which is 2 x the measured bf16 burst peak."""
@@ -588,6 +637,7 @@ def main():
     # ---- every other shape of the suite
     workloads = [head]
     serq = []
+    calib = None
     if not args.headline_only:
         base, prev = None, None
         for name, M in SUITE:
@@ -619,6 +669,8 @@ def main():
             del S0
             torch.cuda.empty_cache()
         workloads.sort(key=lambda w: [n for n, _ in SUITE].index(w["workload"]) * 100000 + w["M"])
+        calib = calibration_record(R)
+        torch.cuda.empty_cache()
 
     targets = {}
     for name, M in TARGET_SHAPES:
@@ -663,6 +715,7 @@ def main():
         "workloads": workloads,
         "serq_overhead": serq,
         "activation_variants": variants,
+        "calibration": calib,
         "peaks": {"hbm_GBs": R.peaks["hbm"], "bf16_TFs_burst": R.peaks["bf16"], "bf16_TFs_sustained": R.peaks["bf16_sus"],
                   "int8_TOPs_denominator": R.int8_peak, "source": R.peaks["src"],
                   "int8_cublaslt_8192_TOPs_live": int8_gemm_crosscheck(R)},

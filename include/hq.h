@@ -357,6 +357,117 @@ hq_status hq_last_device_status(void* stream);
  */
 hq_status hq_debug_wait_probe(uint64_t limit_ns, void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Offline calibration (once per layer, before the online path; the results
+ * are folded into the weights).  Sources: "OffQ: Taming Structured Outliers
+ * in LLM Quantization by Offsetting", Methodology 1 (Top-1 PCA over the
+ * token of largest L-infinity norm of each calibration sequence), Methodology
+ * 3 and the ablation on sorted grouping (groups of 128 channels); "SERQ:
+ * Saliency-Aware Low-Rank Error Reconstruction for LLM Quantization",
+ * technical summary section 1 (static per-channel flattening folded into the
+ * weights) and section 3 (offline channel permutation of the weights).
+ * Element types of X below: HQ_F16, HQ_BF16 or HQ_F32; row stride ld_x in
+ * elements (>= K).  No alignment requirement.
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * hq_calib_extreme_tokens -- for each calibration sequence s (rows
+ * s*L .. s*L+L-1 of X), the token of largest max_k |x[k]| (ties to the earlier
+ * token; NaN entries are ignored by the maximum): its index in the sequence,
+ * tok[s], and its values widened to fp32, T[s][0..K).
+ *  X    device, [S*L][ld_x] calibration activations
+ *  tok  device, [S] int32 (output)
+ *  T    device, [S][K] fp32 (output), contiguous
+ * Errors: HQ_ERR_ARG (S < 0, L <= 0, K <= 0, ld_x < K, bad dtype, NULL with
+ * S > 0), HQ_ERR_UNSUPPORTED (a size above INT32_MAX).  S == 0 is a no-op.
+ */
+hq_status hq_calib_extreme_tokens(const void* X, hq_dtype xt, int64_t S, int64_t L, int64_t K,
+                                  int64_t ld_x, int32_t* tok, float* T, void* stream);
+
+/*
+ * hq_calib_top1_pca -- the principal eigenvector v of the (uncentred)
+ * covariance C = T^T T / S of the S extreme tokens, by `iters` power
+ * iterations (v <- C v / |C v|, C never formed) started from the token of
+ * largest L2 norm, in fp32 with every sum in a fixed order (the result is
+ * deterministic).  v is returned with unit length and its component of
+ * largest magnitude positive; lambda[0] = |C v| of the last iteration (the
+ * eigenvalue estimate; 0 for iters == 0).  All-zero tokens give v = e0,
+ * lambda 0.  Convergence goes as (lambda2 / lambda1)^iters: the caller picks
+ * iters.
+ *  T       device, [S][K] fp32 (from hq_calib_extreme_tokens)
+ *  v       device, [K] fp32 (output);  lambda  device, [1] fp32 (output)
+ * Runs as one CTA with v and T v in shared memory: S + K <=
+ * hq_calib_pca_max_elems() (HQ_ERR_UNSUPPORTED otherwise).
+ * Errors: HQ_ERR_ARG (S <= 0, K <= 0, iters < 0, NULL), HQ_ERR_UNSUPPORTED.
+ */
+size_t hq_calib_pca_max_elems(void);
+hq_status hq_calib_top1_pca(const float* T, int64_t S, int64_t K, int32_t iters, float* v, float* lambda,
+                            void* stream);
+
+/*
+ * hq_calib_householder -- Y = X Q with the reflection Q = I - 2 w w^T / (w^T w),
+ * w = v' - e0, where v' = -v if v[0] > 0 else v: Q is symmetric and
+ * orthogonal and maps v' to e0, so the direction of v (the outlier
+ * direction) lands in channel 0.  Apply it to the activations and to the
+ * weight rows alike (X Q (W Q)^T = X W^T).  fp32 arithmetic: per row
+ * c = fl(2 / w^T w) * (x . w), y = x - c w.
+ *  v  device, [K] fp32 of unit length;  Y  device, [M][K] fp32 (output)
+ * Errors: HQ_ERR_ARG (M < 0, K <= 0, ld_x < K, bad dtype, NULL with M > 0),
+ * HQ_ERR_UNSUPPORTED (K > 58080, M above INT32_MAX).  M == 0 is a no-op.
+ */
+hq_status hq_calib_householder(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                               const float* v, float* Y, void* stream);
+
+/*
+ * hq_calib_channel_absmax -- amax[k] = max over rows m of |X[m][k]| (exact;
+ * NaN entries are ignored).  amax is overwritten (cleared on the stream
+ * first); M == 0 gives zeros.
+ *  amax  device, [K] fp32 (output)
+ * Errors: HQ_ERR_ARG (M < 0, K <= 0, ld_x < K, bad dtype, NULL),
+ * HQ_ERR_UNSUPPORTED (a size above INT32_MAX), HQ_ERR_CUDA.
+ */
+hq_status hq_calib_channel_absmax(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                                  float* amax, void* stream);
+
+/*
+ * hq_calib_sorted_perm -- sorted grouping: perm[j] = the channel at position j
+ * in the order of decreasing stat (ties to the lower channel index; NaN sorts
+ * as -infinity).  Consecutive runs of `group` positions form the groups, so
+ * each group's first channel is its largest, the channel whose outlier the
+ * all-ones first row of H turns into the group's offset.
+ *  stat  device, [K] fp32;  perm  device, [K] int32 (output), a permutation
+ * Errors: HQ_ERR_ARG (K <= 0, NULL), HQ_ERR_UNSUPPORTED (K above INT32_MAX).
+ */
+hq_status hq_calib_sorted_perm(const float* stat, int64_t K, int32_t* perm, void* stream);
+
+/*
+ * hq_calib_flatten_scales -- static flattening: s[k] = xmax[k]^alpha /
+ * wmax[k]^(1-alpha) (fp32 powf and an IEEE divide); 1 where xmax[k] or
+ * wmax[k] is not positive.  Divide the activation channels by s and multiply
+ * the weight columns by s (hq_permute_channels ops 1 and 2).
+ *  xmax, wmax  device, [K] fp32 (per-channel max |x|, max |w|);  s  device, [K]
+ * Errors: HQ_ERR_ARG (K <= 0, NULL, alpha outside [0, 1]), HQ_ERR_UNSUPPORTED.
+ */
+hq_status hq_calib_flatten_scales(const float* xmax, const float* wmax, int64_t K, float alpha, float* s,
+                                  void* stream);
+
+/*
+ * hq_permute_channels -- Y[m][j] = X[m][c] with c = perm[j] (c = j when perm
+ * is NULL), op 0: as is, op 1: fl32(x / s[c]), op 2: fl32(x * s[c]); x widened
+ * to fp32 first.  The offline permutation (and flattening) of weight columns
+ * and, for calibration and tests, of activation rows.  A perm entry outside
+ * [0, K) writes 0 and records HQ_ERR_ARG in the device status word
+ * (hq_last_device_status).
+ *  perm  device, [K] int32 or NULL;  s  device, [K] fp32 (ops 1, 2)
+ *  Y     device, [M][K] fp32 (output), contiguous
+ * Errors: HQ_ERR_ARG (M < 0, K <= 0, ld_x < K, op outside 0..2, NULL X or Y
+ * with M > 0, NULL s with op != 0), HQ_ERR_UNSUPPORTED.  M == 0 is a no-op.
+ */
+hq_status hq_permute_channels(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                              const int32_t* perm, const float* s, int32_t op, float* Y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

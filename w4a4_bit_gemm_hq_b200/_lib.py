@@ -54,6 +54,14 @@ SIGNATURES = {
                      ct.c_size_t, _P], _ST),
     "hq_debug_accum8": ([_P, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32, _P, ct.c_size_t, _P],
                         _ST),
+    "hq_calib_extreme_tokens": ([_P, ct.c_int, _I64, _I64, _I64, _I64, _P, _P, _P], _ST),
+    "hq_calib_pca_max_elems": ([], ct.c_size_t),
+    "hq_calib_top1_pca": ([_P, _I64, _I64, _I32, _P, _P, _P], _ST),
+    "hq_calib_householder": ([_P, ct.c_int, _I64, _I64, _I64, _P, _P, _P], _ST),
+    "hq_calib_channel_absmax": ([_P, ct.c_int, _I64, _I64, _I64, _P, _P], _ST),
+    "hq_calib_sorted_perm": ([_P, _I64, _P, _P], _ST),
+    "hq_calib_flatten_scales": ([_P, _P, _I64, ct.c_float, _P, _P], _ST),
+    "hq_permute_channels": ([_P, ct.c_int, _I64, _I64, _I64, _P, _P, _I32, _P, _P], _ST),
     "hq_last_device_status": ([_P], _ST),
     "hq_debug_wait_probe": ([ct.c_uint64, _P], _ST),
 }

@@ -1,0 +1,401 @@
+// calib.cu -- offline calibration on the GPU: the steps that decide, once per
+// layer, how channels are rotated, ordered and scaled before the online path
+// (rotate/quant + W4A4 GEMM) runs.  Nothing here is on the per-token path;
+// the results are folded into the weights.
+//
+// Sources:
+//  * "OffQ: Taming Structured Outliers in LLM Quantization by Offsetting",
+//    Methodology 1 (Top-1 PCA: keep only the token of largest L-infinity norm
+//    of each calibration sequence, take the principal eigenvector of the
+//    covariance of those tokens, rotate so the outlier energy lands in the
+//    first channel), Methodology 3 and the ablation in the contributions
+//    (channels partitioned into groups of 128, sorted grouping);
+//  * "SERQ: Saliency-Aware Low-Rank Error Reconstruction for LLM
+//    Quantization", technical summary section 1 (static per-channel flattening
+//    in the manner of SmoothQuant, folded into the adjacent weights) and
+//    section 3 (the channel permutation applied to the weights offline, the
+//    activations arriving permuted by the previous layer).
+//
+// Kernels (all SIMT: none of this is a dense contraction worth the tensor
+// cores, and all of it runs once per layer):
+//  k_extreme      one CTA per calibration sequence: max |x| of every token
+//                 (exact), the arg max (ties to the earlier token), and the
+//                 chosen token widened to fp32.
+//  k_top1_pca     one CTA, power iteration on C = T^T T / S without forming C
+//                 (y = T v, z = T^T y / S, v = z / |z|), v and y in shared
+//                 memory, every sum in a fixed order (deterministic).
+//  k_householder  one warp per row: Y = X Q with Q = I - 2 w w^T / (w^T w),
+//                 w = v' - e0, v' = +-v with v'[0] <= 0, so Q v' = e0.
+//  k_col_absmax   column max |x| with integer atomics on the (non-negative)
+//                 float bit patterns: exact, order independent.
+//  k_rank         sorted grouping: position of every channel in the order of
+//                 decreasing statistic (ties to the lower index) by counting,
+//                 perm[position] = channel.
+//  k_flatten      s[k] = xmax[k]^alpha / wmax[k]^(1 - alpha).
+//  k_permute      Y[m][j] = X[m][perm[j]] (divided or multiplied by s[perm[j]]).
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "hq_device.cuh"
+
+namespace hq {
+
+namespace cb {
+constexpr int THREADS = 256;
+constexpr int PCA_THREADS = 1024;
+constexpr int SMEM_MAX = 227 * 1024;
+}  // namespace cb
+
+__device__ __forceinline__ float cb_load(const void* X, int xt, int64_t i) {
+    if (xt == HQ_F16) return __half2float(reinterpret_cast<const __half*>(X)[i]);
+    if (xt == HQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(X)[i]);
+    return reinterpret_cast<const float*>(X)[i];
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// Sum over the CTA of one value per thread, in a fixed order; every thread
+// gets the result.  red: shared, >= 32 floats.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    v = warp_sum(v);
+    __syncthreads();   // red may still be read by a previous call
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = lane < nw ? red[lane] : 0.f;
+    return warp_sum(t);
+}
+
+// ---------------------------------------------------------------- k_extreme
+__global__ void __launch_bounds__(cb::THREADS) k_extreme(const void* __restrict__ X, int xt, int L, int K,
+                                                        int64_t ldx, int32_t* __restrict__ tok,
+                                                        float* __restrict__ T) {
+    __shared__ float bv[cb::THREADS / 32];
+    __shared__ int bi[cb::THREADS / 32];
+    const int s = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int64_t row0 = static_cast<int64_t>(s) * L;
+    // each warp scans tokens warp, warp + nw, ... in increasing order: a later
+    // token replaces the warp's best only when strictly larger
+    float best = -1.f;
+    int besti = 0;
+    for (int t = warp; t < L; t += nw) {
+        const int64_t base = (row0 + t) * ldx;
+        float m = 0.f;
+        for (int k = lane; k < K; k += 32) m = fmaxf(m, fabsf(cb_load(X, xt, base + k)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (m > best) {
+            best = m;
+            besti = t;
+        }
+    }
+    if (lane == 0) {
+        bv[warp] = best;
+        bi[warp] = besti;
+    }
+    __syncthreads();
+    float b = bv[0];
+    int bidx = bi[0];
+    for (int w = 1; w < nw; ++w)
+        if (bv[w] > b || (bv[w] == b && bi[w] < bidx)) {
+            b = bv[w];
+            bidx = bi[w];
+        }
+    if (threadIdx.x == 0) tok[s] = bidx;
+    const int64_t src = (row0 + bidx) * ldx;
+    for (int k = threadIdx.x; k < K; k += blockDim.x)
+        T[static_cast<int64_t>(s) * K + k] = cb_load(X, xt, src + k);
+}
+
+// ---------------------------------------------------------------- k_top1_pca
+// Shared memory: v [K] | y [S] | red [32].
+__global__ void __launch_bounds__(cb::PCA_THREADS, 1)
+    k_top1_pca(const float* __restrict__ T, int S, int K, int iters, float* __restrict__ vout,
+               float* __restrict__ lam) {
+    extern __shared__ float sm[];
+    float* v = sm;
+    float* y = sm + K;
+    float* red = y + S;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const float invS = __fdiv_rn(1.0f, static_cast<float>(S));
+
+    // start: the calibration token of largest L2 norm (ties to the earlier one)
+    for (int s = warp; s < S; s += nw) {
+        float a = 0.f;
+        for (int k = lane; k < K; k += 32) {
+            const float t = T[static_cast<int64_t>(s) * K + k];
+            a = __fmaf_rn(t, t, a);
+        }
+        a = warp_sum(a);
+        if (lane == 0) y[s] = a;
+    }
+    __syncthreads();
+    int s0 = 0;
+    for (int s = 1; s < S; ++s)
+        if (y[s] > y[s0]) s0 = s;
+    const float n0 = y[s0];
+    __syncthreads();
+    float norm = 0.f;   // |C v| of the last iteration (0 before the first)
+    bool dead = !(n0 > 0.f);
+    if (!dead) {
+        const float inv = __fdiv_rn(1.0f, sqrtf(n0));
+        for (int k = threadIdx.x; k < K; k += blockDim.x) v[k] = __fmul_rn(T[static_cast<int64_t>(s0) * K + k], inv);
+        __syncthreads();
+        for (int it = 0; it < iters; ++it) {
+            // y = T v
+            for (int s = warp; s < S; s += nw) {
+                float a = 0.f;
+                for (int k = lane; k < K; k += 32) a = __fmaf_rn(T[static_cast<int64_t>(s) * K + k], v[k], a);
+                a = warp_sum(a);
+                if (lane == 0) y[s] = a;
+            }
+            __syncthreads();
+            // z = T^T y / S (into v: every y has been formed), |z|
+            float sq = 0.f;
+            for (int k = threadIdx.x; k < K; k += blockDim.x) {
+                float z = 0.f;
+                for (int s = 0; s < S; ++s) z = __fmaf_rn(T[static_cast<int64_t>(s) * K + k], y[s], z);
+                z = __fmul_rn(z, invS);
+                v[k] = z;
+                sq = __fmaf_rn(z, z, sq);
+            }
+            norm = sqrtf(block_sum(sq, red));
+            if (norm == 0.f) {
+                dead = true;
+                break;
+            }
+            const float inv = __fdiv_rn(1.0f, norm);
+            for (int k = threadIdx.x; k < K; k += blockDim.x) v[k] = __fmul_rn(v[k], inv);
+            __syncthreads();
+        }
+    }
+    if (dead) {
+        // no direction (all-zero tokens, or T v = 0): e0
+        __syncthreads();
+        for (int k = threadIdx.x; k < K; k += blockDim.x) v[k] = k == 0 ? 1.f : 0.f;
+        norm = 0.f;
+    }
+    __syncthreads();
+    // sign: the component of largest magnitude is positive (ties to the lower index)
+    if (threadIdx.x == 0) {
+        int kb = 0;
+        for (int k = 1; k < K; ++k)
+            if (fabsf(v[k]) > fabsf(v[kb])) kb = k;
+        red[0] = v[kb] < 0.f ? -1.f : 1.f;
+        *lam = norm;
+    }
+    __syncthreads();
+    const float sg = red[0];
+    for (int k = threadIdx.x; k < K; k += blockDim.x) vout[k] = __fmul_rn(v[k], sg);
+}
+
+// ---------------------------------------------------------------- k_householder
+// Shared memory: w [K] | red [32]
+__global__ void __launch_bounds__(cb::THREADS) k_householder(const void* __restrict__ X, int xt, int M, int K,
+                                                            int64_t ldx, const float* __restrict__ v,
+                                                            float* __restrict__ Y) {
+    extern __shared__ float sm[];
+    float* w = sm;
+    float* red = sm + K;
+    const float sg = v[0] > 0.f ? -1.f : 1.f;   // v' = sg v has v'[0] <= 0
+    float sq = 0.f;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const float e = __fmul_rn(sg, v[k]);
+        const float wk = k == 0 ? __fsub_rn(e, 1.0f) : e;
+        w[k] = wk;
+        sq = __fmaf_rn(wk, wk, sq);
+    }
+    const float ww = block_sum(sq, red);   // >= 1 for a unit v (|w0| >= 1)
+    const float two_over = __fdiv_rn(2.0f, ww);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int m = blockIdx.x * nw + warp; m < M; m += gridDim.x * nw) {
+        const int64_t base = static_cast<int64_t>(m) * ldx;
+        float d = 0.f;
+        for (int k = lane; k < K; k += 32) d = __fmaf_rn(cb_load(X, xt, base + k), w[k], d);
+        d = warp_sum(d);
+        const float c = __fmul_rn(two_over, d);
+        float* yr = Y + static_cast<int64_t>(m) * K;
+        for (int k = lane; k < K; k += 32) yr[k] = __fsub_rn(cb_load(X, xt, base + k), __fmul_rn(c, w[k]));
+    }
+}
+
+// ---------------------------------------------------------------- k_col_absmax
+__global__ void __launch_bounds__(cb::THREADS) k_col_absmax(const void* __restrict__ X, int xt, int M, int K,
+                                                           int64_t ldx, int rows_per, unsigned int* __restrict__ out) {
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= K) return;
+    const int m0 = blockIdx.y * rows_per;
+    const int m1 = min(M, m0 + rows_per);
+    float m = 0.f;
+    for (int r = m0; r < m1; ++r) m = fmaxf(m, fabsf(cb_load(X, xt, static_cast<int64_t>(r) * ldx + k)));
+    // fmaxf skips NaN, so m is a non-negative number: its bit pattern orders as its value
+    atomicMax(out + k, __float_as_uint(m));
+}
+
+// ---------------------------------------------------------------- k_rank
+// NaN ranks as -inf.
+__device__ __forceinline__ float cb_key(float x) { return x != x ? -INFINITY : x; }
+
+__global__ void __launch_bounds__(cb::THREADS) k_rank(const float* __restrict__ stat, int K, int32_t* __restrict__ perm) {
+    __shared__ float tile[cb::THREADS];
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const float si = i < K ? cb_key(stat[i]) : 0.f;
+    int rank = 0;
+    for (int j0 = 0; j0 < K; j0 += cb::THREADS) {
+        __syncthreads();
+        const int j = j0 + threadIdx.x;
+        tile[threadIdx.x] = j < K ? cb_key(stat[j]) : 0.f;
+        __syncthreads();
+        const int n = min(cb::THREADS, K - j0);
+        for (int t = 0; t < n; ++t) {
+            const float sj = tile[t];
+            rank += (sj > si || (sj == si && j0 + t < i)) ? 1 : 0;
+        }
+    }
+    if (i < K) perm[rank] = i;
+}
+
+// ---------------------------------------------------------------- k_flatten
+__global__ void k_flatten(const float* __restrict__ xmax, const float* __restrict__ wmax, int K, float alpha,
+                          float* __restrict__ s) {
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= K) return;
+    const float xm = xmax[k], wm = wmax[k];
+    // a channel with no activation or no weight range keeps the scale 1
+    s[k] = (xm > 0.f && wm > 0.f) ? __fdiv_rn(powf(xm, alpha), powf(wm, 1.0f - alpha)) : 1.0f;
+}
+
+// ---------------------------------------------------------------- k_permute
+// op: 0 copy, 1 divide by s, 2 multiply by s.  An index outside [0, K) records
+// HQ_ERR_ARG in the device status word and writes 0.
+__global__ void __launch_bounds__(cb::THREADS) k_permute(const void* __restrict__ X, int xt, int M, int K,
+                                                        int64_t ldx, const int32_t* __restrict__ perm,
+                                                        const float* __restrict__ s, int op, float* __restrict__ Y) {
+    const int64_t total = static_cast<int64_t>(M) * K;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = i / K;
+        const int j = static_cast<int>(i - m * K);
+        const int c = perm ? perm[j] : j;
+        float y = 0.f;
+        if (c < 0 || c >= K) {
+            record_status(HQ_ERR_ARG);
+        } else {
+            y = cb_load(X, xt, m * ldx + c);
+            if (op == 1) y = __fdiv_rn(y, s[c]);
+            else if (op == 2) y = __fmul_rn(y, s[c]);
+        }
+        Y[i] = y;
+    }
+}
+
+static int cb_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+static bool cb_dtype_ok(hq_dtype t) { return t == HQ_F16 || t == HQ_BF16 || t == HQ_F32; }
+static hq_status cb_launched() { return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" hq_status hq_calib_extreme_tokens(const void* X, hq_dtype xt, int64_t S, int64_t L, int64_t K,
+                                             int64_t ld_x, int32_t* tok, float* T, void* stream) {
+    if (!cb_dtype_ok(xt) || S < 0 || L <= 0 || K <= 0 || ld_x < K) return HQ_ERR_ARG;
+    if (S > INT32_MAX || L > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    if (S == 0) return HQ_OK;
+    if (!X || !tok || !T) return HQ_ERR_ARG;
+    k_extreme<<<static_cast<unsigned>(S), cb::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+        X, xt, static_cast<int>(L), static_cast<int>(K), ld_x, tok, T);
+    return cb_launched();
+}
+
+extern "C" size_t hq_calib_pca_max_elems(void) { return (cb::SMEM_MAX - 32 * 4) / 4; }
+
+extern "C" hq_status hq_calib_top1_pca(const float* T, int64_t S, int64_t K, int32_t iters, float* v, float* lambda,
+                                       void* stream) {
+    if (S <= 0 || K <= 0 || iters < 0 || !T || !v || !lambda) return HQ_ERR_ARG;
+    if (static_cast<uint64_t>(S) + static_cast<uint64_t>(K) > hq_calib_pca_max_elems()) return HQ_ERR_UNSUPPORTED;
+    const int smem = static_cast<int>((S + K + 32) * 4);
+    if (cudaFuncSetAttribute(k_top1_pca, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return HQ_ERR_CUDA;
+    k_top1_pca<<<1, cb::PCA_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+        T, static_cast<int>(S), static_cast<int>(K), iters, v, lambda);
+    return cb_launched();
+}
+
+extern "C" hq_status hq_calib_householder(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                                          const float* v, float* Y, void* stream) {
+    if (!cb_dtype_ok(xt) || M < 0 || K <= 0 || ld_x < K) return HQ_ERR_ARG;
+    if (M > INT32_MAX || K + 32 > (cb::SMEM_MAX / 4)) return HQ_ERR_UNSUPPORTED;
+    if (M == 0) return HQ_OK;
+    if (!X || !v || !Y) return HQ_ERR_ARG;
+    const int smem = static_cast<int>((K + 32) * 4);
+    if (cudaFuncSetAttribute(k_householder, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return HQ_ERR_CUDA;
+    const int64_t want = (M + cb::THREADS / 32 - 1) / (cb::THREADS / 32);
+    const int grid = static_cast<int>(want < 4 * cb_sm_count() ? want : 4 * cb_sm_count());
+    k_householder<<<grid, cb::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+        X, xt, static_cast<int>(M), static_cast<int>(K), ld_x, v, Y);
+    return cb_launched();
+}
+
+extern "C" hq_status hq_calib_channel_absmax(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                                             float* amax, void* stream) {
+    if (!cb_dtype_ok(xt) || M < 0 || K <= 0 || ld_x < K || !amax) return HQ_ERR_ARG;
+    if (M > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    if (M > 0 && !X) return HQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax, 0, static_cast<size_t>(K) * sizeof(float), st) != cudaSuccess) return HQ_ERR_CUDA;
+    if (M == 0) return HQ_OK;
+    const int gx = static_cast<int>((K + cb::THREADS - 1) / cb::THREADS);
+    // about four CTAs per SM in all, each over a contiguous run of rows
+    int gy = (4 * cb_sm_count() + gx - 1) / gx;
+    if (gy > M) gy = static_cast<int>(M);
+    const int rows_per = static_cast<int>((M + gy - 1) / gy);
+    gy = static_cast<int>((M + rows_per - 1) / rows_per);
+    k_col_absmax<<<dim3(gx, gy), cb::THREADS, 0, st>>>(X, xt, static_cast<int>(M), static_cast<int>(K), ld_x,
+                                                       rows_per, reinterpret_cast<unsigned int*>(amax));
+    return cb_launched();
+}
+
+extern "C" hq_status hq_calib_sorted_perm(const float* stat, int64_t K, int32_t* perm, void* stream) {
+    if (K <= 0 || !stat || !perm) return HQ_ERR_ARG;
+    if (K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    k_rank<<<static_cast<unsigned>((K + cb::THREADS - 1) / cb::THREADS), cb::THREADS, 0,
+             static_cast<cudaStream_t>(stream)>>>(stat, static_cast<int>(K), perm);
+    return cb_launched();
+}
+
+extern "C" hq_status hq_calib_flatten_scales(const float* xmax, const float* wmax, int64_t K, float alpha, float* s,
+                                             void* stream) {
+    if (K <= 0 || !xmax || !wmax || !s || !(alpha >= 0.f && alpha <= 1.f)) return HQ_ERR_ARG;
+    if (K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    k_flatten<<<static_cast<unsigned>((K + cb::THREADS - 1) / cb::THREADS), cb::THREADS, 0,
+                static_cast<cudaStream_t>(stream)>>>(xmax, wmax, static_cast<int>(K), alpha, s);
+    return cb_launched();
+}
+
+extern "C" hq_status hq_permute_channels(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
+                                         const int32_t* perm, const float* s, int32_t op, float* Y, void* stream) {
+    if (!cb_dtype_ok(xt) || M < 0 || K <= 0 || ld_x < K || op < 0 || op > 2) return HQ_ERR_ARG;
+    if (M > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    if (M == 0) return HQ_OK;
+    if (!X || !Y || (op != 0 && !s)) return HQ_ERR_ARG;
+    const int64_t blocks = (M * K + cb::THREADS - 1) / cb::THREADS;
+    const int grid = static_cast<int>(blocks < 8 * cb_sm_count() ? blocks : 8 * cb_sm_count());
+    k_permute<<<grid, cb::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+        X, xt, static_cast<int>(M), static_cast<int>(K), ld_x, perm, s, op, Y);
+    return cb_launched();
+}

@@ -21,7 +21,9 @@ __all__ = [
     "serq_prepare", "w4a4_linear", "hq_linear_workspace_size", "hq_debug_accum", "hq_last_device_status",
     "hq_debug_wait_probe", "hq_packed_weight_bytes", "wq_tile", "wq_untile", "W4A4Linear",
     "hq_rotate_quant8", "w4a8_linear", "hq_debug_accum8", "hq_rotate_quant_asym", "w4a4_linear_asym",
-    "hq_debug_accum_asym",
+    "hq_debug_accum_asym", "hq_calib_extreme_tokens", "hq_calib_top1_pca", "hq_calib_householder",
+    "hq_calib_channel_absmax", "hq_calib_sorted_perm", "hq_calib_flatten_scales", "hq_permute_channels",
+    "calibrate_rotation_and_grouping",
 ]
 
 
@@ -243,6 +245,92 @@ def hq_debug_accum(Xq, Wq, zw, group, A, sal_idx, N, decode=False, workspace=Non
                              ptr(sal_idx) if r else None, r, ptr(acc), ptr(acc_c), 1 if decode else 0,
                              ptr(workspace), ws_bytes, stream_handle()), "hq_debug_accum")
     return acc, acc_c
+
+
+# ------------------------------------------------------------ offline calibration
+# OffQ, Methodology 1 (Top-1 PCA) and 3 (sorted grouping); SERQ sections 1
+# (static flattening) and 3 (offline permutation).
+
+def hq_calib_extreme_tokens(X, S, L, tok=None, T=None):
+    """(tok int32 [S], T float32 [S, K]): per calibration sequence (L rows of
+    X each) the token of largest max |x| and its values."""
+    K = X.shape[1]
+    assert X.shape[0] == S * L
+    tok = torch.empty((S,), dtype=torch.int32, device=X.device) if tok is None else tok
+    T = torch.empty((S, K), dtype=torch.float32, device=X.device) if T is None else T
+    check(lib.hq_calib_extreme_tokens(ptr(X), dtype_code(X.dtype), S, L, K, X.stride(0), ptr(tok), ptr(T),
+                                      stream_handle()), "hq_calib_extreme_tokens")
+    return tok, T
+
+
+def hq_calib_top1_pca(T, iters=100, v=None, lam=None):
+    """(v float32 [K] unit, lam float32 [1]): principal eigenvector of T^T T / S."""
+    S, K = T.shape
+    assert T.dtype == torch.float32 and T.is_contiguous()
+    v = torch.empty((K,), dtype=torch.float32, device=T.device) if v is None else v
+    lam = torch.empty((1,), dtype=torch.float32, device=T.device) if lam is None else lam
+    check(lib.hq_calib_top1_pca(ptr(T), S, K, iters, ptr(v), ptr(lam), stream_handle()), "hq_calib_top1_pca")
+    return v, lam
+
+
+def hq_calib_householder(X, v, Y=None):
+    """Y float32 [M, K] = X Q, Q the reflection that sends +-v to e0."""
+    M, K = X.shape
+    Y = torch.empty((M, K), dtype=torch.float32, device=X.device) if Y is None else Y
+    check(lib.hq_calib_householder(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), ptr(v), ptr(Y),
+                                   stream_handle()), "hq_calib_householder")
+    return Y
+
+
+def hq_calib_channel_absmax(X, amax=None):
+    """amax float32 [K] = max over rows of |X|."""
+    M, K = X.shape
+    amax = torch.empty((K,), dtype=torch.float32, device=X.device) if amax is None else amax
+    check(lib.hq_calib_channel_absmax(ptr(X), dtype_code(X.dtype), M, K, max(X.stride(0), K), ptr(amax),
+                                      stream_handle()), "hq_calib_channel_absmax")
+    return amax
+
+
+def hq_calib_sorted_perm(stat, perm=None):
+    """perm int32 [K]: channels in decreasing stat (ties to the lower index)."""
+    K = stat.shape[0]
+    perm = torch.empty((K,), dtype=torch.int32, device=stat.device) if perm is None else perm
+    check(lib.hq_calib_sorted_perm(ptr(stat), K, ptr(perm), stream_handle()), "hq_calib_sorted_perm")
+    return perm
+
+
+def hq_calib_flatten_scales(xmax, wmax, alpha=0.5, s=None):
+    """s float32 [K] = xmax^alpha / wmax^(1-alpha)."""
+    K = xmax.shape[0]
+    s = torch.empty((K,), dtype=torch.float32, device=xmax.device) if s is None else s
+    check(lib.hq_calib_flatten_scales(ptr(xmax), ptr(wmax), K, float(alpha), ptr(s), stream_handle()),
+          "hq_calib_flatten_scales")
+    return s
+
+
+def hq_permute_channels(X, perm=None, s=None, op=0, Y=None):
+    """Y float32 [M, K]: Y[:, j] = X[:, perm[j]] (op 1: / s, op 2: * s, taken at perm[j])."""
+    M, K = X.shape
+    Y = torch.empty((M, K), dtype=torch.float32, device=X.device) if Y is None else Y
+    check(lib.hq_permute_channels(ptr(X), dtype_code(X.dtype), M, K, max(X.stride(0), K),
+                                  None if perm is None else ptr(perm), None if s is None else ptr(s), op, ptr(Y),
+                                  stream_handle()), "hq_permute_channels")
+    return Y
+
+
+def calibrate_rotation_and_grouping(X_calib, S, L, W, iters=100):
+    """The offline OffQ calibration of one layer, every step on the GPU:
+    extreme tokens -> Top-1 PCA direction v -> Householder rotation of the
+    calibration activations and of the weight rows -> per-channel max |x| ->
+    sorted-grouping permutation.  Returns (v, perm, W_cal) with W_cal float32
+    [N, K] = (W Q)[:, perm]: activations that arrive as (X Q)[:, perm] give
+    the same product X W^T."""
+    _, T = hq_calib_extreme_tokens(X_calib, S, L)
+    v, _ = hq_calib_top1_pca(T, iters)
+    Xr = hq_calib_householder(X_calib, v)
+    perm = hq_calib_sorted_perm(hq_calib_channel_absmax(Xr))
+    W_cal = hq_permute_channels(hq_calib_householder(W, v), perm)
+    return v, perm, W_cal
 
 
 def hq_last_device_status():
