@@ -75,6 +75,8 @@ def parse():
                     help="headline workload (default: the down-projection)")
     ap.add_argument("--m", type=int, default=None, help="tokens per step of the headline (default: the workload's)")
     ap.add_argument("--headline-only", action="store_true", help="skip the other shapes (profiling runs)")
+    ap.add_argument("--calibration-only", action="store_true",
+                    help="time the offline calibration kernels of the down layer only (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -568,6 +570,10 @@ def main():
 
     dev = torch.device("cuda", local)
     R = Runner(torch, hq, synth, rank, dev)
+    if args.calibration_only:
+        if rank == 0:
+            print(json.dumps({"calibration": calibration_record(R)}), flush=True)
+        return
     steps = args.steps if args.steps is not None else DEFAULT_STEPS
     warm = max(args.warmup, 3)
 
