@@ -29,6 +29,10 @@ def _rows(M, K, g, seed, xdtype):
         x[2, 0] = 3.0                        # a constant group
     if M > 3:
         x[3, :g] = 0.125                     # a group whose rotation is one spike (|first| = g / 8)
+    if M > 4:
+        x[4] = 0.0                           # a tiny spread on a large offset: |u / step| >= 2^22
+        x[4, 0] = 1000.0
+        x[4, 5] = 2.0 ** -10
     return synth.f32_to_bf16_bits(x) if xdtype == "bf16" else x.astype(np.float16)
 
 

@@ -417,22 +417,54 @@ __global__ void __launch_bounds__(rq::THREADS, 1)
                 const float ginv = __fdiv_rn(15.f, dlt);
                 const float zf = rintf(__fmul_rn(-lo, ginv));        // not clamped
                 uint4* dst = reinterpret_cast<uint4*>(Xq + static_cast<int64_t>(m) * (K / 2) + 64 * u);
+                // every |fl32(u * ginv)| is at most fl32(max(|lo|, |hi|) * ginv) (rounding is
+                // monotone); below 2^22, adding 1.5 * 2^23 rounds it to an integer with ties
+                // to even (= rint), adding z is then exact, and the code sits in the low
+                // nibble of the sum's bits.  rint(fl32(u ginv)) + z >= rint(fl32(lo ginv)) + z
+                // = 0 (rint is odd), so only the upper clamp is needed.  Larger ratios
+                // (a tiny spread on a large offset) take the plain sequence.
+                if (__fmul_rn(fmaxf(fabsf(lo), fabsf(hi)), ginv) < 4194304.0f) {
+                    const float2 zz = make_float2(zf, zf);
+                    constexpr float TOP = 12582912.0f + 15.0f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t words[4];
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t words[4];
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        uint32_t wd = 0;
+                        for (int w = 0; w < 4; ++w) {
+                            uint32_t P[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 x = v[16 * q + 4 * w + e];
-                            const float q0 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(x.x, ginv)), zf), 0.f), 15.f);
-                            const float q1 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(x.y, ginv)), zf), 0.f), 15.f);
-                            wd |= (static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << 4)) << (8 * e);
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 x = v[16 * q + 4 * w + e];
+                                float2 r = rq_add2(make_float2(__fmul_rn(x.x, ginv), __fmul_rn(x.y, ginv)),
+                                                   make_float2(12582912.0f, 12582912.0f));
+                                r = rq_add2(r, zz);
+                                r.x = fminf(r.x, TOP);
+                                r.y = fminf(r.y, TOP);
+                                P[e] = (__float_as_uint(r.y) << 4) + __float_as_uint(r.x);   // byte e (low 16 bits)
+                            }
+                            const uint32_t q01 = (P[1] << 8) + P[0], q23 = (P[3] << 8) + P[2];
+                            words[w] = __byte_perm(q01, q23, 0x5410);
                         }
-                        words[w] = wd;
+                        dst[q] = make_uint4(words[0], words[1], words[2], words[3]);
                     }
-                    dst[q] = make_uint4(words[0], words[1], words[2], words[3]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t words[4];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            uint32_t wd = 0;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 x = v[16 * q + 4 * w + e];
+                                const float q0 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(x.x, ginv)), zf), 0.f), 15.f);
+                                const float q1 = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(x.y, ginv)), zf), 0.f), 15.f);
+                                wd |= (static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << 4)) << (8 * e);
+                            }
+                            words[w] = wd;
+                        }
+                        dst[q] = make_uint4(words[0], words[1], words[2], words[3]);
+                    }
                 }
                 const int64_t gi = static_cast<int64_t>(m) * (K / rq::UNIT) + u;
                 sx[gi] = __fmul_rn(__fdiv_rn(dlt, 15.f), cg);
