@@ -501,7 +501,7 @@ def calibration_record(R, S=32, L=128, iters=100):
         return out
 
     tok, T = timed("extreme_tokens", lambda: hq.hq_calib_extreme_tokens(X, S, L), 2 * M * K + 4 * S * K)
-    v, lam = timed("top1_pca (%d iterations, one CTA, T in L2)" % iters, lambda: hq.hq_calib_top1_pca(T, iters))
+    v, lam = timed("top1_pca (%d iterations, cluster of 8 CTAs, T in shared memory)" % iters, lambda: hq.hq_calib_top1_pca(T, iters))
     Xr = timed("householder (activations)", lambda: hq.hq_calib_householder(X, v), 2 * M * K + 4 * M * K)
     Wr = timed("householder (weights)", lambda: hq.hq_calib_householder(W, v), 2 * N * K + 4 * N * K)
     amax = timed("channel_absmax", lambda: hq.hq_calib_channel_absmax(Xr), 4 * M * K)

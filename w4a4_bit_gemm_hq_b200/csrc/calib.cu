@@ -45,6 +45,8 @@ namespace hq {
 namespace cb {
 constexpr int THREADS = 256;
 constexpr int PCA_THREADS = 1024;
+constexpr int CL = 8;               // CTAs of the cluster power iteration
+constexpr int PCL_THREADS = 512;
 constexpr int SMEM_MAX = 227 * 1024;
 }  // namespace cb
 
@@ -196,6 +198,147 @@ __global__ void __launch_bounds__(cb::PCA_THREADS, 1)
     for (int k = threadIdx.x; k < K; k += blockDim.x) vout[k] = __fmul_rn(v[k], sg);
 }
 
+// ---------------------------------------------------------------- k_top1_pca_cl
+// The same power iteration on a cluster of cb::CL CTAs when the S tokens fit in
+// their shared memory: CTA c holds columns [c Kc, c Kc + Kc) of T and of v, so
+// an iteration reads shared memory only.  y = T v is summed over the cluster
+// (each CTA reads every CTA's partial through distributed shared memory, in
+// rank order, so all CTAs hold the same y), z = T^T y is local, |z|^2 is summed
+// over the cluster the same way.  Partials are double-buffered by use count,
+// so one hardware cluster barrier per reduction suffices.
+// Shared memory: Ts [S][Kc] | v [Kc] | yp [2][S] | y [S] | red [32] | sc [2] | fin [2]
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t caddr) {
+    float r;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(r) : "r"(caddr) : "memory");
+    return r;
+}
+
+__global__ void __launch_bounds__(cb::PCL_THREADS, 1)
+    k_top1_pca_cl(const float* __restrict__ T, int S, int K, int Kc, int iters, float* __restrict__ vout,
+                  float* __restrict__ lam) {
+    extern __shared__ float sm[];
+    float* Ts = sm;
+    float* v = Ts + static_cast<int64_t>(S) * Kc;
+    float* yp = v + Kc;
+    float* y = yp + 2 * S;
+    float* red = y + S;
+    float* sc = red + 32;
+    float* fin = sc + 2;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int k0 = rank * Kc;
+    const int kn = K - k0 < Kc ? (K - k0 > 0 ? K - k0 : 0) : Kc;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const float invS = __fdiv_rn(1.0f, static_cast<float>(S));
+
+    for (int i = threadIdx.x; i < S * kn; i += blockDim.x) {
+        const int s = i / kn, j = i - s * kn;
+        Ts[s * Kc + j] = T[static_cast<int64_t>(s) * K + k0 + j];
+    }
+    __syncthreads();
+
+    int ny = 0, nsq = 0;   // uses of yp and of sc (buffer = count & 1)
+    // y[s] = sum over the cluster of the partials p[s] written by this CTA
+    auto cluster_vec = [&](auto partial) {
+        float* b = yp + (ny & 1) * S;
+        for (int s = warp; s < S; s += nw) {
+            const float a = warp_sum(partial(s));
+            if (lane == 0) b[s] = a;
+        }
+        ++ny;
+        cluster_sync();
+        const uint32_t base = smem_u32(b);
+        for (int s = threadIdx.x; s < S; s += blockDim.x) {
+            float a = 0.f;
+            for (int r = 0; r < cb::CL; ++r) a = __fadd_rn(a, ld_dsmem_f32(mapa_shared(base + 4u * s, r)));
+            y[s] = a;
+        }
+        __syncthreads();
+    };
+    auto cluster_scalar = [&](float part) {
+        const float t = block_sum(part, red);
+        float* b = sc + (nsq & 1);
+        if (threadIdx.x == 0) *b = t;
+        ++nsq;
+        cluster_sync();
+        float a = 0.f;
+        for (int r = 0; r < cb::CL; ++r) a = __fadd_rn(a, ld_dsmem_f32(mapa_shared(smem_u32(b), r)));
+        return a;
+    };
+
+    // start: the token of largest L2 norm (ties to the earlier one)
+    cluster_vec([&](int s) {
+        float a = 0.f;
+        for (int j = lane; j < kn; j += 32) a = __fmaf_rn(Ts[s * Kc + j], Ts[s * Kc + j], a);
+        return a;
+    });
+    int s0 = 0;
+    for (int s = 1; s < S; ++s)
+        if (y[s] > y[s0]) s0 = s;
+    const float n0 = y[s0];
+    float norm = 0.f;
+    bool dead = !(n0 > 0.f);
+    if (!dead) {
+        const float inv = __fdiv_rn(1.0f, sqrtf(n0));
+        for (int j = threadIdx.x; j < kn; j += blockDim.x) v[j] = __fmul_rn(Ts[s0 * Kc + j], inv);
+        __syncthreads();
+        for (int it = 0; it < iters; ++it) {
+            cluster_vec([&](int s) {
+                float a = 0.f;
+                for (int j = lane; j < kn; j += 32) a = __fmaf_rn(Ts[s * Kc + j], v[j], a);
+                return a;
+            });
+            float sq = 0.f;
+            for (int j = threadIdx.x; j < kn; j += blockDim.x) {
+                float z = 0.f;
+                for (int s = 0; s < S; ++s) z = __fmaf_rn(Ts[s * Kc + j], y[s], z);
+                z = __fmul_rn(z, invS);
+                v[j] = z;
+                sq = __fmaf_rn(z, z, sq);
+            }
+            norm = sqrtf(cluster_scalar(sq));
+            if (norm == 0.f) {
+                dead = true;
+                break;
+            }
+            const float inv = __fdiv_rn(1.0f, norm);
+            for (int j = threadIdx.x; j < kn; j += blockDim.x) v[j] = __fmul_rn(v[j], inv);
+            __syncthreads();
+        }
+    }
+    if (dead) {
+        __syncthreads();
+        for (int j = threadIdx.x; j < kn; j += blockDim.x) v[j] = (k0 + j == 0) ? 1.f : 0.f;
+        norm = 0.f;
+    }
+    __syncthreads();
+    // sign: the component of largest magnitude over the whole vector is positive
+    if (threadIdx.x == 0) {
+        int jb = 0;
+        for (int j = 1; j < kn; ++j)
+            if (fabsf(v[j]) > fabsf(v[jb])) jb = j;
+        fin[0] = kn > 0 ? fabsf(v[jb]) : -1.f;
+        fin[1] = kn > 0 ? (v[jb] < 0.f ? -1.f : 1.f) : 1.f;
+    }
+    cluster_sync();
+    if (threadIdx.x == 0) {
+        float best = -1.f, sg = 1.f;
+        for (int r = 0; r < cb::CL; ++r) {   // ranks in order: the lower index wins ties
+            const float a = ld_dsmem_f32(mapa_shared(smem_u32(fin), r));
+            if (a > best) {
+                best = a;
+                sg = ld_dsmem_f32(mapa_shared(smem_u32(fin + 1), r));
+            }
+        }
+        red[0] = sg;
+        if (rank == 0) *lam = norm;
+    }
+    __syncthreads();
+    const float sg = red[0];
+    for (int j = threadIdx.x; j < kn; j += blockDim.x) vout[k0 + j] = __fmul_rn(v[j], sg);
+    // no CTA leaves while another may still read its shared memory
+    cluster_sync();
+}
+
 // ---------------------------------------------------------------- k_householder
 // Shared memory: w [K] | red [32]
 __global__ void __launch_bounds__(cb::THREADS) k_householder(const void* __restrict__ X, int xt, int M, int K,
@@ -327,11 +470,35 @@ extern "C" hq_status hq_calib_top1_pca(const float* T, int64_t S, int64_t K, int
                                        void* stream) {
     if (S <= 0 || K <= 0 || iters < 0 || !T || !v || !lambda) return HQ_ERR_ARG;
     if (static_cast<uint64_t>(S) + static_cast<uint64_t>(K) > hq_calib_pca_max_elems()) return HQ_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the tokens fit in the shared memory of a cluster: every iteration runs from shared memory
+    const int64_t Kc = ((K + cb::CL - 1) / cb::CL + 3) / 4 * 4;
+    const int64_t cl_smem = (S * Kc + Kc + 3 * S + 32 + 4) * 4;
+    if (cl_smem <= cb::SMEM_MAX - 1024) {
+        const int sm = static_cast<int>(cl_smem);
+        if (cudaFuncSetAttribute(k_top1_pca_cl, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess)
+            return HQ_ERR_CUDA;
+        cudaLaunchConfig_t cfg{};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cb::CL;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(cb::CL, 1, 1);
+        cfg.blockDim = dim3(cb::PCL_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = sm;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, k_top1_pca_cl, T, static_cast<int>(S), static_cast<int>(K),
+                               static_cast<int>(Kc), static_cast<int>(iters), v, lambda) != cudaSuccess)
+            return HQ_ERR_CUDA;
+        return cb_launched();
+    }
     const int smem = static_cast<int>((S + K + 32) * 4);
     if (cudaFuncSetAttribute(k_top1_pca, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
-    k_top1_pca<<<1, cb::PCA_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
-        T, static_cast<int>(S), static_cast<int>(K), iters, v, lambda);
+    k_top1_pca<<<1, cb::PCA_THREADS, smem, st>>>(T, static_cast<int>(S), static_cast<int>(K), iters, v, lambda);
     return cb_launched();
 }
 
