@@ -620,21 +620,61 @@ def main():
         for i in range(P):
             Xh[i].copy_(S.X[i].cpu())
 
-        def e2e_step(i):
-            S.X[i].copy_(Xh[i], non_blocking=True)
-            S.layers[i](S.X[i], S.Y[i], S.Xq[i], S.sx[i])
-            Yh[i].copy_(S.Y[i], non_blocking=True)
+        # three streams: the copy in of step j waits only for the compute that last
+        # read its input buffer, the compute for its input and for the copy out
+        # that last read its output buffer, the copy out for its compute; so the
+        # host-to-device copies of later steps overlap the compute and the
+        # device-to-host copies of earlier ones (buffers reused round-robin)
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-        g_e2e = R.capture([lambda i=i: e2e_step(i) for i in range(P)])
-        g_e2e.replay()
-        est = max(R.time_graph(g_e2e, 1), 1e-3)
-        r = int(max(2, min(20000, 400.0 / est)))
+        def e2e_steps(nsteps):
+            cur = torch.cuda.current_stream()
+            for st_ in (s_in, s_cmp, s_out):
+                st_.wait_stream(cur)
+            ev_cmp, ev_out = [], []
+            for j in range(nsteps):
+                i = j % P
+                with torch.cuda.stream(s_in):
+                    if j >= P:
+                        s_in.wait_event(ev_cmp[j - P])
+                    S.X[i].copy_(Xh[i], non_blocking=True)
+                    e_in = torch.cuda.Event()
+                    e_in.record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(e_in)
+                    if j >= P:
+                        s_cmp.wait_event(ev_out[j - P])
+                    S.layers[i](S.X[i], S.Y[i], S.Xq[i], S.sx[i])
+                    ev_cmp.append(torch.cuda.Event())
+                    ev_cmp[-1].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_cmp[j])
+                    Yh[i].copy_(S.Y[i], non_blocking=True)
+                    ev_out.append(torch.cuda.Event())
+                    ev_out[-1].record(s_out)
+            for st_ in (s_in, s_cmp, s_out):
+                cur.wait_stream(st_)
+
+        def e2e_time(nsteps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record()
+            e2e_steps(nsteps)
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b)
+
+        e2e_steps(2 * P)
+        est = max(e2e_time(2 * P) / (2 * P), 1e-3)
+        r = int(max(4 * P, min(20000, 400.0 / est)))
         if pg is not None:
             pg.barrier()
-        e_ms = max_over_ranks(R.time_graph(g_e2e, r), pg, dev)
-        e2e = {"value": job_tops(k2_ops(M, N, K), r * P, world, e_ms), "unit": "TOPS",
-               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e_ms / (r * P)}
-        del g_e2e, Xh, Yh
+        e_ms = max_over_ranks(e2e_time(r), pg, dev)
+        e2e = {"value": job_tops(k2_ops(M, N, K), r, world, e_ms), "unit": "TOPS",
+               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e_ms / r,
+               "steps": r, "pipelined": "copy in, compute and copy out on three streams; step j's copy in "
+                                        "overlaps the compute and copy out of earlier steps"}
+        del Xh, Yh
     variants = [] if args.headline_only else S.variants(decode_like)
     S.free()
     del S
