@@ -167,11 +167,13 @@ def test_flatten_scales_within_ulps():
         assert (s[:8] == 1.0).all()
 
 
+# K = 1111: element-wise kernel; K = 1112 (a multiple of 8): rows staged in shared memory
+@pytest.mark.parametrize("K", [1111, 1112])
 @pytest.mark.parametrize("op", [0, 1, 2])
 @pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
-def test_permute_channels_bit_exact(op, dt):
+def test_permute_channels_bit_exact(op, dt, K):
     rng = np.random.default_rng(op + 3)
-    M, K = 333, 1111
+    M = 333
     Xf = rng.standard_normal((M, K)).astype(np.float32) * 3
     X = synth.f32_to_bf16_bits(Xf) if dt == "bf16" else (Xf.astype(np.float16) if dt == "f16" else Xf)
     Xw = synth.to_float32(X, dt) if dt != "f16" else X.astype(np.float32)

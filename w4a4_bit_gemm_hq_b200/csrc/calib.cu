@@ -45,6 +45,7 @@ namespace hq {
 namespace cb {
 constexpr int THREADS = 256;
 constexpr int PCA_THREADS = 1024;
+constexpr int EXT_THREADS = 1024;
 constexpr int CL = 8;               // CTAs of the cluster power iteration
 constexpr int PCL_THREADS = 512;
 constexpr int SMEM_MAX = 227 * 1024;
@@ -114,6 +115,87 @@ __global__ void __launch_bounds__(cb::THREADS) k_extreme(const void* __restrict_
     const int64_t src = (row0 + bidx) * ldx;
     for (int k = threadIdx.x; k < K; k += blockDim.x)
         T[static_cast<int64_t>(s) * K + k] = cb_load(X, xt, src + k);
+}
+
+// ---------------------------------------------------------------- 16-byte paths
+// Used when X is 16-byte aligned, its row stride a multiple of 16 bytes and K a
+// multiple of 8: element i (a multiple of 8) starts an aligned 16-byte (16-bit
+// types) or 32-byte (fp32) chunk of 8 values.
+__device__ __forceinline__ void cb_load8(const void* X, int xt, int64_t i, float (&f)[8]) {
+    if (xt == HQ_F32) {
+        const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(X) + i);
+        const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(X) + i + 4);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        return;
+    }
+    const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(X) + i);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        if (xt == HQ_BF16) {
+            f[2 * e] = __uint_as_float(u[e] << 16);
+            f[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+        } else {
+            const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&u[e]));
+            f[2 * e] = h.x;
+            f[2 * e + 1] = h.y;
+        }
+    }
+}
+
+// k_extreme with 1024 threads and four 16-byte chunks per lane in flight.
+__global__ void __launch_bounds__(cb::EXT_THREADS) k_extreme_v(const void* __restrict__ X, int xt, int L, int K,
+                                                              int64_t ldx, int32_t* __restrict__ tok,
+                                                              float* __restrict__ T) {
+    __shared__ float bv[cb::EXT_THREADS / 32];
+    __shared__ int bi[cb::EXT_THREADS / 32];
+    const int s = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int64_t row0 = static_cast<int64_t>(s) * L;
+    float best = -1.f;
+    int besti = 0;
+    for (int t = warp; t < L; t += nw) {
+        const int64_t base = (row0 + t) * ldx;
+        float m = 0.f;
+        for (int k0 = 8 * lane; k0 < K; k0 += 4 * 256) {
+            float f[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (k0 + 256 * u < K) cb_load8(X, xt, base + k0 + 256 * u, f[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (k0 + 256 * u < K)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[u][e]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (m > best) {
+            best = m;
+            besti = t;
+        }
+    }
+    if (lane == 0) {
+        bv[warp] = best;
+        bi[warp] = besti;
+    }
+    __syncthreads();
+    float b = bv[0];
+    int bidx = bi[0];
+    for (int w = 1; w < nw; ++w)
+        if (bv[w] > b || (bv[w] == b && bi[w] < bidx)) {
+            b = bv[w];
+            bidx = bi[w];
+        }
+    if (threadIdx.x == 0) tok[s] = bidx;
+    const int64_t src = (row0 + bidx) * ldx;
+    float* dst = T + static_cast<int64_t>(s) * K;
+    for (int k0 = 8 * threadIdx.x; k0 < K; k0 += 8 * blockDim.x) {
+        float f[8];
+        cb_load8(X, xt, src + k0, f);
+        *reinterpret_cast<float4*>(dst + k0) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(dst + k0 + 4) = make_float4(f[4], f[5], f[6], f[7]);
+    }
 }
 
 // ---------------------------------------------------------------- k_top1_pca
@@ -369,6 +451,90 @@ __global__ void __launch_bounds__(cb::THREADS) k_householder(const void* __restr
     }
 }
 
+// k_householder over 8-value chunks: per row, the dot product (lane-strided
+// chunks, then a warp sum), then y = x - c w chunk by chunk (the row is read
+// again, from L2).  Shared memory: w [K] | red [32].
+__global__ void __launch_bounds__(cb::THREADS) k_householder_v(const void* __restrict__ X, int xt, int M, int K,
+                                                              int64_t ldx, const float* __restrict__ v,
+                                                              float* __restrict__ Y) {
+    extern __shared__ float sm[];
+    float* w = sm;
+    float* red = sm + K;
+    const float sg = v[0] > 0.f ? -1.f : 1.f;
+    float sq = 0.f;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const float e = __fmul_rn(sg, v[k]);
+        const float wk = k == 0 ? __fsub_rn(e, 1.0f) : e;
+        w[k] = wk;
+        sq = __fmaf_rn(wk, wk, sq);
+    }
+    const float ww = block_sum(sq, red);
+    const float two_over = __fdiv_rn(2.0f, ww);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int m = blockIdx.x * nw + warp; m < M; m += gridDim.x * nw) {
+        const int64_t base = static_cast<int64_t>(m) * ldx;
+        float d = 0.f;
+        for (int k0 = 8 * lane; k0 < K; k0 += 2 * 256) {
+            float f[2][8];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (k0 + 256 * u < K) cb_load8(X, xt, base + k0 + 256 * u, f[u]);
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (k0 + 256 * u < K) {
+                    const float4 wa = *reinterpret_cast<const float4*>(w + k0 + 256 * u);
+                    const float4 wb = *reinterpret_cast<const float4*>(w + k0 + 256 * u + 4);
+                    const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d = __fmaf_rn(f[u][e], wv[e], d);
+                }
+        }
+        d = warp_sum(d);
+        const float c = __fmul_rn(two_over, d);
+        float* yr = Y + static_cast<int64_t>(m) * K;
+        for (int k0 = 8 * lane; k0 < K; k0 += 256) {
+            float f[8];
+            cb_load8(X, xt, base + k0, f);
+            const float4 wa = *reinterpret_cast<const float4*>(w + k0);
+            const float4 wb = *reinterpret_cast<const float4*>(w + k0 + 4);
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = __fsub_rn(f[e], __fmul_rn(c, wv[e]));
+            *reinterpret_cast<float4*>(yr + k0) = make_float4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<float4*>(yr + k0 + 4) = make_float4(o[4], o[5], o[6], o[7]);
+        }
+    }
+}
+
+// k_col_absmax over 8-column chunks: thread t of the strip owns columns
+// [8 t, 8 t + 8).
+__global__ void __launch_bounds__(cb::THREADS) k_col_absmax_v(const void* __restrict__ X, int xt, int M, int K,
+                                                             int64_t ldx, int rows_per,
+                                                             unsigned int* __restrict__ out) {
+    const int k0 = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (k0 >= K) return;
+    const int m0 = blockIdx.y * rows_per;
+    const int m1 = min(M, m0 + rows_per);
+    float mx[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int r = m0;
+    for (; r + 1 < m1; r += 2) {
+        float f[2][8];
+        cb_load8(X, xt, static_cast<int64_t>(r) * ldx + k0, f[0]);
+        cb_load8(X, xt, static_cast<int64_t>(r + 1) * ldx + k0, f[1]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fmaxf(fabsf(f[0][e]), fabsf(f[1][e])));
+    }
+    if (r < m1) {
+        float f[8];
+        cb_load8(X, xt, static_cast<int64_t>(r) * ldx + k0, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(f[e]));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) atomicMax(out + k0 + e, __float_as_uint(mx[e]));
+}
+
 // ---------------------------------------------------------------- k_col_absmax
 __global__ void __launch_bounds__(cb::THREADS) k_col_absmax(const void* __restrict__ X, int xt, int M, int K,
                                                            int64_t ldx, int rows_per, unsigned int* __restrict__ out) {
@@ -439,6 +605,45 @@ __global__ void __launch_bounds__(cb::THREADS) k_permute(const void* __restrict_
     }
 }
 
+// k_permute with the source row staged in shared memory (16-byte loads), then
+// gathered from there; four outputs per thread, one 16-byte store.  One CTA per
+// row at a time.  Shared memory: row [K] floats.
+__global__ void __launch_bounds__(cb::THREADS) k_permute_rows(const void* __restrict__ X, int xt, int M, int K,
+                                                             int64_t ldx, const int32_t* __restrict__ perm,
+                                                             const float* __restrict__ s, int op,
+                                                             float* __restrict__ Y) {
+    extern __shared__ float srow[];
+    for (int m = blockIdx.x; m < M; m += gridDim.x) {
+        const int64_t base = static_cast<int64_t>(m) * ldx;
+        for (int k0 = 8 * threadIdx.x; k0 < K; k0 += 8 * blockDim.x) {
+            float f[8];
+            cb_load8(X, xt, base + k0, f);
+            *reinterpret_cast<float4*>(srow + k0) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(srow + k0 + 4) = make_float4(f[4], f[5], f[6], f[7]);
+        }
+        __syncthreads();
+        float* yr = Y + static_cast<int64_t>(m) * K;
+        for (int j0 = 4 * threadIdx.x; j0 < K; j0 += 4 * blockDim.x) {
+            float o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int c = perm ? perm[j0 + e] : j0 + e;
+                float y = 0.f;
+                if (c < 0 || c >= K) {
+                    record_status(HQ_ERR_ARG);
+                } else {
+                    y = srow[c];
+                    if (op == 1) y = __fdiv_rn(y, s[c]);
+                    else if (op == 2) y = __fmul_rn(y, s[c]);
+                }
+                o[e] = y;
+            }
+            *reinterpret_cast<float4*>(yr + j0) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+        __syncthreads();   // the row is read before the next one is staged
+    }
+}
+
 static int cb_sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -448,6 +653,12 @@ static int cb_sm_count() {
 
 static bool cb_dtype_ok(hq_dtype t) { return t == HQ_F16 || t == HQ_BF16 || t == HQ_F32; }
 static hq_status cb_launched() { return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+static bool cb_al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// the 16-byte paths: X aligned, row stride a multiple of 16 bytes, K a multiple of 8
+static bool cb_vec(const void* X, hq_dtype xt, int64_t K, int64_t ld_x) {
+    const int64_t es = xt == HQ_F32 ? 4 : 2;
+    return cb_al16(X) && (ld_x * es) % 16 == 0 && K % 8 == 0;
+}
 
 }  // namespace hq
 
@@ -459,8 +670,12 @@ extern "C" hq_status hq_calib_extreme_tokens(const void* X, hq_dtype xt, int64_t
     if (S > INT32_MAX || L > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
     if (S == 0) return HQ_OK;
     if (!X || !tok || !T) return HQ_ERR_ARG;
-    k_extreme<<<static_cast<unsigned>(S), cb::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
-        X, xt, static_cast<int>(L), static_cast<int>(K), ld_x, tok, T);
+    if (cb_vec(X, xt, K, ld_x) && cb_al16(T))
+        k_extreme_v<<<static_cast<unsigned>(S), cb::EXT_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+            X, xt, static_cast<int>(L), static_cast<int>(K), ld_x, tok, T);
+    else
+        k_extreme<<<static_cast<unsigned>(S), cb::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+            X, xt, static_cast<int>(L), static_cast<int>(K), ld_x, tok, T);
     return cb_launched();
 }
 
@@ -509,11 +724,13 @@ extern "C" hq_status hq_calib_householder(const void* X, hq_dtype xt, int64_t M,
     if (M == 0) return HQ_OK;
     if (!X || !v || !Y) return HQ_ERR_ARG;
     const int smem = static_cast<int>((K + 32) * 4);
-    if (cudaFuncSetAttribute(k_householder, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    const bool vec = cb_vec(X, xt, K, ld_x) && cb_al16(Y);
+    auto kern = vec ? k_householder_v : k_householder;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
     const int64_t want = (M + cb::THREADS / 32 - 1) / (cb::THREADS / 32);
     const int grid = static_cast<int>(want < 4 * cb_sm_count() ? want : 4 * cb_sm_count());
-    k_householder<<<grid, cb::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+    kern<<<grid, cb::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
         X, xt, static_cast<int>(M), static_cast<int>(K), ld_x, v, Y);
     return cb_launched();
 }
@@ -526,14 +743,16 @@ extern "C" hq_status hq_calib_channel_absmax(const void* X, hq_dtype xt, int64_t
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(amax, 0, static_cast<size_t>(K) * sizeof(float), st) != cudaSuccess) return HQ_ERR_CUDA;
     if (M == 0) return HQ_OK;
-    const int gx = static_cast<int>((K + cb::THREADS - 1) / cb::THREADS);
+    const bool vec = cb_vec(X, xt, K, ld_x);
+    const int64_t cols_per = vec ? 8 * cb::THREADS : cb::THREADS;   // columns per CTA strip
+    const int gx = static_cast<int>((K + cols_per - 1) / cols_per);
     // about four CTAs per SM in all, each over a contiguous run of rows
     int gy = (4 * cb_sm_count() + gx - 1) / gx;
     if (gy > M) gy = static_cast<int>(M);
     const int rows_per = static_cast<int>((M + gy - 1) / gy);
     gy = static_cast<int>((M + rows_per - 1) / rows_per);
-    k_col_absmax<<<dim3(gx, gy), cb::THREADS, 0, st>>>(X, xt, static_cast<int>(M), static_cast<int>(K), ld_x,
-                                                       rows_per, reinterpret_cast<unsigned int*>(amax));
+    (vec ? k_col_absmax_v : k_col_absmax)<<<dim3(gx, gy), cb::THREADS, 0, st>>>(
+        X, xt, static_cast<int>(M), static_cast<int>(K), ld_x, rows_per, reinterpret_cast<unsigned int*>(amax));
     return cb_launched();
 }
 
@@ -560,6 +779,16 @@ extern "C" hq_status hq_permute_channels(const void* X, hq_dtype xt, int64_t M, 
     if (M > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
     if (M == 0) return HQ_OK;
     if (!X || !Y || (op != 0 && !s)) return HQ_ERR_ARG;
+    if (cb_vec(X, xt, K, ld_x) && cb_al16(Y) && K * 4 <= cb::SMEM_MAX - 1024) {
+        // the source row staged in shared memory, gathered from there
+        const int smem = static_cast<int>(K * 4);
+        if (cudaFuncSetAttribute(k_permute_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return HQ_ERR_CUDA;
+        const int grid = static_cast<int>(M < 4 * cb_sm_count() ? M : 4 * cb_sm_count());
+        k_permute_rows<<<grid, cb::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+            X, xt, static_cast<int>(M), static_cast<int>(K), ld_x, perm, s, op, Y);
+        return cb_launched();
+    }
     const int64_t blocks = (M * K + cb::THREADS - 1) / cb::THREADS;
     const int grid = static_cast<int>(blocks < 8 * cb_sm_count() ? blocks : 8 * cb_sm_count());
     k_permute<<<grid, cb::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
