@@ -21,9 +21,11 @@
 //  k_extreme      one CTA per calibration sequence: max |x| of every token
 //                 (exact), the arg max (ties to the earlier token), and the
 //                 chosen token widened to fp32.
-//  k_top1_pca     one CTA, power iteration on C = T^T T / S without forming C
-//                 (y = T v, z = T^T y / S, v = z / |z|), v and y in shared
-//                 memory, every sum in a fixed order (deterministic).
+//  k_top1_pca_cl  power iteration on C = T^T T / S without forming C
+//                 (y = T v, z = T^T y / S, v = z / |z|) on a cluster of 8 CTAs
+//                 holding T in their shared memory; k_top1_pca, one CTA reading
+//                 T from L2, when it does not fit.  Every sum in a fixed order
+//                 (deterministic).
 //  k_householder  one warp per row: Y = X Q with Q = I - 2 w w^T / (w^T w),
 //                 w = v' - e0, v' = +-v with v'[0] <= 0, so Q v' = e0.
 //  k_col_absmax   column max |x| with integer atomics on the (non-negative)
@@ -33,6 +35,9 @@
 //                 perm[position] = channel.
 //  k_flatten      s[k] = xmax[k]^alpha / wmax[k]^(1 - alpha).
 //  k_permute      Y[m][j] = X[m][perm[j]] (divided or multiplied by s[perm[j]]).
+// k_extreme_v, k_householder_v, k_col_absmax_v and k_permute_rows are the same
+// operations with 16-byte loads, taken when X is 16-byte aligned, its row stride
+// a multiple of 16 bytes and K a multiple of 8.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
