@@ -571,8 +571,13 @@ def main():
     dev = torch.device("cuda", local)
     R = Runner(torch, hq, synth, rank, dev)
     if args.calibration_only:
+        # every rank calibrates its own copy (no collective); rank 0 prints
+        rec = calibration_record(R)
         if rank == 0:
-            print(json.dumps({"calibration": calibration_record(R)}), flush=True)
+            print(json.dumps({"calibration": rec}), flush=True)
+        if pg is not None:
+            pg.barrier()
+            pg.destroy_process_group()
         return
     steps = args.steps if args.steps is not None else DEFAULT_STEPS
     warm = max(args.warmup, 3)
