@@ -15,7 +15,14 @@ attention projection (M = 2048; 4096 -> 4096, one Hadamard group of 4096) and
 the Llama-70B MLP shape (M = 512, 2048, 8192; 8192 -> 28672), each with K1's
 HBM throughput and fraction of the HBM roofline and K2's TOP/s and fraction of
 the dense int8 tensor peak (of HBM for decode).  "serq_overhead" compares K2
-with and without the SERQ term on the same weights.
+with and without the SERQ term on the same weights; "activation_variants"
+times the W4A8 and OffQ activations on the decode and down layers;
+"calibration" times the offline calibration kernels of the down layer.
+
+"e2e" is the same metric through the public call (W4A4Linear) with pinned host
+buffers: every step copies its activations in and its output back, on three
+streams (copy in, compute, copy out) with events guarding buffer reuse, so a
+later step's copy in overlaps the compute and copy out of earlier ones.
 
 Timing: every layer shape runs over a rotating pool of layers and batches
 (distinct weights and activations) holding more bytes than 2x the 126 MB L2;
