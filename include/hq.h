@@ -468,6 +468,29 @@ hq_status hq_calib_flatten_scales(const float* xmax, const float* wmax, int64_t 
 hq_status hq_permute_channels(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x,
                               const int32_t* perm, const float* s, int32_t op, float* Y, void* stream);
 
+/*
+ * hq_quant_mxfp4 -- MXFP4 block quantisation of rows of values (the 4-bit
+ * format SERQ names beside INT4 for its main and residual paths, "SERQ:
+ * Saliency-Aware Low-Rank Error Reconstruction for LLM Quantization",
+ * technical summary sections 2 and 3).  Per block of 32 consecutive values
+ * of a row: E = floor(log2(amax)) - 2, scale byte = clamp(E + 127, 0, 254)
+ * (UE8M0; 0 for an all-zero block), t = v * 2^-(byte - 127), |t| rounded to
+ * the E2M1 grid {0, 0.5, 1, 1.5, 2, 3, 4, 6} to nearest with ties to the even
+ * mantissa (0, 1, 2, 4) and saturated at 6, sign bit 3 for t < 0 with a
+ * non-zero magnitude; element 2j in the low nibble of byte j.  Activations
+ * are quantised after hq_rotate (fp32 rows), weights as W_rot.  Inputs must
+ * be finite.
+ *  X       device, [M][ld_x] (HQ_F16, HQ_BF16 or HQ_F32), 16-byte aligned,
+ *          ld_x * element size a multiple of 16
+ *  Xq      device, [M][K/2] codes (output), 16-byte aligned
+ *  scales  device, [M][K/32] scale bytes (output)
+ * Errors: HQ_ERR_ARG (M < 0, K <= 0, K % 32, ld_x < K, bad dtype, NULL with
+ * M > 0), HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED (a size above INT32_MAX),
+ * HQ_ERR_CUDA.  M == 0 is a no-op.
+ */
+hq_status hq_quant_mxfp4(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x, uint8_t* Xq,
+                         uint8_t* scales, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

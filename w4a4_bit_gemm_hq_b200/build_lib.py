@@ -8,7 +8,7 @@ from concurrent.futures import ThreadPoolExecutor
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhq.so")
-SOURCES = ["abi.cu", "rotate.cu", "rotq.cu", "pack.cu", "gemm.cu", "gemm_small.cu", "noalloc.cu", "calib.cu"]
+SOURCES = ["abi.cu", "rotate.cu", "rotq.cu", "pack.cu", "gemm.cu", "gemm_small.cu", "noalloc.cu", "calib.cu", "mxfp4.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-Xptxas", "-v"]

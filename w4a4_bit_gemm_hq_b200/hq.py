@@ -23,7 +23,7 @@ __all__ = [
     "hq_rotate_quant8", "w4a8_linear", "hq_debug_accum8", "hq_rotate_quant_asym", "w4a4_linear_asym",
     "hq_debug_accum_asym", "hq_calib_extreme_tokens", "hq_calib_top1_pca", "hq_calib_householder",
     "hq_calib_channel_absmax", "hq_calib_sorted_perm", "hq_calib_flatten_scales", "hq_permute_channels",
-    "calibrate_rotation_and_grouping",
+    "calibrate_rotation_and_grouping", "hq_quant_mxfp4",
 ]
 
 
@@ -331,6 +331,17 @@ def calibrate_rotation_and_grouping(X_calib, S, L, W, iters=100):
     perm = hq_calib_sorted_perm(hq_calib_channel_absmax(Xr))
     W_cal = hq_permute_channels(hq_calib_householder(W, v), perm)
     return v, perm, W_cal
+
+
+def hq_quant_mxfp4(X, Xq=None, scales=None):
+    """(codes uint8 [M, K/2], scale bytes uint8 [M, K/32]): MXFP4 blocks of 32
+    values (E2M1 codes, UE8M0 shared exponent) of the rows of X."""
+    M, K = X.shape
+    Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device) if Xq is None else Xq
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=X.device) if scales is None else scales
+    check(lib.hq_quant_mxfp4(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), ptr(Xq), ptr(scales),
+                             stream_handle()), "hq_quant_mxfp4")
+    return Xq, scales
 
 
 def hq_last_device_status():
