@@ -93,3 +93,9 @@ def dequant_mxfp4(packed, sb, K):
     sign = np.where(q & 8, -1.0, 1.0)
     X = np.ldexp(1.0, np.repeat(np.asarray(sb, np.int64), 32, axis=1) - 127)
     return sign * mag * X
+
+
+def linear_f64(qx, sbx, qw, sbw, K):
+    """Y = X^ W^T in float64 with X^, W^ the values the MXFP4 codes stand for
+    (every product and sum is exact in float64 for these magnitudes)."""
+    return dequant_mxfp4(qx, sbx, K) @ dequant_mxfp4(qw, sbw, K).T

@@ -71,3 +71,39 @@ def test_zero_block_and_packing():
     codes = [OM.code_of((j - 16.0) / 4.0) for j in range(32)]
     for j in range(16):
         assert q[1, 16 + j] == codes[2 * j] | (codes[2 * j + 1] << 4)
+
+
+def test_linear_of_representable_values_is_the_exact_product():
+    # values already on the MXFP4 grid quantise to themselves: the product of
+    # the codes is the plain matrix product of the inputs
+    rng = np.random.default_rng(7)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    def on_grid(rows):
+        v = grid[rng.integers(0, 8, size=(rows, 64))] * np.where(rng.random((rows, 64)) < 0.5, -1, 1)
+        v[:, 0] = 6.0                        # amax 6 -> E = 0 in block 0
+        v[:, 32] = -4.0                      # amax 4 -> E = 0 in block 1
+        return (v * np.repeat(np.ldexp(1.0, rng.integers(-6, 6, size=(rows, 2))), 32, axis=1)).astype(np.float32)
+    X, W = on_grid(5), on_grid(3)
+    qx, sx = OM.quant_mxfp4(X)
+    qw, sw = OM.quant_mxfp4(W)
+    np.testing.assert_array_equal(OM.dequant_mxfp4(qx, sx, 64), X.astype(np.float64))
+    np.testing.assert_array_equal(OM.linear_f64(qx, sx, qw, sw, 64), X.astype(np.float64) @ W.T.astype(np.float64))
+
+
+def test_linear_brute_force():
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((3, 64)).astype(np.float32)
+    W = rng.standard_normal((2, 64)).astype(np.float32)
+    qx, sx = OM.quant_mxfp4(X)
+    qw, sw = OM.quant_mxfp4(W)
+    Y = OM.linear_f64(qx, sx, qw, sw, 64)
+    for m in range(3):
+        for n in range(2):
+            acc = 0.0
+            for k in range(64):
+                cx = (qx[m, k // 2] >> (4 * (k % 2))) & 15
+                cw = (qw[n, k // 2] >> (4 * (k % 2))) & 15
+                vx = (-1 if cx & 8 else 1) * OM.E2M1[cx & 7] * 2.0 ** (int(sx[m, k // 32]) - 127)
+                vw = (-1 if cw & 8 else 1) * OM.E2M1[cw & 7] * 2.0 ** (int(sw[n, k // 32]) - 127)
+                acc += vx * vw
+            assert Y[m, n] == acc
