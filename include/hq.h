@@ -491,6 +491,24 @@ hq_status hq_permute_channels(const void* X, hq_dtype xt, int64_t M, int64_t K, 
 hq_status hq_quant_mxfp4(const void* X, hq_dtype xt, int64_t M, int64_t K, int64_t ld_x, uint8_t* Xq,
                          uint8_t* scales, void* stream);
 
+/*
+ * hq_mxfp4_linear -- Y = X^ W^T for MXFP4 operands (codes and scale bytes as
+ * hq_quant_mxfp4 writes them), X^, W^ the values the codes stand for.  Twice
+ * an E2M1 value is an integer in [-12, 12], so each 32-value block of a row
+ * pair is an exact int8 dot product (warp-level int8 MMA); the block sums are
+ * scaled by 2^(Ex + Ew) (exact) and added in fp32 in block order.  The
+ * block-scaled tensor-core MMA (tcgen05 kind::mxf4) is not used.  Two calls
+ * with accumulate = 1 on the second add SERQ's residual product (salient
+ * activation block against the MXFP4 error rows) to the main one.
+ *  Xq, sx   device, [M][K/2] codes and [M][K/32] scale bytes (2-byte aligned)
+ *  Wq, sw   device, [N][K/2] codes and [N][K/32] scale bytes (row-major)
+ *  Y        device, [M][N] fp32 (output; accumulate != 0: added to), 4-byte aligned
+ * Errors: HQ_ERR_ARG (M < 0, N < 0, K <= 0, K % 32, NULL with M, N > 0),
+ * HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED (a size above INT32_MAX), HQ_ERR_CUDA.
+ */
+hq_status hq_mxfp4_linear(const uint8_t* Xq, const uint8_t* sx, int64_t M, int64_t K, const uint8_t* Wq,
+                          const uint8_t* sw, int64_t N, float* Y, int32_t accumulate, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

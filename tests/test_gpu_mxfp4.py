@@ -79,3 +79,53 @@ def test_argument_errors():
     assert lib.hq_quant_mxfp4(p(X), 2, 4, 64, 66, p(q), p(s), None) == E.HQ_ERR_ALIGN     # stride 264 bytes
     assert lib.hq_quant_mxfp4(p(X), 2, 0, 64, 64, None, None, None) == E.HQ_OK
     no_device_error()
+
+
+def _bound(qx, sx, qw, sw, K):
+    """fp32 accumulation of K/32 exact block sums: |err| <= (K/32) 2^-24 sum |x^ w^|."""
+    ax = np.abs(OM.dequant_mxfp4(qx, sx, K))
+    aw = np.abs(OM.dequant_mxfp4(qw, sw, K))
+    return (K // 32) * 2.0 ** -24 * (ax @ aw.T)
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 8, 32), (33, 70, 256), (100, 130, 1024), (7, 2048, 4096)])
+def test_mxfp4_linear_within_accumulation_bound(M, N, K):
+    rng = np.random.default_rng(M + N)
+    X = (rng.standard_t(3, size=(M, K)) * 2).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    qx, sx = hq.hq_quant_mxfp4(torch.from_numpy(X).cuda())
+    qw, sw = hq.hq_quant_mxfp4(torch.from_numpy(W).cuda())
+    Y = host(hq.hq_mxfp4_linear(qx, sx, qw, sw)).astype(np.float64)
+    hqx, hsx, hqw, hsw = host(qx), host(sx), host(qw), host(sw)
+    Y64 = OM.linear_f64(hqx, hsx, hqw, hsw, K)
+    assert (np.abs(Y - Y64) <= _bound(hqx, hsx, hqw, hsw, K)).all()
+    no_device_error()
+
+
+def test_mxfp4_layer_with_residual_term_on_the_down_shape():
+    # main product over K = 11008 plus SERQ's residual path on 32 salient
+    # channels (one MXFP4 block), the second call accumulating into the first
+    wl = synth.WORKLOADS["down"]
+    M, N, K, r = 64, 512, wl.K, 32
+    X = synth.activations(wl, M=M)
+    d = torch.from_numpy(synth.hadamard_signs(wl.g)).cuda()
+    V = hq.hq_rotate(dev(X, wl.xdtype), wl.g, d)
+    W = (np.random.default_rng(3).standard_normal((N, K)) * 0.015).astype(np.float32)
+    sal = np.sort(np.random.default_rng(4).choice(K, r, replace=False))
+    R = (np.random.default_rng(5).standard_normal((N, r)) * 0.003).astype(np.float32)
+    qx, sx = hq.hq_quant_mxfp4(V)
+    qw, sw = hq.hq_quant_mxfp4(torch.from_numpy(W).cuda())
+    Vs = V[:, torch.from_numpy(sal).cuda()].contiguous()
+    qs, ss = hq.hq_quant_mxfp4(Vs)
+    qr, sr = hq.hq_quant_mxfp4(torch.from_numpy(R).cuda())
+    Y = hq.hq_mxfp4_linear(qx, sx, qw, sw)
+    Y = host(hq.hq_mxfp4_linear(qs, ss, qr, sr, Y=Y, accumulate=True)).astype(np.float64)
+    h = [host(t) for t in (qx, sx, qw, sw, qs, ss, qr, sr)]
+    Y64 = OM.linear_f64(h[0], h[1], h[2], h[3], K) + OM.linear_f64(h[4], h[5], h[6], h[7], r)
+    bound = _bound(h[0], h[1], h[2], h[3], K) + _bound(h[4], h[5], h[6], h[7], r) + 2.0 ** -24 * np.abs(Y64)
+    assert (np.abs(Y - Y64) <= bound).all()
+    # and the codes of the gathered salient block are the oracle's
+    q_o, s_o = OM.quant_mxfp4(host(Vs))
+    assert_same(h[4], q_o, "salient codes")
+    assert_same(h[5], s_o, "salient scale bytes")
+    no_device_error()

@@ -63,6 +63,7 @@ SIGNATURES = {
     "hq_calib_flatten_scales": ([_P, _P, _I64, ct.c_float, _P, _P], _ST),
     "hq_permute_channels": ([_P, ct.c_int, _I64, _I64, _I64, _P, _P, _I32, _P, _P], _ST),
     "hq_quant_mxfp4": ([_P, ct.c_int, _I64, _I64, _I64, _P, _P, _P], _ST),
+    "hq_mxfp4_linear": ([_P, _P, _I64, _I64, _P, _P, _I64, _P, _I32, _P], _ST),
     "hq_last_device_status": ([_P], _ST),
     "hq_debug_wait_probe": ([ct.c_uint64, _P], _ST),
 }

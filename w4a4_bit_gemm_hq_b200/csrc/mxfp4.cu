@@ -15,8 +15,9 @@
 //
 // One thread per block: the 32 values arrive as 16-byte loads, the block
 // maximum is the thread's own, 16 bytes of codes and one scale byte leave.
-// The layer's own GEMM on these codes (tcgen05.mma kind::mxf4) is not part of
-// this file.
+// hq_mxfp4_linear multiplies two such code matrices exactly per block on the
+// warp-level int8 MMA (twice an E2M1 value is an integer); the block-scaled
+// tensor-core form (tcgen05.mma kind::mxf4) is not built.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -102,6 +103,75 @@ __global__ void __launch_bounds__(MX_THREADS) k_mxfp4(const void* __restrict__ X
     }
 }
 
+// ---------------------------------------------------------------- k_mx_gemm
+// Y[m][n] (+)= sum over blocks b of 2^(Ex + Ew) sum_{k in b} x_k w_k with x, w
+// the E2M1 values of the codes.  Twice an E2M1 value is an integer in
+// [-12, 12], so one block of one row pair is one exact int8 dot product of 32
+// terms: one warp-level mma.sync.m16n8k32.s8 per block computes a 16 x 8 tile's
+// block sums exactly (|sum| <= 32 * 144); the tile adds them, scaled by the
+// power of two 2^(bx + bw - 256) (exact), in fp32 in block order.
+__device__ __forceinline__ uint32_t mx_expand4(uint32_t v) {
+    // nibble i = code of element i -> byte i = 2 * value, two's complement
+    const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, v & 0x7777u);   // 0,1,2,3,4,6,8,12
+    uint32_t neg = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) neg |= ((v >> (4 * i + 3)) & 1u) * (0xFFu << (8 * i));
+    return (mag & ~neg) | (__vsub4(0u, mag) & neg);
+}
+
+__device__ __forceinline__ void mx_mma(int32_t (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+constexpr int MXG_WARPS = 8;
+
+__global__ void __launch_bounds__(MXG_WARPS * 32) k_mx_gemm(const uint8_t* __restrict__ Xq, const uint8_t* __restrict__ sx,
+                                                           const uint8_t* __restrict__ Wq, const uint8_t* __restrict__ sw,
+                                                           int M, int N, int K, float* __restrict__ Y, int accumulate) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const int tiles_n = (N + 7) / 8;
+    const int64_t tile = static_cast<int64_t>(blockIdx.x) * MXG_WARPS + warp;
+    const int64_t tiles = static_cast<int64_t>((M + 15) / 16) * tiles_n;
+    if (tile >= tiles) return;   // whole warps only
+    const int tm = static_cast<int>(tile / tiles_n), tn = static_cast<int>(tile % tiles_n);
+    const int r0 = 16 * tm + g8, r1 = r0 + 8, nB = 8 * tn + g8;   // A rows, B column of this lane
+    const int c0 = 8 * tn + 2 * t4;                                // C columns c0, c0 + 1
+    const bool v0 = r0 < M, v1 = r1 < M, vB = nB < N, vc0 = c0 < N, vc1 = c0 + 1 < N;
+    const int nb = K / 32;
+    const int64_t ldq = K / 2;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int b = 0; b < nb; ++b) {
+        const int64_t o = 16 * static_cast<int64_t>(b) + 2 * t4;
+        uint32_t a[4];
+        a[0] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o)) : 0u;
+        a[1] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o)) : 0u;
+        a[2] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o + 8)) : 0u;
+        a[3] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o + 8)) : 0u;
+        const uint32_t b0 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o)) : 0u;
+        const uint32_t b1 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o + 8)) : 0u;
+        int32_t c[4] = {0, 0, 0, 0};
+        mx_mma(c, a, b0, b1);
+        const int ex0 = v0 ? sx[static_cast<int64_t>(r0) * nb + b] : 0, ex1 = v1 ? sx[static_cast<int64_t>(r1) * nb + b] : 0;
+        const int ew0 = vc0 ? sw[static_cast<int64_t>(c0) * nb + b] : 0, ew1 = vc1 ? sw[static_cast<int64_t>(c0 + 1) * nb + b] : 0;
+        // (2x)(2w) / 4 * 2^(bx - 127) * 2^(bw - 127)
+        y[0] = __fmaf_rn(static_cast<float>(c[0]), ldexpf(1.0f, ex0 + ew0 - 256), y[0]);
+        y[1] = __fmaf_rn(static_cast<float>(c[1]), ldexpf(1.0f, ex0 + ew1 - 256), y[1]);
+        y[2] = __fmaf_rn(static_cast<float>(c[2]), ldexpf(1.0f, ex1 + ew0 - 256), y[2]);
+        y[3] = __fmaf_rn(static_cast<float>(c[3]), ldexpf(1.0f, ex1 + ew1 - 256), y[3]);
+    }
+    float* Y0 = Y + static_cast<int64_t>(r0) * N;
+    float* Y1 = Y + static_cast<int64_t>(r1) * N;
+    if (v0 && vc0) Y0[c0] = accumulate ? __fadd_rn(Y0[c0], y[0]) : y[0];
+    if (v0 && vc1) Y0[c0 + 1] = accumulate ? __fadd_rn(Y0[c0 + 1], y[1]) : y[1];
+    if (v1 && vc0) Y1[c0] = accumulate ? __fadd_rn(Y1[c0], y[2]) : y[2];
+    if (v1 && vc1) Y1[c0 + 1] = accumulate ? __fadd_rn(Y1[c0 + 1], y[3]) : y[3];
+}
+
 bool mx_al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
@@ -125,5 +195,22 @@ extern "C" hq_status hq_quant_mxfp4(const void* X, hq_dtype xt, int64_t M, int64
     const int grid = static_cast<int>(blocks < 8 * nsm ? blocks : 8 * nsm);
     k_mxfp4<<<grid, MX_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(X, xt, static_cast<int>(M),
                                                                       static_cast<int>(K), ld_x, Xq, scales);
+    return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+extern "C" hq_status hq_mxfp4_linear(const uint8_t* Xq, const uint8_t* sx, int64_t M, int64_t K, const uint8_t* Wq,
+                                     const uint8_t* sw, int64_t N, float* Y, int32_t accumulate, void* stream) {
+    if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return HQ_ERR_ARG;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return HQ_OK;
+    if (!Xq || !sx || !Wq || !sw || !Y) return HQ_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(Xq) & 1u) || (reinterpret_cast<uintptr_t>(Wq) & 1u) ||
+        (reinterpret_cast<uintptr_t>(Y) & 3u))
+        return HQ_ERR_ALIGN;
+    const int64_t tiles = ((M + 15) / 16) * ((N + 7) / 8);
+    const int64_t grid = (tiles + MXG_WARPS - 1) / MXG_WARPS;
+    if (grid > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+    k_mx_gemm<<<static_cast<unsigned>(grid), MXG_WARPS * 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        Xq, sx, Wq, sw, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), Y, accumulate ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }

@@ -23,7 +23,7 @@ __all__ = [
     "hq_rotate_quant8", "w4a8_linear", "hq_debug_accum8", "hq_rotate_quant_asym", "w4a4_linear_asym",
     "hq_debug_accum_asym", "hq_calib_extreme_tokens", "hq_calib_top1_pca", "hq_calib_householder",
     "hq_calib_channel_absmax", "hq_calib_sorted_perm", "hq_calib_flatten_scales", "hq_permute_channels",
-    "calibrate_rotation_and_grouping", "hq_quant_mxfp4",
+    "calibrate_rotation_and_grouping", "hq_quant_mxfp4", "hq_mxfp4_linear",
 ]
 
 
@@ -342,6 +342,17 @@ def hq_quant_mxfp4(X, Xq=None, scales=None):
     check(lib.hq_quant_mxfp4(ptr(X), dtype_code(X.dtype), M, K, X.stride(0), ptr(Xq), ptr(scales),
                              stream_handle()), "hq_quant_mxfp4")
     return Xq, scales
+
+
+def hq_mxfp4_linear(Xq, sx, Wq, sw, Y=None, accumulate=False):
+    """Y float32 [M, N] (+)= X^ W^T for MXFP4 codes and scale bytes."""
+    M, N, K = Xq.shape[0], Wq.shape[0], 2 * Xq.shape[1]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=Xq.device)
+        accumulate = False
+    check(lib.hq_mxfp4_linear(ptr(Xq), ptr(sx), M, K, ptr(Wq), ptr(sw), N, ptr(Y), 1 if accumulate else 0,
+                              stream_handle()), "hq_mxfp4_linear")
+    return Y
 
 
 def hq_last_device_status():
