@@ -444,6 +444,29 @@ class Shape:
             b2 = k2_bytes(M, wl.N, wl.K, wl.gw, self.r) + 8 * M * G - 4 * M
             out.append(self._variant("offq", k1_a, k2_a, b1, b2, decode_like))
             del sxa, zxa
+        if not decode_like:
+            # MXFP4: hq_rotate (fp32 rows) + hq_quant_mxfp4, then hq_mxfp4_linear on
+            # MXFP4 weights (one weight set, quantised once, shared by the pool)
+            G = wl.K // 32
+            V = [torch.empty((M, wl.K), dtype=torch.float32, device=R.dev) for _ in range(P)]
+            qx = [torch.empty((M, wl.K // 2), dtype=torch.uint8, device=R.dev) for _ in range(P)]
+            sbx = [torch.empty((M, G), dtype=torch.uint8, device=R.dev) for _ in range(P)]
+            Wf = R.to_dev(R.synth.weights(wl), wl.wdtype)
+            qw, sbw = hq.hq_quant_mxfp4(hq.hq_rotate(Wf, wl.g, self.layers[0].H_signs))
+            del Wf
+            Ymx = [torch.empty((M, wl.N), dtype=torch.float32, device=R.dev) for _ in range(P)]
+
+            def k1_m(i):
+                hq.hq_rotate(self.X[i], wl.g, self.layers[i].H_signs, V[i])
+                hq.hq_quant_mxfp4(V[i], qx[i], sbx[i])
+
+            k2_m = lambda i: hq.hq_mxfp4_linear(qx[i], sbx[i], qw, sbw, Ymx[i])
+            b1 = 2 * M * wl.K + 2 * 4 * M * wl.K + M * wl.K // 2 + M * G
+            b2 = wl.N * wl.K // 2 + wl.N * G + M * wl.K // 2 + M * G + 4 * M * wl.N
+            rec = self._variant("mxfp4 (rotate to fp32 + block quantiser; int8 mma.sync GEMM)", k1_m, k2_m, b1, b2,
+                                decode_like)
+            out.append(rec)
+            del V, qx, sbx, qw, sbw, Ymx
         return out
 
     def _variant(self, name, k1, k2, b1, b2, decode_like):

@@ -109,7 +109,8 @@ __global__ void __launch_bounds__(MX_THREADS) k_mxfp4(const void* __restrict__ X
 // [-12, 12], so one block of one row pair is one exact int8 dot product of 32
 // terms: one warp-level mma.sync.m16n8k32.s8 per block computes a 16 x 8 tile's
 // block sums exactly (|sum| <= 32 * 144); the tile adds them, scaled by the
-// power of two 2^(bx + bw - 256) (exact), in fp32 in block order.
+// power of two 2^(bx + bw - 256) (exact), in fp32 in block order.  A warp owns
+// 32 x 32 outputs, so each expanded fragment feeds several MMAs.
 __device__ __forceinline__ uint32_t mx_expand4(uint32_t v) {
     // nibble i = code of element i -> byte i = 2 * value, two's complement
     const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, v & 0x7777u);   // 0,1,2,3,4,6,8,12
@@ -127,49 +128,90 @@ __device__ __forceinline__ void mx_mma(int32_t (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 2^(e - 128) for a scale byte e, exactly (subnormal for e < 2)
+__device__ __forceinline__ float mx_half_scale(int e) {
+    return __int_as_float(e >= 2 ? (e - 1) << 23 : 1 << (21 + e));
+}
+
+// an int32 of magnitude below 2^22 as a float, exactly: its bits added to those
+// of 1.5 * 2^23 form the float 1.5 * 2^23 + c
+__device__ __forceinline__ float mx_i2f(int32_t c) { return __fsub_rn(__int_as_float(c + 0x4B400000), 12582912.0f); }
+
 constexpr int MXG_WARPS = 8;
+constexpr int MXG_MT = 2, MXG_NT = 4;   // a warp's tile: 2 x 16 rows by 4 x 8 columns
 
 __global__ void __launch_bounds__(MXG_WARPS * 32) k_mx_gemm(const uint8_t* __restrict__ Xq, const uint8_t* __restrict__ sx,
                                                            const uint8_t* __restrict__ Wq, const uint8_t* __restrict__ sw,
                                                            int M, int N, int K, float* __restrict__ Y, int accumulate) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
-    const int tiles_n = (N + 7) / 8;
+    const int tiles_n = (N + 8 * MXG_NT - 1) / (8 * MXG_NT);
     const int64_t tile = static_cast<int64_t>(blockIdx.x) * MXG_WARPS + warp;
-    const int64_t tiles = static_cast<int64_t>((M + 15) / 16) * tiles_n;
+    const int64_t tiles = static_cast<int64_t>((M + 16 * MXG_MT - 1) / (16 * MXG_MT)) * tiles_n;
     if (tile >= tiles) return;   // whole warps only
-    const int tm = static_cast<int>(tile / tiles_n), tn = static_cast<int>(tile % tiles_n);
-    const int r0 = 16 * tm + g8, r1 = r0 + 8, nB = 8 * tn + g8;   // A rows, B column of this lane
-    const int c0 = 8 * tn + 2 * t4;                                // C columns c0, c0 + 1
-    const bool v0 = r0 < M, v1 = r1 < M, vB = nB < N, vc0 = c0 < N, vc1 = c0 + 1 < N;
+    const int m0 = static_cast<int>(tile / tiles_n) * 16 * MXG_MT, n0 = static_cast<int>(tile % tiles_n) * 8 * MXG_NT;
     const int nb = K / 32;
     const int64_t ldq = K / 2;
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    float y[MXG_MT][MXG_NT][4];
+#pragma unroll
+    for (int mt = 0; mt < MXG_MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < MXG_NT; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y[mt][nt][q] = 0.f;
     for (int b = 0; b < nb; ++b) {
         const int64_t o = 16 * static_cast<int64_t>(b) + 2 * t4;
-        uint32_t a[4];
-        a[0] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o)) : 0u;
-        a[1] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o)) : 0u;
-        a[2] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o + 8)) : 0u;
-        a[3] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o + 8)) : 0u;
-        const uint32_t b0 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o)) : 0u;
-        const uint32_t b1 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o + 8)) : 0u;
-        int32_t c[4] = {0, 0, 0, 0};
-        mx_mma(c, a, b0, b1);
-        const int ex0 = v0 ? sx[static_cast<int64_t>(r0) * nb + b] : 0, ex1 = v1 ? sx[static_cast<int64_t>(r1) * nb + b] : 0;
-        const int ew0 = vc0 ? sw[static_cast<int64_t>(c0) * nb + b] : 0, ew1 = vc1 ? sw[static_cast<int64_t>(c0 + 1) * nb + b] : 0;
-        // (2x)(2w) / 4 * 2^(bx - 127) * 2^(bw - 127)
-        y[0] = __fmaf_rn(static_cast<float>(c[0]), ldexpf(1.0f, ex0 + ew0 - 256), y[0]);
-        y[1] = __fmaf_rn(static_cast<float>(c[1]), ldexpf(1.0f, ex0 + ew1 - 256), y[1]);
-        y[2] = __fmaf_rn(static_cast<float>(c[2]), ldexpf(1.0f, ex1 + ew0 - 256), y[2]);
-        y[3] = __fmaf_rn(static_cast<float>(c[3]), ldexpf(1.0f, ex1 + ew1 - 256), y[3]);
+        uint32_t a[MXG_MT][4];
+        int ex[MXG_MT][2];
+        float fx[MXG_MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MXG_MT; ++mt) {
+            const int r0 = m0 + 16 * mt + g8, r1 = r0 + 8;
+            const bool v0 = r0 < M, v1 = r1 < M;
+            a[mt][0] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o)) : 0u;
+            a[mt][1] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o)) : 0u;
+            a[mt][2] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o + 8)) : 0u;
+            a[mt][3] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o + 8)) : 0u;
+            ex[mt][0] = v0 ? sx[static_cast<int64_t>(r0) * nb + b] : 0;
+            ex[mt][1] = v1 ? sx[static_cast<int64_t>(r1) * nb + b] : 0;
+            fx[mt][0] = mx_half_scale(ex[mt][0]);
+            fx[mt][1] = mx_half_scale(ex[mt][1]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < MXG_NT; ++nt) {
+            const int nB = n0 + 8 * nt + g8, c0 = n0 + 8 * nt + 2 * t4;
+            const bool vB = nB < N;
+            const uint32_t b0 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o)) : 0u;
+            const uint32_t b1 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o + 8)) : 0u;
+            const int ew0 = c0 < N ? sw[static_cast<int64_t>(c0) * nb + b] : 0;
+            const int ew1 = c0 + 1 < N ? sw[static_cast<int64_t>(c0 + 1) * nb + b] : 0;
+            const float fw0 = mx_half_scale(ew0), fw1 = mx_half_scale(ew1);
+#pragma unroll
+            for (int mt = 0; mt < MXG_MT; ++mt) {
+                int32_t c[4] = {0, 0, 0, 0};
+                mx_mma(c, a[mt], b0, b1);
+                // (2x)(2w) / 4 * 2^(bx - 127) * 2^(bw - 127) = c 2^(bx - 128) 2^(bw - 128)
+                y[mt][nt][0] = __fmaf_rn(mx_i2f(c[0]), __fmul_rn(fx[mt][0], fw0), y[mt][nt][0]);
+                y[mt][nt][1] = __fmaf_rn(mx_i2f(c[1]), __fmul_rn(fx[mt][0], fw1), y[mt][nt][1]);
+                y[mt][nt][2] = __fmaf_rn(mx_i2f(c[2]), __fmul_rn(fx[mt][1], fw0), y[mt][nt][2]);
+                y[mt][nt][3] = __fmaf_rn(mx_i2f(c[3]), __fmul_rn(fx[mt][1], fw1), y[mt][nt][3]);
+            }
+        }
     }
-    float* Y0 = Y + static_cast<int64_t>(r0) * N;
-    float* Y1 = Y + static_cast<int64_t>(r1) * N;
-    if (v0 && vc0) Y0[c0] = accumulate ? __fadd_rn(Y0[c0], y[0]) : y[0];
-    if (v0 && vc1) Y0[c0 + 1] = accumulate ? __fadd_rn(Y0[c0 + 1], y[1]) : y[1];
-    if (v1 && vc0) Y1[c0] = accumulate ? __fadd_rn(Y1[c0], y[2]) : y[2];
-    if (v1 && vc1) Y1[c0 + 1] = accumulate ? __fadd_rn(Y1[c0 + 1], y[3]) : y[3];
+#pragma unroll
+    for (int mt = 0; mt < MXG_MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < MXG_NT; ++nt) {
+            const int r0 = m0 + 16 * mt + g8, r1 = r0 + 8, c0 = n0 + 8 * nt + 2 * t4;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = q < 2 ? r0 : r1, cc = c0 + (q & 1);
+                if (r < M && cc < N) {
+                    float* dst = Y + static_cast<int64_t>(r) * N + cc;
+                    *dst = accumulate ? __fadd_rn(*dst, y[mt][nt][q]) : y[mt][nt][q];
+                }
+            }
+        }
 }
 
 bool mx_al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -207,7 +249,7 @@ extern "C" hq_status hq_mxfp4_linear(const uint8_t* Xq, const uint8_t* sx, int64
     if ((reinterpret_cast<uintptr_t>(Xq) & 1u) || (reinterpret_cast<uintptr_t>(Wq) & 1u) ||
         (reinterpret_cast<uintptr_t>(Y) & 3u))
         return HQ_ERR_ALIGN;
-    const int64_t tiles = ((M + 15) / 16) * ((N + 7) / 8);
+    const int64_t tiles = ((M + 16 * MXG_MT - 1) / (16 * MXG_MT)) * ((N + 8 * MXG_NT - 1) / (8 * MXG_NT));
     const int64_t grid = (tiles + MXG_WARPS - 1) / MXG_WARPS;
     if (grid > INT32_MAX) return HQ_ERR_UNSUPPORTED;
     k_mx_gemm<<<static_cast<unsigned>(grid), MXG_WARPS * 32, 0, static_cast<cudaStream_t>(stream)>>>(
