@@ -140,7 +140,7 @@ __device__ __forceinline__ float mx_i2f(int32_t c) { return __fsub_rn(__int_as_f
 constexpr int MXG_WARPS = 8;
 constexpr int MXG_MT = 2, MXG_NT = 4;   // a warp's tile: 2 x 16 rows by 4 x 8 columns
 
-__global__ void __launch_bounds__(MXG_WARPS * 32) k_mx_gemm(const uint8_t* __restrict__ Xq, const uint8_t* __restrict__ sx,
+__global__ void __launch_bounds__(MXG_WARPS * 32, 2) k_mx_gemm(const uint8_t* __restrict__ Xq, const uint8_t* __restrict__ sx,
                                                            const uint8_t* __restrict__ Wq, const uint8_t* __restrict__ sw,
                                                            int M, int N, int K, float* __restrict__ Y, int accumulate) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -159,44 +159,64 @@ __global__ void __launch_bounds__(MXG_WARPS * 32) k_mx_gemm(const uint8_t* __res
         for (int nt = 0; nt < MXG_NT; ++nt)
 #pragma unroll
             for (int q = 0; q < 4; ++q) y[mt][nt][q] = 0.f;
-    for (int b = 0; b < nb; ++b) {
+    // the raw codes and scale bytes of block b + 1 are loaded while block b is
+    // expanded and multiplied (the loads' latency off the dependent chain)
+    uint32_t ra[MXG_MT][4], rb[MXG_NT][2];
+    int ex[MXG_MT][2], ew[MXG_NT][2];
+    auto load_block = [&](int b) {
         const int64_t o = 16 * static_cast<int64_t>(b) + 2 * t4;
-        uint32_t a[MXG_MT][4];
-        int ex[MXG_MT][2];
-        float fx[MXG_MT][2];
 #pragma unroll
         for (int mt = 0; mt < MXG_MT; ++mt) {
             const int r0 = m0 + 16 * mt + g8, r1 = r0 + 8;
             const bool v0 = r0 < M, v1 = r1 < M;
-            a[mt][0] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o)) : 0u;
-            a[mt][1] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o)) : 0u;
-            a[mt][2] = v0 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o + 8)) : 0u;
-            a[mt][3] = v1 ? mx_expand4(*reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o + 8)) : 0u;
+            ra[mt][0] = v0 ? *reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o) : 0u;
+            ra[mt][1] = v1 ? *reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o) : 0u;
+            ra[mt][2] = v0 ? *reinterpret_cast<const uint16_t*>(Xq + r0 * ldq + o + 8) : 0u;
+            ra[mt][3] = v1 ? *reinterpret_cast<const uint16_t*>(Xq + r1 * ldq + o + 8) : 0u;
             ex[mt][0] = v0 ? sx[static_cast<int64_t>(r0) * nb + b] : 0;
             ex[mt][1] = v1 ? sx[static_cast<int64_t>(r1) * nb + b] : 0;
-            fx[mt][0] = mx_half_scale(ex[mt][0]);
-            fx[mt][1] = mx_half_scale(ex[mt][1]);
         }
 #pragma unroll
         for (int nt = 0; nt < MXG_NT; ++nt) {
             const int nB = n0 + 8 * nt + g8, c0 = n0 + 8 * nt + 2 * t4;
             const bool vB = nB < N;
-            const uint32_t b0 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o)) : 0u;
-            const uint32_t b1 = vB ? mx_expand4(*reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o + 8)) : 0u;
-            const int ew0 = c0 < N ? sw[static_cast<int64_t>(c0) * nb + b] : 0;
-            const int ew1 = c0 + 1 < N ? sw[static_cast<int64_t>(c0 + 1) * nb + b] : 0;
-            const float fw0 = mx_half_scale(ew0), fw1 = mx_half_scale(ew1);
+            rb[nt][0] = vB ? *reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o) : 0u;
+            rb[nt][1] = vB ? *reinterpret_cast<const uint16_t*>(Wq + nB * ldq + o + 8) : 0u;
+            ew[nt][0] = c0 < N ? sw[static_cast<int64_t>(c0) * nb + b] : 0;
+            ew[nt][1] = c0 + 1 < N ? sw[static_cast<int64_t>(c0 + 1) * nb + b] : 0;
+        }
+    };
+    load_block(0);
+    for (int b = 0; b < nb; ++b) {
+        uint32_t a[MXG_MT][4], bf[MXG_NT][2];
+        float fx[MXG_MT][2], fw[MXG_NT][2];
+#pragma unroll
+        for (int mt = 0; mt < MXG_MT; ++mt) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[mt][i] = mx_expand4(ra[mt][i]);
+            fx[mt][0] = mx_half_scale(ex[mt][0]);
+            fx[mt][1] = mx_half_scale(ex[mt][1]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < MXG_NT; ++nt) {
+            bf[nt][0] = mx_expand4(rb[nt][0]);
+            bf[nt][1] = mx_expand4(rb[nt][1]);
+            fw[nt][0] = mx_half_scale(ew[nt][0]);
+            fw[nt][1] = mx_half_scale(ew[nt][1]);
+        }
+        if (b + 1 < nb) load_block(b + 1);
+#pragma unroll
+        for (int nt = 0; nt < MXG_NT; ++nt)
 #pragma unroll
             for (int mt = 0; mt < MXG_MT; ++mt) {
                 int32_t c[4] = {0, 0, 0, 0};
-                mx_mma(c, a[mt], b0, b1);
+                mx_mma(c, a[mt], bf[nt][0], bf[nt][1]);
                 // (2x)(2w) / 4 * 2^(bx - 127) * 2^(bw - 127) = c 2^(bx - 128) 2^(bw - 128)
-                y[mt][nt][0] = __fmaf_rn(mx_i2f(c[0]), __fmul_rn(fx[mt][0], fw0), y[mt][nt][0]);
-                y[mt][nt][1] = __fmaf_rn(mx_i2f(c[1]), __fmul_rn(fx[mt][0], fw1), y[mt][nt][1]);
-                y[mt][nt][2] = __fmaf_rn(mx_i2f(c[2]), __fmul_rn(fx[mt][1], fw0), y[mt][nt][2]);
-                y[mt][nt][3] = __fmaf_rn(mx_i2f(c[3]), __fmul_rn(fx[mt][1], fw1), y[mt][nt][3]);
+                y[mt][nt][0] = __fmaf_rn(mx_i2f(c[0]), __fmul_rn(fx[mt][0], fw[nt][0]), y[mt][nt][0]);
+                y[mt][nt][1] = __fmaf_rn(mx_i2f(c[1]), __fmul_rn(fx[mt][0], fw[nt][1]), y[mt][nt][1]);
+                y[mt][nt][2] = __fmaf_rn(mx_i2f(c[2]), __fmul_rn(fx[mt][1], fw[nt][0]), y[mt][nt][2]);
+                y[mt][nt][3] = __fmaf_rn(mx_i2f(c[3]), __fmul_rn(fx[mt][1], fw[nt][1]), y[mt][nt][3]);
             }
-        }
     }
 #pragma unroll
     for (int mt = 0; mt < MXG_MT; ++mt)
