@@ -456,9 +456,10 @@ __global__ void __launch_bounds__(cb::THREADS) k_householder(const void* __restr
     }
 }
 
-// k_householder over 8-value chunks: per row, the dot product (lane-strided
-// chunks, then a warp sum), then y = x - c w chunk by chunk (the row is read
-// again, from L2).  Shared memory: w [K] | red [32].
+// k_householder over 8-value chunks, one CTA per row: the dot product
+// (thread-strided chunks, then a block sum in a fixed order), then
+// y = x - c w chunk by chunk (the row is read again, from L2).  Shared memory:
+// w [K] | red [32].
 __global__ void __launch_bounds__(cb::THREADS) k_householder_v(const void* __restrict__ X, int xt, int M, int K,
                                                               int64_t ldx, const float* __restrict__ v,
                                                               float* __restrict__ Y) {
@@ -475,29 +476,25 @@ __global__ void __launch_bounds__(cb::THREADS) k_householder_v(const void* __res
     }
     const float ww = block_sum(sq, red);
     const float two_over = __fdiv_rn(2.0f, ww);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int m = blockIdx.x * nw + warp; m < M; m += gridDim.x * nw) {
+    // one CTA per row: the row's chunks are spread over all threads, so each
+    // thread walks only K / (8 * blockDim) chunks per pass
+    const int step = 8 * blockDim.x;
+    for (int m = blockIdx.x; m < M; m += gridDim.x) {
         const int64_t base = static_cast<int64_t>(m) * ldx;
         float d = 0.f;
-        for (int k0 = 8 * lane; k0 < K; k0 += 2 * 256) {
-            float f[2][8];
+        for (int k0 = 8 * threadIdx.x; k0 < K; k0 += step) {
+            float f[8];
+            cb_load8(X, xt, base + k0, f);
+            const float4 wa = *reinterpret_cast<const float4*>(w + k0);
+            const float4 wb = *reinterpret_cast<const float4*>(w + k0 + 4);
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int u = 0; u < 2; ++u)
-                if (k0 + 256 * u < K) cb_load8(X, xt, base + k0 + 256 * u, f[u]);
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-                if (k0 + 256 * u < K) {
-                    const float4 wa = *reinterpret_cast<const float4*>(w + k0 + 256 * u);
-                    const float4 wb = *reinterpret_cast<const float4*>(w + k0 + 256 * u + 4);
-                    const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) d = __fmaf_rn(f[u][e], wv[e], d);
-                }
+            for (int e = 0; e < 8; ++e) d = __fmaf_rn(f[e], wv[e], d);
         }
-        d = warp_sum(d);
+        d = block_sum(d, red);
         const float c = __fmul_rn(two_over, d);
         float* yr = Y + static_cast<int64_t>(m) * K;
-        for (int k0 = 8 * lane; k0 < K; k0 += 256) {
+        for (int k0 = 8 * threadIdx.x; k0 < K; k0 += step) {
             float f[8];
             cb_load8(X, xt, base + k0, f);
             const float4 wa = *reinterpret_cast<const float4*>(w + k0);
@@ -733,8 +730,10 @@ extern "C" hq_status hq_calib_householder(const void* X, hq_dtype xt, int64_t M,
     auto kern = vec ? k_householder_v : k_householder;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return HQ_ERR_CUDA;
-    const int64_t want = (M + cb::THREADS / 32 - 1) / (cb::THREADS / 32);
-    const int grid = static_cast<int>(want < 4 * cb_sm_count() ? want : 4 * cb_sm_count());
+    // warp per row (element-wise kernel) or CTA per row (16-byte kernel)
+    const int64_t want = vec ? M : (M + cb::THREADS / 32 - 1) / (cb::THREADS / 32);
+    const int64_t cap = (vec ? 8 : 4) * static_cast<int64_t>(cb_sm_count());
+    const int grid = static_cast<int>(want < cap ? want : cap);
     kern<<<grid, cb::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
         X, xt, static_cast<int>(M), static_cast<int>(K), ld_x, v, Y);
     return cb_launched();
