@@ -41,8 +41,10 @@ def test_extreme_tokens_bit_exact(name, S, L):
     no_device_error()
 
 
-def test_extreme_tokens_ties_nan_and_fp32_strided():
-    S, L, K = 4, 6, 300
+# K = 300: element-wise kernel; K = 304: the two-launch 16-byte path
+@pytest.mark.parametrize("K", [300, 304])
+def test_extreme_tokens_ties_nan_and_fp32_strided(K):
+    S, L = 4, 6
     rng = np.random.default_rng(9)
     Xf = rng.standard_normal((S * L, K + 20)).astype(np.float32)
     Xf[1, 5] = 50.0

@@ -35,8 +35,8 @@
 //                 perm[position] = channel.
 //  k_flatten      s[k] = xmax[k]^alpha / wmax[k]^(1 - alpha).
 //  k_permute      Y[m][j] = X[m][perm[j]] (divided or multiplied by s[perm[j]]).
-// k_extreme_v, k_householder_v, k_col_absmax_v and k_permute_rows are the same
-// operations with 16-byte loads, taken when X is 16-byte aligned, its row stride
+// k_token_linf + k_extreme_pick (L <= K), k_extreme_v, k_householder_v,
+// k_col_absmax_v and k_permute_rows are the same operations with 16-byte loads, taken when X is 16-byte aligned, its row stride
 // a multiple of 16 bytes and K a multiple of 8.
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -200,6 +200,83 @@ __global__ void __launch_bounds__(cb::EXT_THREADS) k_extreme_v(const void* __res
         cb_load8(X, xt, src + k0, f);
         *reinterpret_cast<float4*>(dst + k0) = make_float4(f[0], f[1], f[2], f[3]);
         *reinterpret_cast<float4*>(dst + k0 + 4) = make_float4(f[4], f[5], f[6], f[7]);
+    }
+}
+
+// The extreme tokens in two launches when L <= K (the usual case): k_token_linf
+// gives every token its own warp (max |x| with 16-byte loads) and parks the
+// results of sequence s in T's row s; k_extreme_pick (one CTA per sequence)
+// reads them, takes the first maximum, and only then overwrites the row with
+// the chosen token.
+__global__ void __launch_bounds__(cb::THREADS) k_token_linf(const void* __restrict__ X, int xt, int S, int L, int K,
+                                                           int64_t ldx, float* __restrict__ T) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (t >= static_cast<int64_t>(S) * L) return;   // whole warps
+    const int64_t base = t * ldx;
+    float m = 0.f;
+    for (int k0 = 8 * lane; k0 < K; k0 += 4 * 256) {
+        float f[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (k0 + 256 * u < K) cb_load8(X, xt, base + k0 + 256 * u, f[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (k0 + 256 * u < K)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[u][e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const int64_t s = t / L, l = t - s * L;
+    if (lane == 0) T[s * K + l] = m;
+}
+
+__global__ void __launch_bounds__(cb::EXT_THREADS) k_extreme_pick(const void* __restrict__ X, int xt, int L, int K,
+                                                                 int64_t ldx, int32_t* __restrict__ tok,
+                                                                 float* __restrict__ T) {
+    __shared__ float bv[cb::EXT_THREADS / 32];
+    __shared__ int bi[cb::EXT_THREADS / 32];
+    const int s = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    float* row = T + static_cast<int64_t>(s) * K;
+    float best = -1.f;
+    int besti = 0;
+    for (int l = threadIdx.x; l < L; l += blockDim.x) {   // increasing l per thread: strict > keeps the first
+        const float m = row[l];
+        if (m > best) {
+            best = m;
+            besti = l;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, besti, o);
+        if (ob > best || (ob == best && oi < besti)) {
+            best = ob;
+            besti = oi;
+        }
+    }
+    if (lane == 0) {
+        bv[warp] = best;
+        bi[warp] = besti;
+    }
+    __syncthreads();   // every read of the row is done before it is overwritten
+    float b = bv[0];
+    int bidx = bi[0];
+    for (int w = 1; w < nw; ++w)
+        if (bv[w] > b || (bv[w] == b && bi[w] < bidx)) {
+            b = bv[w];
+            bidx = bi[w];
+        }
+    if (threadIdx.x == 0) tok[s] = bidx;
+    const int64_t src = (static_cast<int64_t>(s) * L + bidx) * ldx;
+    for (int k0 = 8 * threadIdx.x; k0 < K; k0 += 8 * blockDim.x) {
+        float f[8];
+        cb_load8(X, xt, src + k0, f);
+        *reinterpret_cast<float4*>(row + k0) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(row + k0 + 4) = make_float4(f[4], f[5], f[6], f[7]);
     }
 }
 
@@ -672,6 +749,18 @@ extern "C" hq_status hq_calib_extreme_tokens(const void* X, hq_dtype xt, int64_t
     if (S > INT32_MAX || L > INT32_MAX || K > INT32_MAX) return HQ_ERR_UNSUPPORTED;
     if (S == 0) return HQ_OK;
     if (!X || !tok || !T) return HQ_ERR_ARG;
+    if (cb_vec(X, xt, K, ld_x) && cb_al16(T) && L <= K) {
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const int64_t warps = S * L;
+        const int64_t grid = (warps + cb::THREADS / 32 - 1) / (cb::THREADS / 32);
+        if (grid > INT32_MAX) return HQ_ERR_UNSUPPORTED;
+        k_token_linf<<<static_cast<unsigned>(grid), cb::THREADS, 0, st>>>(X, xt, static_cast<int>(S),
+                                                                          static_cast<int>(L), static_cast<int>(K),
+                                                                          ld_x, T);
+        k_extreme_pick<<<static_cast<unsigned>(S), cb::EXT_THREADS, 0, st>>>(X, xt, static_cast<int>(L),
+                                                                             static_cast<int>(K), ld_x, tok, T);
+        return cb_launched();
+    }
     if (cb_vec(X, xt, K, ld_x) && cb_al16(T))
         k_extreme_v<<<static_cast<unsigned>(S), cb::EXT_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
             X, xt, static_cast<int>(L), static_cast<int>(K), ld_x, tok, T);
