@@ -379,7 +379,8 @@ hq_status hq_debug_wait_probe(uint64_t limit_ns, void* stream);
  * tok[s], and its values widened to fp32, T[s][0..K).
  *  X    device, [S*L][ld_x] calibration activations
  *  tok  device, [S] int32 (output)
- *  T    device, [S][K] fp32 (output), contiguous
+ *  T    device, [S][K] fp32 (output), contiguous; while the call runs, row s
+ *       may first hold the per-token maxima of sequence s (when L <= K)
  * Errors: HQ_ERR_ARG (S < 0, L <= 0, K <= 0, ld_x < K, bad dtype, NULL with
  * S > 0), HQ_ERR_UNSUPPORTED (a size above INT32_MAX).  S == 0 is a no-op.
  */
